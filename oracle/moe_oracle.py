@@ -1,0 +1,385 @@
+"""fp64 CPU oracle of the sparse MoE FFN layer forward.
+
+TEST INFRASTRUCTURE.  Only tests, the smoke check and the benchmark's
+CPU-baseline leg may import this module.  It shares no code with the CUDA
+library and imports nothing from it.
+
+Sources (reference pages, cited by page title and section):
+  [DSMoE]  "論文解説: DeepSeekMoE — 細粒度エキスパート分割と共有エキスパートによる
+           MoE効率化" (0h-n0.github.io): §共有エキスパート機構 (layer output h_t),
+           §ルーティングとバランス損失 (gate g_j, softmax s_j, balance loss),
+           §アルゴリズム (the reference nn.Module: router Linear without bias,
+           expert = Linear -> SiLU -> Linear with biases, top-K, renormalise),
+           §実装のポイント (alpha = 0.01).
+  [TopK]   "Sparse MoE Top-Kルーティング" (jisaku.com glossary):
+           §ルーティングの仕組み (top-K, gate weights, weighted sum),
+           §解決策2 エキスパートキャパシティファクター and FAQ Q2 (capacity,
+           overflow tokens dropped).
+  [EP]     "エキスパート並列（Expert Parallelism）" (jisaku.com glossary):
+           §推論フロー (route tokens to their expert and back).
+  [DeepEP] "DeepSeek DeepEP" (blogs.novita.ai): §DeepEP とは item 5 and
+           §DeepEP の性能 (FP8 dispatch, BF16 combine).
+
+Readings where the pages leave a step open (each is also listed in the design
+notes of the repository):
+  * selection uses the logits (softmax is monotone); ties go to the lower
+    expert index; slot order is descending logit, then ascending index;
+  * capacity C = ceil(cf * T * K / N_r); within an expert, slots keep token
+    order and the first C are kept (earliest token first); a dropped slot adds
+    nothing and the other gates are not renormalised;
+  * f_j uses pre-drop counts over T*K slots; P_j is the mean of the full
+    softmax (including any logit bias) over all T tokens;
+  * FP8: activations are quantised per row per 128 columns and weights per
+    128x128 block, each with the smallest power-of-two scale 2^k such that
+    amax / 2^k <= 448 (scale 1 for an all-zero block), codes by
+    round-to-nearest-even with saturation to +-448; the hidden activation h is
+    re-quantised the same way before the second linear layer, expert outputs
+    are rounded to bf16 before the combine and the layer output is rounded to
+    bf16 at the end.  In bf16 and fp32 workloads nothing is rounded in between.
+
+Parity pins (tests/test_oracle_pins.py): gates sum to one; counts sum to T*K;
+the dispatch permutation is a bijection with rows in token order; N_r = K = 1
+reduces to a dense FFN checked against torch's CPU linear/SiLU; the
+dense masked form of the reference module (every expert on every token, then
+masked) gives the same output; brute-force top-K over all K-subsets on tiny
+inputs; the C(8,2) = 28 and C(16,2) = 120 selected-set counts; active-parameter
+fraction K/N_r; balance loss closed forms (uniform routing gives alpha, a
+collapsed router gives alpha * N_r); the first C tokens kept under capacity;
+the e4m3 and bf16 rounding against torch's conversions.  The expert FFN
+arithmetic beyond these is pinned only through the dense limit.
+"""
+from __future__ import annotations
+
+import math
+from fractions import Fraction
+from typing import Dict, Optional
+
+import numpy as np
+
+__all__ = [
+    "E4M3_MAX", "e4m3_decode", "e4m3_round", "pow2_scale", "quantize_rows_1x128",
+    "dequant_rows_1x128", "dequant_blocks_128x128", "bf16_round",
+    "router_logits", "softmax", "topk_select", "gates_of", "capacity_of",
+    "dispatch_plan", "silu", "expert_ffn", "balance_stats", "topk_gap",
+    "route", "layer_forward", "to_f64",
+]
+
+E4M3_MAX = 448.0
+_QBLOCK = 128
+
+
+# ----------------------------------------------------------------------------
+# Number formats ([DeepEP] FP8 dispatch / BF16 combine; format definitions:
+# e4m3 = 1 sign, 4 exponent bits with bias 7, 3 mantissa bits, subnormals,
+# no infinities, S.1111.111 is NaN; bf16 = the upper half of an IEEE fp32)
+# ----------------------------------------------------------------------------
+
+def e4m3_decode(codes: np.ndarray) -> np.ndarray:
+    """uint8 e4m3 codes -> fp64 values (NaN for S.1111.111)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((e == 15) & ((c & 0x7) == 7), np.nan, mag)
+    return sign * mag
+
+
+_E4M3_POS = e4m3_decode(np.arange(127, dtype=np.uint8))   # codes 0x00..0x7E, ascending
+
+
+def e4m3_round(v: np.ndarray) -> np.ndarray:
+    """Round fp64 values to e4m3 codes: nearest representable value, ties to
+    the even code, magnitudes beyond 448 saturate to 448."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.minimum(np.abs(v), E4M3_MAX)
+    hi = np.searchsorted(_E4M3_POS, a, side="left")          # first table value >= a
+    hi = np.minimum(hi, len(_E4M3_POS) - 1)
+    lo = np.maximum(hi - 1, 0)
+    d_hi = _E4M3_POS[hi] - a
+    d_lo = a - _E4M3_POS[lo]
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo).astype(np.uint8)
+    code = np.where(np.signbit(v) & (code != 0), code | 0x80, code)
+    return code.astype(np.uint8)
+
+
+def pow2_scale(amax: np.ndarray) -> np.ndarray:
+    """Smallest power of two 2^k with amax / 2^k <= 448; 1 where amax == 0."""
+    amax = np.asarray(amax, dtype=np.float64)
+    out = np.ones_like(amax)
+    nz = amax > 0
+    k = np.ceil(np.log2(amax[nz] / E4M3_MAX))
+    s = np.exp2(k)
+    # guard the float log2 against an off-by-one at exact powers of two
+    s = np.where(amax[nz] / s > E4M3_MAX, s * 2.0, s)
+    s = np.where(amax[nz] / (s / 2.0) <= E4M3_MAX, s / 2.0, s)
+    out[nz] = s
+    return out
+
+
+def quantize_rows_1x128(v: np.ndarray):
+    """(rows, cols) fp64 -> e4m3 codes (rows, cols) and fp64 scales
+    (rows, cols/128): one scale per row per 128 columns."""
+    rows, cols = v.shape
+    assert cols % _QBLOCK == 0
+    vb = v.reshape(rows, cols // _QBLOCK, _QBLOCK)
+    scale = pow2_scale(np.abs(vb).max(axis=2))
+    codes = e4m3_round(vb / scale[:, :, None])     # division by 2^k is exact
+    return codes.reshape(rows, cols), scale
+
+
+def dequant_rows_1x128(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    rows, cols = codes.shape
+    vals = e4m3_decode(codes).reshape(rows, cols // _QBLOCK, _QBLOCK)
+    return (vals * np.asarray(scales, np.float64)[:, :, None]).reshape(rows, cols)
+
+
+def dequant_blocks_128x128(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    rows, cols = codes.shape
+    vals = e4m3_decode(codes).reshape(rows // _QBLOCK, _QBLOCK, cols // _QBLOCK, _QBLOCK)
+    return (vals * np.asarray(scales, np.float64)[:, None, :, None]).reshape(rows, cols)
+
+
+def bf16_round(v: np.ndarray) -> np.ndarray:
+    """Round fp64 values to the nearest bf16 value (ties to even), returned as
+    fp64.  bf16 keeps 8 significant bits; below 2^-126 the spacing is 2^-133."""
+    v = np.asarray(v, dtype=np.float64)
+    _, e = np.frexp(v)                      # v = m * 2^e, |m| in [0.5, 1)
+    quantum = np.exp2(np.maximum(e - 8, -133).astype(np.float64))
+    return np.rint(v / quantum) * quantum   # rint rounds halves to even
+
+
+def to_f64(a) -> np.ndarray:
+    """torch tensor / numpy array of fp32, bf16 or fp64 values -> fp64 numpy."""
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            return a.detach().to("cpu", torch.float64).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(a, dtype=np.float64)
+
+
+# ----------------------------------------------------------------------------
+# Router ([DSMoE] §ルーティングとバランス損失: s_j = softmax(W_r x)_j,
+# g_j = s_j / sum_{k in TopK} s_k; [TopK] §ルーティングの仕組み)
+# ----------------------------------------------------------------------------
+
+def router_logits(x: np.ndarray, W_r: np.ndarray, logit_bias: Optional[np.ndarray] = None) -> np.ndarray:
+    """l[t, j] = sum_i x[t, i] W_r[j, i] (+ b_j), fp64.  The router is a linear
+    map without bias ([DSMoE] §アルゴリズム); b_j is the decode workload's
+    per-expert logit bias."""
+    l = np.asarray(x, np.float64) @ np.asarray(W_r, np.float64).T
+    if logit_bias is not None:
+        l = l + np.asarray(logit_bias, np.float64)[None, :]
+    return l
+
+
+def softmax(l: np.ndarray) -> np.ndarray:
+    """Softmax over all routed experts of each token."""
+    z = l - l.max(axis=1, keepdims=True)
+    e = np.exp(z)
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def topk_select(l: np.ndarray, K: int) -> np.ndarray:
+    """Indices of the K largest logits per token, in slot order: descending
+    logit, equal logits by ascending expert index (the lower index wins a tie).
+    A stable sort of -l keeps equal keys in index order."""
+    order = np.argsort(-np.asarray(l, np.float64), axis=1, kind="stable")
+    return order[:, :K].astype(np.int32)
+
+
+def gates_of(s: np.ndarray, idx: np.ndarray) -> np.ndarray:
+    """g[t, k] = s[t, idx[t, k]] / sum_k' s[t, idx[t, k']]."""
+    sel = np.take_along_axis(s, idx.astype(np.int64), axis=1)
+    return sel / sel.sum(axis=1, keepdims=True)
+
+
+def topk_gap(l: np.ndarray, K: int) -> np.ndarray:
+    """l_(K) - l_(K+1) of each token's descending logits (inf when K = N_r)."""
+    srt = -np.sort(-np.asarray(l, np.float64), axis=1)
+    if K >= srt.shape[1]:
+        return np.full(srt.shape[0], np.inf)
+    return srt[:, K - 1] - srt[:, K]
+
+
+# ----------------------------------------------------------------------------
+# Dispatch plan ([EP] §推論フロー: tokens go to the expert that serves them;
+# [TopK] §解決策2 / FAQ Q2: per-expert capacity per batch, overflow dropped)
+# ----------------------------------------------------------------------------
+
+def capacity_of(T: int, K: int, N_r: int, cf: float) -> Optional[int]:
+    """C = ceil(cf * T * K / N_r), evaluated exactly on the fp32 value of cf;
+    None when cf <= 0 (no limit)."""
+    cf32 = float(np.float32(cf))
+    if cf32 <= 0:
+        return None
+    return int(math.ceil(Fraction(cf32) * T * K / N_r))
+
+
+def dispatch_plan(idx: np.ndarray, N_r: int, C: Optional[int]) -> Dict[str, np.ndarray]:
+    """Counts, kept counts, segment offsets and the slot<->row permutation.
+
+    Slots (t, k) of expert j are ranked in ascending token order; slot of rank
+    r is kept iff r < C.  Kept slots of expert j occupy rows
+    offsets[j] .. offsets[j] + kept[j] - 1 in token order.
+    """
+    T, K = idx.shape
+    counts = np.zeros(N_r, np.int64)
+    rank = np.full((T, K), -1, np.int64)
+    for t in range(T):
+        for k in range(K):
+            j = int(idx[t, k])
+            rank[t, k] = counts[j]
+            counts[j] += 1
+    kept = counts.copy() if C is None else np.minimum(counts, C)
+    offsets = np.zeros(N_r + 1, np.int64)
+    offsets[1:] = np.cumsum(kept)
+    R = int(offsets[-1])
+    slot_row = np.full((T, K), -1, np.int64)
+    row_slot = np.full(R, -1, np.int64)
+    for t in range(T):
+        for k in range(K):
+            j = int(idx[t, k])
+            if C is None or rank[t, k] < C:
+                r = int(offsets[j] + rank[t, k])
+                slot_row[t, k] = r
+                row_slot[r] = t * K + k
+    return {"counts": counts, "kept": kept, "offsets": offsets,
+            "slot_row": slot_row, "row_slot": row_slot, "R": R}
+
+
+# ----------------------------------------------------------------------------
+# Expert FFN ([DSMoE] §アルゴリズム: Linear(d, d_ff) + bias -> SiLU ->
+# Linear(d_ff, d) + bias)
+# ----------------------------------------------------------------------------
+
+def silu(z: np.ndarray) -> np.ndarray:
+    return z / (1.0 + np.exp(-z))
+
+
+def expert_ffn(xr: np.ndarray, W1: np.ndarray, b1: np.ndarray, W2: np.ndarray,
+               b2: np.ndarray, fp8_hidden: bool = False) -> np.ndarray:
+    """y = W2 SiLU(W1 x + b1) + b2 for each row of xr, fp64.  With fp8_hidden
+    the hidden activation is quantised per row per 128 columns first."""
+    h = silu(xr @ W1.T + b1[None, :])
+    if fp8_hidden:
+        codes, sc = quantize_rows_1x128(h)
+        h = dequant_rows_1x128(codes, sc)
+    return h @ W2.T + b2[None, :]
+
+
+# ----------------------------------------------------------------------------
+# Balance statistics ([DSMoE] §ルーティングとバランス損失:
+# L = alpha * N_r * sum_j f_j P_j)
+# ----------------------------------------------------------------------------
+
+def balance_stats(counts: np.ndarray, s: np.ndarray, K: int, alpha: float):
+    T, N_r = s.shape
+    f = np.asarray(counts, np.float64) / float(T * K)
+    P = s.mean(axis=0)
+    L = alpha * N_r * float(np.sum(f * P))
+    return f, P, L
+
+
+# ----------------------------------------------------------------------------
+# Whole layer ([DSMoE] §共有エキスパート機構: h_t = sum_i E_s,i(x_t)
+# + sum_{j in TopK} g_j(x_t) E_r,j(x_t))
+# ----------------------------------------------------------------------------
+
+def route(shape, inputs, logits: Optional[np.ndarray] = None):
+    """Router, top-K, gates, plan and balance statistics for all T tokens.
+
+    `logits`, when given, replaces the oracle's own fp64 logits as the
+    selection keys (used to check the product's routing bit-exactly on its own
+    fp32 logits); s and P still come from the oracle's fp64 logits."""
+    x = to_f64(inputs["x"])
+    lb = inputs.get("logit_bias")
+    l64 = router_logits(x, to_f64(inputs["W_r"]), None if lb is None else to_f64(lb))
+    s = softmax(l64)
+    keys = l64 if logits is None else np.asarray(logits, np.float64)
+    idx = topk_select(keys, shape.top_k)
+    g = gates_of(s, idx)
+    C = capacity_of(shape.T, shape.top_k, shape.n_routed, shape.capacity_factor)
+    plan = dispatch_plan(idx, shape.n_routed, C)
+    f, P, L = balance_stats(plan["counts"], s, shape.top_k, shape.alpha)
+    return {"logits": l64, "s": s, "idx": idx, "gates": g, "C": C, "plan": plan,
+            "f": f, "P": P, "loss": L, "gap": topk_gap(l64, shape.top_k)}
+
+
+def _expert_weights(inputs, prefix: str, e: int, fp8: bool):
+    """fp64 (W1, b1, W2, b2) of routed (prefix 'W') or shared (prefix 'Ws')
+    expert e."""
+    b = "b" if prefix == "W" else "bs"
+    if fp8:
+        W1 = dequant_blocks_128x128(_np_u8(inputs[prefix + "1"][e]), to_f64(inputs[prefix + "1_scales"][e]))
+        W2 = dequant_blocks_128x128(_np_u8(inputs[prefix + "2"][e]), to_f64(inputs[prefix + "2_scales"][e]))
+    else:
+        W1 = to_f64(inputs[prefix + "1"][e])
+        W2 = to_f64(inputs[prefix + "2"][e])
+    return W1, to_f64(inputs[b + "1"][e]), W2, to_f64(inputs[b + "2"][e])
+
+
+def _np_u8(a) -> np.ndarray:
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            return a.detach().to("cpu").view(torch.uint8).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(a, np.uint8)
+
+
+def layer_forward(shape, inputs, tokens: Optional[np.ndarray] = None,
+                  routing: Optional[dict] = None) -> dict:
+    """The layer output for `tokens` (default: all T), plus the routing.
+
+    Returns {"out": (len(tokens), d) fp64, "tokens", "routing"}.  Each token's
+    output is sum_k g[t, k] * E_{idx[t, k]}(x_t) over its kept slots in
+    ascending k, then the shared experts in ascending order.  In FP8 workloads
+    x is quantised per row per 128 columns before the experts, h is
+    re-quantised, each expert output is rounded to bf16 and the sum is rounded
+    to bf16 at the end.
+    """
+    fp8 = shape.dtype == 2
+    rt = routing if routing is not None else route(shape, inputs)
+    T, K = shape.T, shape.top_k
+    tokens = np.arange(T) if tokens is None else np.asarray(tokens, np.int64)
+    x = to_f64(inputs["x"])[tokens]
+    if fp8:
+        xc, xs = quantize_rows_1x128(x)
+        xin = dequant_rows_1x128(xc, xs)
+    else:
+        xin = x
+    slot_row = rt["plan"]["slot_row"]
+    # expert outputs of every kept slot of the requested tokens, one expert at a time
+    by_expert: Dict[int, list] = {}
+    for i, t in enumerate(tokens):
+        for k in range(K):
+            if slot_row[t, k] >= 0:
+                by_expert.setdefault(int(rt["idx"][t, k]), []).append((i, k))
+    y_slot: Dict[tuple, np.ndarray] = {}
+    for e in sorted(by_expert):
+        W1, b1, W2, b2 = _expert_weights(inputs, "W", e, fp8)
+        rows = by_expert[e]
+        y = expert_ffn(xin[np.array([i for i, _ in rows])], W1, b1, W2, b2, fp8_hidden=fp8)
+        if fp8:
+            y = bf16_round(y)
+        for n, key in enumerate(rows):
+            y_slot[key] = y[n]
+    out = np.zeros((len(tokens), shape.d_model), np.float64)
+    for i, t in enumerate(tokens):
+        for k in range(K):
+            if (i, k) in y_slot:
+                out[i] += rt["gates"][t, k] * y_slot[(i, k)]
+    for s_i in range(shape.n_shared):
+        W1, b1, W2, b2 = _expert_weights(inputs, "Ws", s_i, fp8)
+        y = expert_ffn(xin, W1, b1, W2, b2, fp8_hidden=fp8)
+        if fp8:
+            y = bf16_round(y)
+        out += y
+    if fp8:
+        out = bf16_round(out)
+    return {"out": out, "tokens": tokens, "routing": rt}
