@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""Benchmark of the sparse MoE FFN layer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2] [--impl ours|reference]
+
+A step is one pass of the whole layer (router, dispatch, expert FFN grouped
+GEMMs, combine, balance statistics) over one batch of seeded synthetic input
+that is already resident in HBM.  The default workload is the
+Mixtral-8x7B-shaped bf16 layer (T=4096, d=4096, 8 experts, top-2,
+d_ff=14336).  Each timed step is bracketed by CUDA events on the launching
+stream, with a 256 MiB write between steps to flush L2.  Under torchrun each
+rank runs an independent replica (the layer forward has no cross-GPU
+exchange); the time is the max over ranks and the value counts the tokens of
+all ranks.
+
+One JSON line on rank 0: tokens/s plus the grouped-GEMM roofline, the CPU
+oracle baseline (rank 0, N=1), an end-to-end figure through the public API
+with host buffers, and the SM clocks sampled during the timed region.
+
+--impl reference times the CPU oracle (the reference implementation of this
+repository: a plain fp64 restatement of the pages) on bounded token samples
+of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s; grouped-GEMM TFLOP/s and HBM GB/s as % of B200 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+CPU_SAMPLE = {1: 64, 2: 256, 3: 256, 4: 64, 5: 128}     # oracle tokens per baseline sample
+REF_SAMPLE = {1: 64, 2: 32, 3: 64, 4: 16, 5: 32}         # oracle tokens per reference step
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(sh, seed, parallelism):
+    return {"workload": sh.name, "T": sh.T, "d_model": sh.d_model, "n_routed": sh.n_routed,
+            "top_k": sh.top_k, "d_ff": sh.d_ff, "n_shared": sh.n_shared, "d_ff_shared": sh.d_ff_shared,
+            "capacity_factor": sh.capacity_factor, "seed": seed, "parallelism": parallelism,
+            "l2": "flushed between timed steps (256 MiB write)"}
+
+
+def dtype_name(sh):
+    return {0: "f32", 1: "bf16", 2: "fp8-e4m3 (bf16 combine)"}[sh.dtype]
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"moe_clocks_{os.getpid()}.csv")
+        self.marks = []
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=timestamp," + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def mark(self):
+        self.marks.append(time.time())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[5:9]))
+            except Exception:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        t0, t1 = (self.marks[0], self.marks[-1]) if len(self.marks) >= 2 else (0, 1e18)
+        sel = [r for r in rows if t0 - 1 <= r[0] <= t1 + 1] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in sel for i in range(4) if r[3][i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[1] for r in sel), "sm_max_mhz": max(r[2] for r in sel),
+                "reasons": reasons, "samples": len(sel)}
+
+
+# ----------------------------------------------------------------------------- oracle timing
+
+def oracle_inputs_on_host(inp):
+    return {k: (None if v is None else v.detach().cpu()) for k, v in inp.items()}
+
+
+def time_oracle(sh, host_inp, n_tokens, seed):
+    import numpy as np
+    import oracle as O
+    rng = np.random.default_rng(seed)
+    toks = np.sort(rng.choice(sh.T, size=min(n_tokens, sh.T), replace=False))
+    t0 = time.perf_counter()
+    O.layer_forward(sh, host_inp, tokens=toks)
+    dt = time.perf_counter() - t0
+    return len(toks), dt
+
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def algorithmic_ffn(sh, kept_sum):
+    """FLOPs and bytes of the expert FFN stage (both grouped GEMMs) for one
+    step: real rows only.  Bytes: weights and biases of every expert that has
+    rows, the dispatched activations read, the hidden activations written and
+    read, the expert outputs written."""
+    d, dff, S, T = sh.d_model, sh.d_ff, sh.n_shared, sh.T
+    flops = 4.0 * d * dff * kept_sum + 4.0 * d * sh.d_ff_shared * S * T
+    return flops
+
+
+def ffn_bytes(sh, kept):
+    d, dff, S, T, dfs = sh.d_model, sh.d_ff, sh.n_shared, sh.T, sh.d_ff_shared
+    wb = {0: 4, 1: 2, 2: 1}[sh.dtype]
+    ab = {0: 4, 1: 2, 2: 1}[sh.dtype]
+    ob = 4 if sh.dtype == 0 else 2
+    touched = int((kept > 0).sum())
+    R = int(kept.sum())
+    w = touched * (2 * d * dff * wb + 4 * (dff + d)) + S * (2 * d * dfs * wb + 4 * (dfs + d))
+    if sh.dtype == 2:
+        w += touched * 2 * (d // 128) * (dff // 128) * 4 + S * 2 * (d // 128) * (dfs // 128) * 4
+    act = (R + S * T) * d * ab + 2 * (R * dff + S * T * dfs) * ab + (R + S * T) * d * ob
+    return float(w + act), touched
+
+
+def traffic_from_profile(kernel_src_hash, cid):
+    """dram bytes per FFN launch pair from the committed ncu summary, valid only
+    while the kernel source is unchanged since the capture."""
+    p = os.path.join(ROOT, "profiles", "grouped_ffn_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        e = d.get(str(cid))
+        if e and e.get("ffn_tc_sha1") == kernel_src_hash:
+            return e.get("dram_bytes_per_step")
+    except Exception:
+        return None
+    return None
+
+
+def ffn_src_hash():
+    src = os.path.join(ROOT, "sparse_mixture_experts_20_b200", "csrc", "ffn_tc.cu")
+    return hashlib.sha1(open(src, "rb").read()).hexdigest()
+
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import sparse_mixture_experts_20_b200 as M
+    from synthetic import CONFIGS, make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    sh = CONFIGS[args.config]
+    M.lib()
+    inp = make_inputs(sh, seed=args.seed + rank, device=dev)
+    cfg = M.make_config(sh)
+    T, K, E, d = sh.T, sh.top_k, sh.n_routed, sh.d_model
+    cap, r_cap, x_rows, y_rows = M.moe_buffer_rows(cfg)
+    fp8 = sh.dtype == 2
+    act = torch.float32 if sh.dtype == 0 else torch.bfloat16
+    ws = torch.empty(M.moe_workspace_size(cfg), dtype=torch.uint8, device=dev)
+    M.moe_workspace_init(cfg, ws)
+    i32 = dict(dtype=torch.int32, device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    b = {
+        "topk_idx": torch.empty((T, K), **i32), "gates": torch.empty((T, K), **f32),
+        "counts": torch.empty(E, **i32), "kept": torch.empty(E, **i32), "offsets": torch.empty(E + 1, **i32),
+        "slot_row": torch.empty((T, K), **i32), "row_slot": torch.empty(max(r_cap, 1), **i32),
+        "x_disp": torch.empty((x_rows, d), dtype=torch.uint8 if fp8 else act, device=dev),
+        "x_disp_scales": torch.empty((x_rows, d // 128), **f32) if fp8 else None,
+        "y": torch.empty((y_rows, d), dtype=act, device=dev), "out": torch.empty((T, d), dtype=act, device=dev),
+        "f": torch.empty(E, **f32), "P": torch.empty(E, **f32), "loss": torch.empty(1, **f32),
+    }
+    g = inp.get
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    n_stage = 5
+    launches_per_step = 1 + 3 + 2 + 1 + 1
+
+    def step(ev):
+        ev[0].record(stream)
+        M.moe_route(cfg, inp["x"], g("W_r"), g("logit_bias"), b["topk_idx"], b["gates"], None, ws)
+        ev[1].record(stream)
+        M.moe_dispatch(cfg, inp["x"], b["topk_idx"], b["counts"], b["kept"], b["offsets"], b["slot_row"],
+                       b["row_slot"], b["x_disp"], b["x_disp_scales"], ws)
+        ev[2].record(stream)
+        M.moe_expert_ffn(cfg, inp["x"], b["x_disp"], b["x_disp_scales"], b["offsets"], g("W1"), g("W1_scales"),
+                         g("b1"), g("W2"), g("W2_scales"), g("b2"), g("Ws1"), g("Ws1_scales"), g("bs1"),
+                         g("Ws2"), g("Ws2_scales"), g("bs2"), b["y"], ws)
+        ev[3].record(stream)
+        M.moe_combine(cfg, b["y"], b["gates"], b["slot_row"], b["out"])
+        ev[4].record(stream)
+        M.moe_balance_stats(cfg, b["counts"], ws, b["f"], b["P"], b["loss"])
+        ev[5].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    for _ in range(args.warmup):
+        flush.zero_()
+        step([torch.cuda.Event(enable_timing=True) for _ in range(n_stage + 1)])
+    torch.cuda.synchronize(dev)
+    assert M.moe_get_device_status(cfg, ws) == 0, "device status after warm-up"
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_stage + 1)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler.mark()
+    for k in range(args.steps):
+        flush.zero_()
+        step(evs[k])
+    torch.cuda.synchronize(dev)
+    sampler.mark()
+    barrier()
+    stage_ms = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(n_stage)]
+                         for k in range(args.steps)])
+    step_ms = stage_ms.sum(axis=1)
+    total_ms = float(step_ms.sum())
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    kept = b["kept"].cpu().numpy()
+    counts = b["counts"].cpu().numpy()
+    status = M.moe_get_device_status(cfg, ws)
+
+    # ---- end to end through the public API: pinned host x in, out + loss back
+    layer = M.MoELayer(cfg, inp, device=dev)
+    x_h = inp["x"].cpu().pin_memory()
+    out_h = torch.empty((T, d), dtype=act).pin_memory()
+    loss_h = torch.empty(1, dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(inp["x"])
+    for _ in range(max(1, min(args.warmup, 3))):
+        x_dev.copy_(x_h, non_blocking=True)
+        layer.forward(x_dev)
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    for k in range(args.steps):
+        flush.zero_()
+        e2e_ev[k][0].record(stream)
+        x_dev.copy_(x_h, non_blocking=True)
+        out, f, P, loss = layer.forward(x_dev)
+        out_h.copy_(out, non_blocking=True)
+        loss_h.copy_(loss, non_blocking=True)
+        e2e_ev[k][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = float(sum(a.elapsed_time(c) for a, c in e2e_ev))
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    clocks = sampler.stop()
+
+    peaks, peak_src = load_peaks()
+    ffn_ms = float(stage_ms[:, 2].mean())
+    flops = algorithmic_ffn(sh, int(kept.sum()))
+    fbytes, touched = ffn_bytes(sh, kept)
+    tens_peak = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
+    t_tensor = flops / (tens_peak * 1e12)
+    t_hbm = fbytes / (peaks["hbm_gbs"] * 1e9)
+    if t_tensor >= t_hbm:
+        ach = flops / (ffn_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(ach, 1), "peak": tens_peak, "unit": "TFLOP/s",
+                "frac": round(ach / tens_peak, 4)}
+    else:
+        ach = fbytes / (ffn_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(ach / peaks["hbm_gbs"], 4)}
+    roof["kernel"] = "grouped_ffn_tc_kernel (first + second layer launches, per step)"
+    roof["peak_source"] = (f"{peak_src} ({'bf16 burst x2 nominal fp8/bf16 ratio' if fp8 else 'bf16 burst'})"
+                           if roof["bound"] == "tensor" else f"{peak_src} HBM copy")
+    roof["traffic"] = traffic_from_profile(ffn_src_hash(), args.config)
+    roof["algorithmic"] = {"flops": flops, "bytes": fbytes, "experts_touched": touched}
+
+    n_tok = T * world * args.steps
+    value = n_tok / (total_ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype_name(sh),
+        "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights, N(0,0.01) biases)",
+        "config": workload_config(sh, args.seed, "replicas" if world > 1 else "single"),
+        "impl": "ours",
+        "stages_ms": {n: round(float(stage_ms[:, i].mean()), 4) for i, n in
+                      enumerate(["route", "dispatch", "expert_ffn", "combine", "balance"])},
+        "grouped_gemm_tflops": round(flops / (ffn_ms * 1e-3) / 1e12, 1),
+        "roofline": roof,
+        "e2e": {"value": round(T * world * args.steps / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(inp["x"].numel() * inp["x"].element_size()),
+                "d2h_bytes_per_step": int(T * d * (4 if sh.dtype == 0 else 2) + 4)},
+        "gpu_launches": launches_per_step * args.steps,
+        "routing": {"max_load": int(counts.max()), "mean_load": float(counts.mean()),
+                    "experts_touched": int((counts > 0).sum()), "dropped": int(counts.sum() - kept.sum())},
+        "device_status": status,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host = oracle_inputs_on_host(inp)
+        n, dt = time_oracle(sh, host, CPU_SAMPLE[args.config], args.seed)
+        line["cpu_baseline"] = {"value": round(n / dt, 3), "unit": "tokens/s", "cores": oracle_threads(),
+                                "kind": "oracle",
+                                "sample": f"{n} of {T} tokens (routing of all {T}), fp64 numpy, {dt:.1f} s"}
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import torch
+    from synthetic import CONFIGS, make_inputs
+    sh = CONFIGS[args.config]
+    gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
+    host = oracle_inputs_on_host(make_inputs(sh, seed=args.seed, device=gen_dev))
+    n_tok = REF_SAMPLE[args.config]
+    for w in range(args.warmup):
+        time_oracle(sh, host, n_tok, args.seed + 1000 + w)
+    total_t, total_n = 0.0, 0
+    for k in range(args.steps):
+        n, dt = time_oracle(sh, host, n_tok, args.seed + k)
+        total_t += dt
+        total_n += n
+    value = total_n / total_t
+    cores = oracle_threads()
+    sample = f"{n_tok} of {sh.T} tokens per step (routing of all {sh.T}), fp64 numpy"
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1000 * total_t / args.steps, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)", "config": workload_config(sh, args.seed, "cpu"),
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

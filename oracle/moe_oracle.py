@@ -61,7 +61,7 @@ __all__ = [
     "dequant_rows_1x128", "dequant_blocks_128x128", "bf16_round",
     "router_logits", "softmax", "topk_select", "gates_of", "capacity_of",
     "dispatch_plan", "silu", "expert_ffn", "balance_stats", "topk_gap",
-    "route", "layer_forward", "to_f64",
+    "route", "layer_forward", "to_f64", "expert_weights",
 ]
 
 E4M3_MAX = 448.0
@@ -74,15 +74,24 @@ _QBLOCK = 128
 # no infinities, S.1111.111 is NaN; bf16 = the upper half of an IEEE fp32)
 # ----------------------------------------------------------------------------
 
+def _e4m3_value(c: int) -> float:
+    """Value of one e4m3 code from the format definition."""
+    sign = -1.0 if c & 0x80 else 1.0
+    e = (c >> 3) & 0xF
+    m = c & 0x7
+    if e == 15 and m == 7:
+        return math.nan
+    if e == 0:
+        return sign * (m / 8.0) * 2.0 ** -6
+    return sign * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+
+
+_E4M3_TABLE = np.array([_e4m3_value(c) for c in range(256)], dtype=np.float64)
+
+
 def e4m3_decode(codes: np.ndarray) -> np.ndarray:
     """uint8 e4m3 codes -> fp64 values (NaN for S.1111.111)."""
-    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
-    sign = np.where(c & 0x80, -1.0, 1.0)
-    e = (c >> 3) & 0xF
-    m = (c & 0x7).astype(np.float64)
-    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
-    mag = np.where((e == 15) & ((c & 0x7) == 7), np.nan, mag)
-    return sign * mag
+    return _E4M3_TABLE[np.asarray(codes, dtype=np.uint8)]
 
 
 _E4M3_POS = e4m3_decode(np.arange(127, dtype=np.uint8))   # codes 0x00..0x7E, ascending
@@ -309,7 +318,7 @@ def route(shape, inputs, logits: Optional[np.ndarray] = None):
             "f": f, "P": P, "loss": L, "gap": topk_gap(l64, shape.top_k)}
 
 
-def _expert_weights(inputs, prefix: str, e: int, fp8: bool):
+def expert_weights(inputs, prefix: str, e: int, fp8: bool):
     """fp64 (W1, b1, W2, b2) of routed (prefix 'W') or shared (prefix 'Ws')
     expert e."""
     b = "b" if prefix == "W" else "bs"
@@ -362,7 +371,7 @@ def layer_forward(shape, inputs, tokens: Optional[np.ndarray] = None,
                 by_expert.setdefault(int(rt["idx"][t, k]), []).append((i, k))
     y_slot: Dict[tuple, np.ndarray] = {}
     for e in sorted(by_expert):
-        W1, b1, W2, b2 = _expert_weights(inputs, "W", e, fp8)
+        W1, b1, W2, b2 = expert_weights(inputs, "W", e, fp8)
         rows = by_expert[e]
         y = expert_ffn(xin[np.array([i for i, _ in rows])], W1, b1, W2, b2, fp8_hidden=fp8)
         if fp8:
@@ -375,7 +384,7 @@ def layer_forward(shape, inputs, tokens: Optional[np.ndarray] = None,
             if (i, k) in y_slot:
                 out[i] += rt["gates"][t, k] * y_slot[(i, k)]
     for s_i in range(shape.n_shared):
-        W1, b1, W2, b2 = _expert_weights(inputs, "Ws", s_i, fp8)
+        W1, b1, W2, b2 = expert_weights(inputs, "Ws", s_i, fp8)
         y = expert_ffn(xin, W1, b1, W2, b2, fp8_hidden=fp8)
         if fp8:
             y = bf16_round(y)

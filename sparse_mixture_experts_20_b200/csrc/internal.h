@@ -1,0 +1,103 @@
+// Internal (non-exported) launch interface between the C ABI layer and the
+// kernel files.  Every launcher enqueues on `stream` and returns the
+// cudaError_t of the launch.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+#include "../../include/moe_b200.h"
+
+namespace moe {
+
+// Workspace layout: byte offsets of every region, all 256-byte aligned.
+struct WsLayout {
+    size_t status;        // int32 status word (+ padding)
+    size_t psum;          // (route_blocks, N_r) f32: per-block sums of s
+    size_t bitmap;        // (T_words, N_r) u32: bit t%32 of word t/32 set if t selected j
+    size_t word_base;     // (T_words, N_r) i32: slots of j in earlier words
+    size_t h_r;           // routed hidden activations (R_cap, d_ff)
+    size_t h_r_scales;    // FP8: (R_cap, d_ff/128) f32
+    size_t h_s;           // shared hidden activations (n_shared*T, d_ff_shared)
+    size_t h_s_scales;    // FP8: (n_shared*T, d_ff_shared/128) f32
+    // used by moe_layer_forward only
+    size_t x_disp;
+    size_t x_disp_scales;
+    size_t y;
+    size_t topk_idx, gates, counts, kept, offsets, slot_row, row_slot;
+    size_t total;
+};
+
+struct Dims {
+    int T, d, E, K, dff, S, dffs;
+    int capacity;   // -1: none
+    int r_cap;
+    int x_disp_rows;
+    int y_rows;
+    int dtype;
+    float alpha;
+    int route_blocks;
+    int t_words;
+};
+
+constexpr int kRouteTokens = 32;    // tokens per router block
+
+int validate(const moe_config* cfg, Dims* dm);
+WsLayout ws_layout(const Dims& dm);
+
+// elements
+inline size_t act_bytes(int dtype) { return dtype == MOE_F32 ? 4 : 2; }
+inline size_t wt_bytes(int dtype) { return dtype == MOE_F32 ? 4 : (dtype == MOE_BF16 ? 2 : 1); }
+
+cudaError_t launch_router(const Dims& dm, const void* x, const float* W_r, const float* logit_bias,
+                          int32_t* topk_idx, float* gates, float* logits_out, float* psum,
+                          cudaStream_t st);
+
+cudaError_t launch_dispatch(const Dims& dm, const void* x, const int32_t* topk_idx,
+                            int32_t* counts, int32_t* kept, int32_t* offsets,
+                            int32_t* slot_row, int32_t* row_slot, void* x_disp,
+                            float* x_disp_scales, uint32_t* bitmap, int32_t* word_base,
+                            int32_t* status, cudaStream_t st);
+
+cudaError_t launch_combine(const Dims& dm, const void* y, const float* gates,
+                           const int32_t* slot_row, void* out, cudaStream_t st);
+
+cudaError_t launch_balance(const Dims& dm, const int32_t* counts, const float* psum,
+                           float* f, float* P, float* loss, cudaStream_t st);
+
+// One group of segments of a grouped GEMM C = act(A B^T + bias).
+struct GemmGroup {
+    const void* A;          // (a_rows, K) rows; element type per engine
+    int a_rows;             // rows addressable through A (for the TMA map)
+    int a_row_base;         // first A row of segment 0
+    int a_seg_stride;       // A rows between consecutive fixed segments (shared group)
+    const float* a_scales;  // FP8: (a_rows, K/128)
+    const void* B;          // (n_mats, N, K)
+    int n_mats;
+    const float* b_scales;  // FP8: (n_mats, N/128, K/128)
+    const float* bias;      // (n_mats, N)
+    void* C;                // output rows
+    int c_rows;
+    int c_row_base;
+    float* c_scales;        // FP8 GEMM1 output scales (c_rows, N/128)
+    int N, K;
+    // segments: routed groups take rows from offsets; fixed groups have
+    // n_fixed segments of fixed_rows rows each.
+    const int32_t* offsets; // (n_mats+1) or nullptr for a fixed group
+    int fixed_rows;
+};
+
+struct GemmArgs {
+    GemmGroup g[2];         // g[0] routed, g[1] shared (n_mats == 0 if none)
+    int silu;               // 1: first layer (bias + SiLU), 0: second layer (bias)
+    int out_fp8;            // FP8 engine: quantise the output (first layer)
+    int32_t* status;
+};
+
+cudaError_t launch_grouped_ffn_f32(const Dims& dm, const GemmArgs& a, cudaStream_t st);
+cudaError_t launch_grouped_ffn_bf16(const Dims& dm, const GemmArgs& a, cudaStream_t st);
+cudaError_t launch_grouped_ffn_fp8(const Dims& dm, const GemmArgs& a, cudaStream_t st);
+
+cudaError_t launch_wait_selftest(int64_t timeout_ns, int32_t* status, cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,132 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared
+entry point, and rejects bad arguments before touching the GPU."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as O
+import sparse_mixture_experts_20_b200 as M
+from synthetic import CONFIGS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"MOE_EXPORT\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text))
+    return names
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    L = M.lib()
+    names = declared_symbols()
+    assert len(names) >= 13
+    for n in sorted(names):
+        assert hasattr(L, n), n
+    assert set(M.EXPORTED) <= names
+
+
+def declared_arity():
+    """Parameter count of every exported function in include/*.h."""
+    out = {}
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            for m in re.finditer(r"MOE_EXPORT\s+[\w\s\*]+?\b(moe_\w+)\s*\(([^)]*)\)", text):
+                params = [p for p in m.group(2).split(",") if p.strip() and p.strip() != "void"]
+                out[m.group(1)] = len(params)
+    return out
+
+
+def test_binding_signatures_match_header():
+    """The ctypes argument lists have exactly the header's parameter count
+    (an extra argument would be passed as a C varargs int)."""
+    L = M.lib()
+    ar = declared_arity()
+    for name, n in ar.items():
+        assert len(getattr(L, name).argtypes) == n, (name, n, len(getattr(L, name).argtypes))
+
+
+def test_status_strings():
+    L = M.lib()
+    assert L.moe_status_string(0) == b"MOE_OK"
+    assert L.moe_status_string(5) == b"MOE_ERR_DEVICE_TIMEOUT"
+
+
+@pytest.mark.parametrize("cid", sorted(CONFIGS))
+def test_workspace_and_rows_for_every_config(cid):
+    sh = CONFIGS[cid]
+    cfg = M.make_config(sh)
+    assert M.moe_workspace_size(cfg) > 0
+    cap, r_cap, xr, yr = M.moe_buffer_rows(cfg)
+    C = O.capacity_of(sh.T, sh.top_k, sh.n_routed, sh.capacity_factor)
+    assert cap == (-1 if C is None else C)
+    assert r_cap == (sh.T * sh.top_k if C is None else min(sh.T * sh.top_k, sh.n_routed * C))
+    assert yr == r_cap + sh.n_shared * sh.T
+    assert xr == r_cap + (sh.T if (sh.dtype == 2 and sh.n_shared) else 0)
+
+
+def test_capacity_is_exact_ceiling():
+    rng = np.random.default_rng(0)
+    for _ in range(2000):
+        T = int(rng.integers(1, 5000))
+        E = int(rng.integers(1, 257))
+        K = int(rng.integers(1, min(E, 16) + 1))
+        cf = float(np.float32(rng.choice([rng.uniform(0.01, 3.0), 1.0, 1.25, 0.5, 2.0])))
+        cfg = M.make_config(T=T, d_model=64, n_routed=E, top_k=K, d_ff=64, capacity_factor=cf)
+        cap = M.moe_buffer_rows(cfg)[0]
+        assert cap == O.capacity_of(T, K, E, cf), (T, E, K, cf)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(T=0), dict(d_model=0), dict(n_routed=0), dict(top_k=0), dict(top_k=9), dict(d_ff=0),
+    dict(n_shared=-1), dict(n_shared=1, d_ff_shared=0), dict(capacity_factor=-1.0),
+    dict(capacity_factor=float("inf")), dict(dtype=7),
+])
+def test_invalid_config_rejected(bad):
+    kw = dict(T=64, d_model=128, n_routed=8, top_k=2, d_ff=256)
+    kw.update(bad)
+    cfg = M.make_config(**kw)
+    n = ctypes.c_size_t(0)
+    assert M.lib().moe_workspace_size(ctypes.byref(cfg), ctypes.byref(n)) == M.MOE_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("bad", [
+    dict(n_routed=300), dict(top_k=17, n_routed=32), dict(n_shared=9, d_ff_shared=64),
+    dict(d_model=96), dict(d_ff=200), dict(dtype=2, d_model=192), dict(dtype=2, d_ff=64),
+])
+def test_unsupported_shapes_rejected(bad):
+    kw = dict(T=64, d_model=128, n_routed=8, top_k=2, d_ff=256)
+    kw.update(bad)
+    cfg = M.make_config(**kw)
+    n = ctypes.c_size_t(0)
+    assert M.lib().moe_workspace_size(ctypes.byref(cfg), ctypes.byref(n)) == M.MOE_ERR_UNSUPPORTED
+
+
+def test_null_pointers_rejected_without_launch():
+    L = M.lib()
+    cfg = M.make_config(T=64, d_model=128, n_routed=8, top_k=2, d_ff=256)
+    c = ctypes.byref(cfg)
+    assert L.moe_route(c, None, None, None, None, None, None, None, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_dispatch(c, *([None] * 11)) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_expert_ffn(c, *([None] * 19)) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_combine(c, None, None, None, None, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_balance_stats(c, None, None, None, None, None, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_layer_forward(c, *([None] * 24)) == M.MOE_ERR_INVALID_ARG
+    # misaligned workspace / inputs (fake, never dereferenced)
+    assert L.moe_route(c, 0x1000, 0x1000, None, 0x1000, 0x1000, None, 0x1001, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_route(c, 0x1008, 0x1000, None, 0x1000, 0x1000, None, 0x1000, None) == M.MOE_ERR_INVALID_ARG
+
+
+def test_fp8_requires_scales():
+    L = M.lib()
+    cfg = M.make_config(T=64, d_model=128, n_routed=8, top_k=2, d_ff=128, dtype=2)
+    p = 0x10000
+    args = [p] * 8 + [None, p, None]     # x .. x_disp valid, x_disp_scales NULL, ws, stream
+    assert L.moe_dispatch(ctypes.byref(cfg), *args) == M.MOE_ERR_INVALID_ARG

@@ -1,0 +1,129 @@
+"""GPU parity of every stage and of the whole layer against the CPU oracle,
+on seeded inputs small enough for the oracle to finish in seconds but
+spanning several tiles, ragged segment tails and the edge cases of the
+method (capacity drops, empty experts, K = N_r, one expert, one token)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import sparse_mixture_experts_20_b200 as M
+from synthetic import CONFIGS, DTYPE_BF16, DTYPE_F32, DTYPE_FP8, MoEShape
+
+import moe_testlib as TL
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "cfg1-tiny-f32": CONFIGS[1],
+    "f32-ragged-shared-cap": MoEShape("f32r", 203, 128, 6, 2, 192, n_shared=1, d_ff_shared=128,
+                                      capacity_factor=1.0, dtype=DTYPE_F32),
+    "bf16-ragged-shared-cap": MoEShape("b1", 777, 256, 8, 2, 384, n_shared=1, d_ff_shared=192,
+                                       capacity_factor=1.1, dtype=DTYPE_BF16),
+    "bf16-fine-grained": MoEShape("b2", 1000, 512, 64, 8, 320, n_shared=2, d_ff_shared=256,
+                                  capacity_factor=1.25, dtype=DTYPE_BF16),
+    "bf16-nocap": MoEShape("b3", 513, 384, 16, 4, 640, dtype=DTYPE_BF16),
+    "bf16-k-equals-n": MoEShape("b4", 100, 128, 4, 4, 128, dtype=DTYPE_BF16),
+    "bf16-single-expert": MoEShape("b5", 70, 128, 1, 1, 256, dtype=DTYPE_BF16),
+    "bf16-one-token": MoEShape("b6", 1, 256, 8, 2, 256, n_shared=1, d_ff_shared=128, dtype=DTYPE_BF16),
+    "fp8-ragged-shared": MoEShape("f1", 300, 512, 16, 4, 256, n_shared=1, d_ff_shared=384, dtype=DTYPE_FP8),
+    "fp8-decode-skewed": MoEShape("f2", 37, 1024, 256, 8, 256, n_shared=1, d_ff_shared=256,
+                                  dtype=DTYPE_FP8, zipf_logit_bias=True),
+}
+
+
+def require_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_stage_and_layer_parity(name):
+    require_gpu()
+    sh = CASES[name]
+    inp = TL.gpu_inputs(sh, seed=1234)
+    o = TL.run_stages(sh, inp)
+    assert o["status"] == 0
+    rt_prod = TL.check_routing(sh, inp, o)
+    TL.check_dispatch(sh, inp, o, rt_prod)
+    TL.check_expert_ffn(sh, inp, o, rt_prod)
+    TL.check_combine(sh, o, rt_prod)
+    lay = TL.run_layer(sh, inp)
+    assert lay["status"] == 0
+    # the fused entry point runs the same kernels in the same order
+    assert torch.equal(lay["out"], o["out"])
+    assert torch.equal(lay["topk_idx"], o["topk_idx"])
+    assert torch.equal(lay["P"], o["P"]) and torch.equal(lay["f"], o["f"])
+    err, excluded = TL.check_end_to_end(sh, inp, lay["out"], TL.cpu(lay["topk_idx"]).numpy())
+    assert excluded <= max(2, sh.T // 100)
+    assert err < TL.TOL_REL_FROB[sh.dtype], err
+
+
+def test_all_tokens_to_one_expert_with_capacity():
+    require_gpu()
+    sh = MoEShape("hot", 500, 256, 8, 2, 256, capacity_factor=1.0, dtype=DTYPE_BF16)
+    inp = TL.gpu_inputs(sh, seed=7)
+    bias = torch.zeros(8, device="cuda")
+    bias[3] = 60.0                        # every token's first choice is expert 3
+    bias[5] = -60.0                       # expert 5 is never chosen (empty segment)
+    inp["logit_bias"] = bias
+    o = TL.run_stages(sh, inp)
+    rt = TL.check_routing(sh, inp, o)
+    C = rt["C"]
+    assert rt["plan"]["counts"][3] == 500 and rt["plan"]["kept"][3] == C
+    assert rt["plan"]["counts"][5] == 0
+    TL.check_dispatch(sh, inp, o, rt)
+    TL.check_expert_ffn(sh, inp, o, rt)
+    TL.check_combine(sh, o, rt)
+    err, _ = TL.check_end_to_end(sh, inp, o["out"], TL.cpu(o["topk_idx"]).numpy())
+    assert err < TL.TOL_REL_FROB[sh.dtype]
+
+
+def test_bad_routing_is_flagged_and_dropped():
+    require_gpu()
+    sh = MoEShape("bad", 64, 128, 8, 2, 128, dtype=DTYPE_BF16)
+    inp = TL.gpu_inputs(sh, seed=3)
+    cfg = M.make_config(sh)
+    dev = "cuda"
+    idx = torch.tensor(np.stack([np.arange(64) % 8, (np.arange(64) + 1) % 8], 1), dtype=torch.int32, device=dev)
+    idx[5, 1] = 8                         # out of range
+    idx[9, 1] = idx[9, 0]                 # repeated within the token
+    ws = torch.empty(M.moe_workspace_size(cfg), dtype=torch.uint8, device=dev)
+    M.moe_workspace_init(cfg, ws)
+    E, T, K = 8, 64, 2
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    kept = torch.empty_like(counts)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    slot_row = torch.empty((T, K), dtype=torch.int32, device=dev)
+    row_slot = torch.empty(T * K, dtype=torch.int32, device=dev)
+    x_disp = torch.empty((T * K, 128), dtype=torch.bfloat16, device=dev)
+    M.moe_dispatch(cfg, inp["x"], idx, counts, kept, offsets, slot_row, row_slot, x_disp, None, ws)
+    status = M.moe_get_device_status(cfg, ws, clear=True)
+    assert status & M.MOE_DEV_BAD_ROUTING
+    sr = slot_row.cpu().numpy()
+    assert sr[5, 1] == -1 and sr[9, 1] == -1
+    assert int(counts.sum()) == T * K - 2
+    assert M.moe_get_device_status(cfg, ws) == 0
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    require_gpu()
+    sh = MoEShape("to", 64, 128, 8, 2, 128, dtype=DTYPE_BF16)
+    cfg = M.make_config(sh)
+    ws = torch.empty(M.moe_workspace_size(cfg), dtype=torch.uint8, device="cuda")
+    M.moe_workspace_init(cfg, ws)
+    M.moe_selftest_wait_timeout(cfg, 20_000_000, ws)          # 20 ms
+    assert M.moe_get_device_status(cfg, ws, clear=True) & M.MOE_DEV_TIMEOUT
+    inp = TL.gpu_inputs(sh, seed=5)
+    o = TL.run_stages(sh, inp)                                  # the context still works
+    assert o["status"] == 0
+    TL.check_routing(sh, inp, o)
+
+
+def test_layer_is_deterministic():
+    require_gpu()
+    sh = CASES["bf16-fine-grained"]
+    inp = TL.gpu_inputs(sh, seed=99)
+    a = TL.run_layer(sh, inp)
+    b = TL.run_layer(sh, inp)
+    assert torch.equal(a["out"], b["out"]) and torch.equal(a["P"], b["P"]) and torch.equal(a["loss"], b["loss"])
