@@ -99,7 +99,8 @@ _E4M3_POS = e4m3_decode(np.arange(127, dtype=np.uint8))   # codes 0x00..0x7E, as
 
 def e4m3_round(v: np.ndarray) -> np.ndarray:
     """Round fp64 values to e4m3 codes: nearest representable value, ties to
-    the even code, magnitudes beyond 448 saturate to 448."""
+    the even code, magnitudes beyond 448 saturate to 448; as in IEEE
+    rounding, a negative value that rounds to zero gives negative zero."""
     v = np.asarray(v, dtype=np.float64)
     a = np.minimum(np.abs(v), E4M3_MAX)
     hi = np.searchsorted(_E4M3_POS, a, side="left")          # first table value >= a
@@ -109,7 +110,8 @@ def e4m3_round(v: np.ndarray) -> np.ndarray:
     d_lo = a - _E4M3_POS[lo]
     pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
     code = np.where(pick_hi, hi, lo).astype(np.uint8)
-    code = np.where(np.signbit(v) & (code != 0), code | 0x80, code)
+    # the sign is kept, also when the magnitude rounds to zero (-0 is S=1, E=0, M=0)
+    code = np.where(np.signbit(v), code | 0x80, code)
     return code.astype(np.uint8)
 
 

@@ -100,9 +100,13 @@ def check_routing(shape, inp, o):
     l64 = rt_prod["logits"]
     scale = np.abs(l64).max() + 1e-30
     assert np.max(np.abs(logits - l64)) / scale < 2e-5
+    # softmax, gates and P of the product's logits (the fused part of the
+    # router), then P against the oracle's own fp64 logits (spec 1e-6)
+    s_prod = O.softmax(logits)
     g = cpu(o["gates"]).double().numpy()
-    assert np.max(np.abs(g - rt_prod["gates"])) < 2e-6
+    assert np.max(np.abs(g - O.gates_of(s_prod, idx))) < 2e-6
     P = cpu(o["P"]).double().numpy()
+    assert np.max(np.abs(P - s_prod.mean(axis=0))) < 1e-6
     assert np.max(np.abs(P - rt_prod["P"])) < 1e-6
     f = cpu(o["f"]).double().numpy()
     assert np.max(np.abs(f - rt_prod["f"])) < 1e-6
