@@ -229,6 +229,32 @@ MOE_EXPORT int moe_layer_forward(const moe_config* cfg, const void* x, const flo
 MOE_EXPORT int moe_selftest_wait_timeout(const moe_config* cfg, int64_t timeout_ns,
                               void* ws, void* stream);
 
+/* ---- dispatch without a workspace ------------------------------------------
+ * No counterpart in the paper: an addition for callers that cannot allocate
+ * device memory -- code running inside a host framework that owns every
+ * device allocation and gives a plugin none of its own, or a latency-critical
+ * caller that cannot afford the device-wide synchronisation of cudaMalloc.
+ * Same outputs as moe_dispatch (same kernels, bit for bit) but no `ws`
+ * argument: the dispatch scratch (token bitmaps and prefix counts,
+ * 2 * ceil(T/32) * N_r 32-bit words, each half rounded up to 256 bytes) comes
+ * from a 2 MiB array in device memory that belongs to the library, so every
+ * GPU that loads the library holds those 2 MiB until the process exits.
+ * Shapes whose scratch exceeds 2 MiB return MOE_ERR_UNSUPPORTED (e.g. T up to
+ * 32768 tokens at N_r = 256).  The call allocates nothing.  The first call on
+ * each device looks up the array's device address (cudaGetSymbolAddress, with
+ * that device current); make that first call before any stream capture.
+ * Every call on a device shares the one array and leaves its contents behind;
+ * the kernels rewrite all of it before reading, so nothing needs clearing,
+ * but calls that overlap on the GPU (other streams, other threads) race on it
+ * and must be serialised by the caller.  Bad routing indices are dropped as
+ * in moe_dispatch but not reported (there is no status word).
+ *   x, topk_idx, counts, kept, offsets, slot_row, row_slot, x_disp,
+ *   x_disp_scales: as moe_dispatch. */
+MOE_EXPORT int moe_dispatch_noalloc(const moe_config* cfg, const void* x, const int32_t* topk_idx,
+                                    int32_t* counts, int32_t* kept, int32_t* offsets,
+                                    int32_t* slot_row, int32_t* row_slot, void* x_disp,
+                                    float* x_disp_scales, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

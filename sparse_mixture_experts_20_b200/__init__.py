@@ -34,6 +34,7 @@ EXPORTED = (
     "moe_workspace_size", "moe_buffer_rows", "moe_workspace_init", "moe_get_device_status",
     "moe_last_cuda_error", "moe_status_string", "moe_route", "moe_dispatch", "moe_expert_ffn",
     "moe_combine", "moe_balance_stats", "moe_layer_forward", "moe_selftest_wait_timeout",
+    "moe_dispatch_noalloc",
 )
 
 
@@ -85,6 +86,7 @@ def lib() -> ctypes.CDLL:
             "moe_balance_stats": [cfgp, P, P, P, P, P, P],
             "moe_layer_forward": [cfgp] + [P] * 24,
             "moe_selftest_wait_timeout": [cfgp, ctypes.c_int64, P, P],
+            "moe_dispatch_noalloc": [cfgp, P, P, P, P, P, P, P, P, P, P],
         }
         for name, args in sig.items():
             fn = getattr(L, name)
@@ -199,6 +201,16 @@ def moe_layer_forward(cfg, x, W_r, logit_bias, W1, W1_scales, b1, W2, W2_scales,
 def moe_selftest_wait_timeout(cfg, timeout_ns: int, ws, stream=None):
     _check(lib().moe_selftest_wait_timeout(ctypes.byref(cfg), int(timeout_ns), _p(ws), _stream(stream)),
            "moe_selftest_wait_timeout")
+
+
+def moe_dispatch_noalloc(cfg, x, topk_idx, counts, kept, offsets, slot_row, row_slot, x_disp,
+                         x_disp_scales, stream=None):
+    """moe_dispatch with its scratch in the library's own 2 MiB device array
+    instead of a workspace: for callers that cannot allocate device memory.
+    Calls that overlap on the GPU race on that array."""
+    _check(lib().moe_dispatch_noalloc(ctypes.byref(cfg), _p(x), _p(topk_idx), _p(counts), _p(kept),
+                                      _p(offsets), _p(slot_row), _p(row_slot), _p(x_disp),
+                                      _p(x_disp_scales), _stream(stream)), "moe_dispatch_noalloc")
 
 
 class MoELayer:

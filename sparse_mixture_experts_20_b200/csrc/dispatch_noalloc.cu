@@ -1,0 +1,76 @@
+// moe_dispatch_noalloc: moe_dispatch without a caller-provided workspace.
+//
+// The dispatch kernels need scratch memory for their per-expert token bitmaps
+// and word prefix counts.  moe_dispatch takes it from the caller's workspace;
+// this entry point takes it from a fixed array in device memory that is part
+// of the library image instead, so that a caller which cannot allocate device
+// memory can still dispatch.  Every GPU that loads the library holds the
+// array (kNoAllocScratchBytes) until the process exits.
+#include <mutex>
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 2u << 20;   // 2 MiB
+
+// Scratch shared by every call of moe_dispatch_noalloc on this device.
+static __device__ __align__(256) uint8_t g_dispatch_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+void* g_scratch_dev_ptr[kMaxDevices] = {};
+std::mutex g_scratch_mutex;
+
+// Device address of g_dispatch_scratch on the current device, looked up once
+// per device (host code cannot use the symbol itself as a device pointer).
+cudaError_t scratch_on_current_device(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_dev_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_dispatch_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_dev_ptr[dev] = p;
+    }
+    *out = g_scratch_dev_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" int moe_dispatch_noalloc(const moe_config* cfg, const void* x, const int32_t* topk_idx,
+                                    int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* slot_row,
+                                    int32_t* row_slot, void* x_disp, float* x_disp_scales, void* stream) {
+    Dims dm;
+    const int v = validate(cfg, &dm);
+    if (v != MOE_OK) return v;
+    if (!x || !topk_idx || !counts || !kept || !offsets || !slot_row || !row_slot || !x_disp)
+        return MOE_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(x_disp) & 15u))
+        return MOE_ERR_INVALID_ARG;
+    if (dm.dtype == MOE_FP8_E4M3_BLOCK && !x_disp_scales) return MOE_ERR_INVALID_ARG;
+    // bitmap and word bases, each (T/32, N_r) 32-bit words, 256-byte aligned
+    const size_t part = (static_cast<size_t>(dm.t_words) * dm.E * 4 + 255) & ~static_cast<size_t>(255);
+    if (2 * part > kNoAllocScratchBytes) return MOE_ERR_UNSUPPORTED;
+    void* base = nullptr;
+    cudaError_t e = scratch_on_current_device(&base);
+    if (e == cudaSuccess) {
+        // Both regions are fully rewritten by every call: nothing to clear.
+        uint32_t* bitmap = static_cast<uint32_t*>(base);
+        int32_t* word_base = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(base) + part);
+        e = launch_dispatch(dm, x, topk_idx, counts, kept, offsets, slot_row, row_slot, x_disp, x_disp_scales,
+                            bitmap, word_base, nullptr, static_cast<cudaStream_t>(stream));
+    }
+    if (e != cudaSuccess) {
+        note_cuda_error(static_cast<int>(e));
+        return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+}

@@ -100,4 +100,7 @@ cudaError_t launch_grouped_ffn_fp8(const Dims& dm, const GemmArgs& a, cudaStream
 
 cudaError_t launch_wait_selftest(int64_t timeout_ns, int32_t* status, cudaStream_t st);
 
+// Records a failed CUDA call for moe_last_cuda_error() on this thread.
+void note_cuda_error(int err);
+
 }  // namespace moe

@@ -225,6 +225,8 @@ __global__ void wait_selftest_kernel(int64_t timeout_ns, int32_t* status) {
 
 }  // namespace
 
+void note_cuda_error(int err) { g_last_cuda_error = err; }
+
 cudaError_t launch_wait_selftest(int64_t timeout_ns, int32_t* status, cudaStream_t st) {
     wait_selftest_kernel<<<1, 32, 0, st>>>(timeout_ns, status);
     return cudaGetLastError();
