@@ -448,57 +448,6 @@ grouped_ffn_tc_kernel(const __grid_constant__ TcParams p) {
 
 // ------------------------------------------------------------------ host side
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
-}
-
-// 2D map over (rows, K) row-major with box (128 bytes of K, box_rows rows).
-bool encode_2d(CUtensorMap* m, const void* base, int rows, int K, int elem, int box_rows) {
-    auto fn = get_encode_fn();
-    if (!fn) return false;
-    const CUtensorMapDataType dt = elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
-    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
-    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * elem};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem), static_cast<cuuint32_t>(box_rows)};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// 3D map over (n_mats, N, K) with box (128 bytes of K, box_rows of N, 1).
-bool encode_3d(CUtensorMap* m, const void* base, int n_mats, int N, int K, int elem, int box_rows) {
-    auto fn = get_encode_fn();
-    if (!fn) return false;
-    const CUtensorMapDataType dt = elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(n_mats)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(K) * elem, static_cast<cuuint64_t>(N) * K * elem};
-    cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem), static_cast<cuuint32_t>(box_rows), 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int num_sms() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
-    return n;
-}
-
 template <bool FP8>
 cudaError_t launch_tc(const GemmArgs& a, cudaStream_t st) {
     using C = Cfg<FP8>;
@@ -521,8 +470,8 @@ cudaError_t launch_tc(const GemmArgs& a, cudaStream_t st) {
         d.c_scales = g.c_scales;
         d.N = g.N;
         d.K = g.K;
-        if (!encode_2d(&p.a_map[gi], g.A, g.a_rows, g.K, C::ELEM, BM)) return cudaErrorInvalidValue;
-        if (!encode_3d(&p.b_map[gi], g.B, g.n_mats, g.N, g.K, C::ELEM, C::BN)) return cudaErrorInvalidValue;
+        if (!encode_tma_2d(&p.a_map[gi], g.A, g.a_rows, g.K, C::ELEM, BM)) return cudaErrorInvalidValue;
+        if (!encode_tma_3d(&p.b_map[gi], g.B, g.n_mats, g.N, g.K, C::ELEM, C::BN)) return cudaErrorInvalidValue;
     }
     p.silu = a.silu;
     p.out_fp8 = a.out_fp8;
@@ -533,7 +482,7 @@ cudaError_t launch_tc(const GemmArgs& a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(grouped_ffn_tc_kernel<FP8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    grouped_ffn_tc_kernel<FP8><<<num_sms(), NUM_THREADS, smem, st>>>(p);
+    grouped_ffn_tc_kernel<FP8><<<device_sm_count(), NUM_THREADS, smem, st>>>(p);
     return cudaGetLastError();
 }
 

@@ -20,6 +20,9 @@ struct WsLayout {
     size_t h_r_scales;    // FP8: (R_cap, d_ff/128) f32
     size_t h_s;           // shared hidden activations (n_shared*T, d_ff_shared)
     size_t h_s_scales;    // FP8: (n_shared*T, d_ff_shared/128) f32
+    size_t router_w3;     // tensor-core router: (N_r, 3 d) bf16 planes of W_r
+    size_t router_part;   // tensor-core router: (ksplit, T, N_r) f32 partial logits
+    size_t router_logits; // tensor-core router: (T, N_r) f32 summed logits
     // used by moe_layer_forward only
     size_t x_disp;
     size_t x_disp_scales;
@@ -49,9 +52,29 @@ WsLayout ws_layout(const Dims& dm);
 inline size_t act_bytes(int dtype) { return dtype == MOE_F32 ? 4 : 2; }
 inline size_t wt_bytes(int dtype) { return dtype == MOE_F32 ? 4 : (dtype == MOE_BF16 ? 2 : 1); }
 
+// Scratch of the tensor-core router (workspace regions; unused otherwise).
+struct RouterScratch {
+    void* w3;
+    float* part;
+    float* logits;
+    int32_t* status;
+};
+
+// Tile plan of the tensor-core router: m-tiles of 128 tokens, nt tiles of bn
+// experts, ksplit splits of K = 3 d.
+struct RouterTcPlan {
+    int mt, nt, bn, ksplit;
+};
+
+bool router_uses_small(const Dims& dm);
+bool router_uses_tc(const Dims& dm);
+RouterTcPlan router_tc_plan(const Dims& dm);
+cudaError_t launch_router_tc(const Dims& dm, const RouterTcPlan& plan, const void* x, const float* W_r,
+                             void* w3, float* part, int32_t* status, cudaStream_t st);
+
 cudaError_t launch_router(const Dims& dm, const void* x, const float* W_r, const float* logit_bias,
                           int32_t* topk_idx, float* gates, float* logits_out, float* psum,
-                          cudaStream_t st);
+                          const RouterScratch& rs, cudaStream_t st);
 
 cudaError_t launch_dispatch(const Dims& dm, const void* x, const int32_t* topk_idx,
                             int32_t* counts, int32_t* kept, int32_t* offsets,
@@ -99,6 +122,11 @@ cudaError_t launch_grouped_ffn_bf16(const Dims& dm, const GemmArgs& a, cudaStrea
 cudaError_t launch_grouped_ffn_fp8(const Dims& dm, const GemmArgs& a, cudaStream_t st);
 
 cudaError_t launch_wait_selftest(int64_t timeout_ns, int32_t* status, cudaStream_t st);
+
+// TMA tensor maps (tma_host.cu).  `map` points at a CUtensorMap.
+bool encode_tma_2d(void* map, const void* base, int rows, int K, int elem, int box_rows);
+bool encode_tma_3d(void* map, const void* base, int n_mats, int N, int K, int elem, int box_rows);
+int device_sm_count();
 
 // Records a failed CUDA call for moe_last_cuda_error() on this thread.
 void note_cuda_error(int err);

@@ -100,6 +100,14 @@ WsLayout ws_layout(const Dims& dm) {
     L.h_r_scales = take(fp8 ? static_cast<size_t>(dm.r_cap) * (dm.dff / 128) * 4 : 0);
     L.h_s = take(static_cast<size_t>(dm.S) * dm.T * dm.dffs * hb);
     L.h_s_scales = take(fp8 ? static_cast<size_t>(dm.S) * dm.T * (dm.dffs / 128) * 4 : 0);
+    if (router_uses_tc(dm)) {
+        const RouterTcPlan rp = router_tc_plan(dm);
+        L.router_w3 = take(static_cast<size_t>(dm.E) * 3 * dm.d * 2);
+        L.router_part = take(static_cast<size_t>(rp.ksplit) * dm.T * dm.E * 4);
+        L.router_logits = take(static_cast<size_t>(dm.T) * dm.E * 4);
+    } else {
+        L.router_w3 = L.router_part = L.router_logits = take(0);
+    }
     L.x_disp = take(static_cast<size_t>(dm.x_disp_rows) * dm.d * hb);
     L.x_disp_scales = take(fp8 ? static_cast<size_t>(dm.x_disp_rows) * (dm.d / 128) * 4 : 0);
     L.y = take(static_cast<size_t>(dm.y_rows) * dm.d * (dm.dtype == MOE_F32 ? 4 : 2));
@@ -118,6 +126,15 @@ namespace {
 
 template <typename T> T* at(void* ws, size_t off) {
     return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+RouterScratch router_scratch(void* ws, const WsLayout& L) {
+    RouterScratch rs;
+    rs.w3 = at<uint8_t>(ws, L.router_w3);
+    rs.part = at<float>(ws, L.router_part);
+    rs.logits = at<float>(ws, L.router_logits);
+    rs.status = at<int32_t>(ws, L.status);
+    return rs;
 }
 
 // Builds the two grouped-GEMM launches of the expert FFN and runs them.
@@ -306,7 +323,7 @@ int moe_route(const moe_config* cfg, const void* x, const float* W_r, const floa
     if (!aligned16(x) || !aligned16(W_r) || (reinterpret_cast<uintptr_t>(ws) & 255u)) return MOE_ERR_INVALID_ARG;
     const WsLayout L = ws_layout(dm);
     return cuda_status(launch_router(dm, x, W_r, logit_bias, topk_idx, gates, logits_out,
-                                     at<float>(ws, L.psum), static_cast<cudaStream_t>(stream)));
+                                     at<float>(ws, L.psum), router_scratch(ws, L), static_cast<cudaStream_t>(stream)));
 }
 
 int moe_dispatch(const moe_config* cfg, const void* x, const int32_t* topk_idx, int32_t* counts,
@@ -389,7 +406,8 @@ int moe_layer_forward(const moe_config* cfg, const void* x, const float* W_r, co
                      Ws1_scales, bs1, Ws2, Ws2_scales, bs2))
         return MOE_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_router(dm, x, W_r, logit_bias, idx, g, nullptr, at<float>(ws, L.psum), st);
+    cudaError_t e = launch_router(dm, x, W_r, logit_bias, idx, g, nullptr, at<float>(ws, L.psum),
+                                  router_scratch(ws, L), st);
     if (e != cudaSuccess) return cuda_status(e);
     e = launch_dispatch(dm, x, idx, cnt, at<int32_t>(ws, L.kept), offsets, slot_row, at<int32_t>(ws, L.row_slot),
                         x_disp, x_disp_sc, at<uint32_t>(ws, L.bitmap), at<int32_t>(ws, L.word_base),

@@ -1,15 +1,23 @@
-// Router: logits, softmax, top-K and gate renormalisation in one kernel.
+// Router: logits, softmax, top-K and gate renormalisation.
 //
 // "論文解説: DeepSeekMoE" §ルーティングとバランス損失: s_j = softmax(W_r x)_j,
 // g_j = s_j / sum_{k in TopK} s_k; §アルゴリズム: the router is a Linear
 // layer without bias.  "Sparse MoE Top-Kルーティング" §ルーティングの仕組み.
 //
-// One block of 256 threads handles 32 tokens and every expert.  The logits
-// are an fp32 GEMM (x tile x W_r^T) staged through shared memory in chunks of
-// 32 columns; warp w then owns tokens w, w+8, w+16, w+24 and does the
-// softmax, a K-round warp arg-max (ties to the lower expert index) and the
-// gates with shuffles.  Per-block column sums of s go to psum in a fixed
-// order, so the balance statistics are bit-reproducible.
+// The logits come from one of three producers, chosen by shape:
+//   * router_small_kernel (N_r <= 32 and W_r fits in shared memory): W_r is
+//     staged once per block; each warp takes 4 (or 2) tokens, lanes split the
+//     model dimension with 16-byte loads of x, and a reduce-scatter over the
+//     lanes leaves each lane with whole dot products.  x is read once.
+//   * the tensor-core router (router_tc.cu, bf16 x, larger N_r): W_r split into
+//     three bf16 planes, one tcgen05 GEMM with K = 3 d, partial logits per K
+//     split summed here by router_reduce_kernel;
+//   * router_generic_kernel (fp32 x with a large W_r): a shared-memory tiled
+//     fp32 GEMM.
+// All three end in select_block: per token a warp-wide softmax, a K-round
+// arg-max (ties to the lower expert index) and the gates; per block the
+// column sums of s over its 32 tokens go to psum in token order, so the
+// balance statistics are bit-reproducible.
 #include "common.cuh"
 #include "internal.h"
 
@@ -17,82 +25,23 @@ namespace moe {
 namespace {
 
 constexpr int TT = kRouteTokens;   // tokens per block
-constexpr int KC = 32;             // columns per shared-memory chunk
+constexpr int KC = 32;             // columns per shared-memory chunk (generic kernel)
 constexpr int NTHREADS = 256;
 
 template <typename XT> __device__ __forceinline__ float to_f(XT v);
 template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
 template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
 
-template <typename XT, int EPT>
-__global__ void __launch_bounds__(NTHREADS)
-router_kernel(const XT* __restrict__ x, const float* __restrict__ W_r,
-              const float* __restrict__ logit_bias, int T, int d, int E, int K,
-              int32_t* __restrict__ topk_idx, float* __restrict__ gates,
-              float* __restrict__ logits_out, float* __restrict__ psum) {
-    constexpr int NP = EPT * 32;                     // experts padded to the lanes
-    __shared__ float xs[TT][KC + 1];
-    __shared__ float wsh[(NP * (KC + 1) > TT * (NP + 1)) ? NP * (KC + 1) : TT * (NP + 1)];
-    float (*wtile)[KC + 1] = reinterpret_cast<float (*)[KC + 1]>(wsh);
-    float (*lg)[NP + 1] = reinterpret_cast<float (*)[NP + 1]>(wsh);
-
+// lg: TT rows of EPT*32 (+1 pad) logits with the bias already added and -inf
+// in padded expert columns.  Rows of tokens >= T are ignored.  Overwrites lg
+// with s.
+template <int EPT>
+__device__ __forceinline__ void select_block(float* lg_raw, int t0, int T, int E, int K,
+                                             int32_t* __restrict__ topk_idx, float* __restrict__ gates,
+                                             float* __restrict__ logits_out, float* __restrict__ psum) {
+    constexpr int NP = EPT * 32;
+    float (*lg)[NP + 1] = reinterpret_cast<float (*)[NP + 1]>(lg_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int t0 = blockIdx.x * TT;
-
-    float acc[4][EPT];
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < EPT; ++b) acc[a][b] = 0.f;
-
-    for (int k0 = 0; k0 < d; k0 += KC) {
-        // x chunk: TT x KC values, 4 per thread
-#pragma unroll
-        for (int i = 0; i < (TT * KC) / NTHREADS; ++i) {
-            const int e = tid + i * NTHREADS;
-            const int r = e / KC, c = e % KC;
-            const int t = t0 + r;
-            xs[r][c] = (t < T) ? to_f<XT>(x[static_cast<size_t>(t) * d + k0 + c]) : 0.f;
-        }
-        // W_r chunk: NP x KC values as float4
-        for (int e = tid; e < NP * (KC / 4); e += NTHREADS) {
-            const int r = e / (KC / 4), c4 = e % (KC / 4);
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (r < E) v = *reinterpret_cast<const float4*>(W_r + static_cast<size_t>(r) * d + k0 + c4 * 4);
-            wtile[r][c4 * 4 + 0] = v.x;
-            wtile[r][c4 * 4 + 1] = v.y;
-            wtile[r][c4 * 4 + 2] = v.z;
-            wtile[r][c4 * 4 + 3] = v.w;
-        }
-        __syncthreads();
-#pragma unroll 8
-        for (int kk = 0; kk < KC; ++kk) {
-            float xv[4], wv[EPT];
-#pragma unroll
-            for (int a = 0; a < 4; ++a) xv[a] = xs[warp * 4 + a][kk];
-#pragma unroll
-            for (int b = 0; b < EPT; ++b) wv[b] = wtile[lane + 32 * b][kk];
-#pragma unroll
-            for (int a = 0; a < 4; ++a)
-#pragma unroll
-                for (int b = 0; b < EPT; ++b) acc[a][b] = fmaf(xv[a], wv[b], acc[a][b]);
-        }
-        __syncthreads();
-    }
-
-    // logits (+ bias) into shared memory; padded experts get -inf
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < EPT; ++b) {
-            const int j = lane + 32 * b;
-            float v = -INFINITY;
-            if (j < E) v = acc[a][b] + (logit_bias ? logit_bias[j] : 0.f);
-            lg[warp * 4 + a][j] = v;
-        }
-    __syncthreads();
-
-    // per-token softmax / top-K / gates: warp w owns tokens w + 8*i
 #pragma unroll 1
     for (int i = 0; i < TT / 8; ++i) {
         const int r = warp + 8 * i;
@@ -132,7 +81,6 @@ router_kernel(const XT* __restrict__ x, const float* __restrict__ W_r,
             if ((bj & 31) == lane) taken |= 1u << (bj >> 5);
             if (lane == k) { sel_v = bv; sel_j = bj; }
         }
-        // softmax over all experts
         float e_sum = 0.f;
 #pragma unroll
         for (int b = 0; b < EPT; ++b) {
@@ -145,7 +93,6 @@ router_kernel(const XT* __restrict__ x, const float* __restrict__ W_r,
         const float inv = 1.0f / e_sum;
 #pragma unroll
         for (int b = 0; b < EPT; ++b) lg[r][lane + 32 * b] = v[b] * inv;
-        // gates: s_sel / sum s_sel over the K selected experts
         const float es = (lane < K) ? expf(sel_v - vmax) * inv : 0.f;
         float g_sum = es;
 #pragma unroll
@@ -156,8 +103,6 @@ router_kernel(const XT* __restrict__ x, const float* __restrict__ W_r,
         }
     }
     __syncthreads();
-
-    // per-block column sums of s, token order
     for (int j = tid; j < E; j += NTHREADS) {
         float s = 0.f;
         for (int r = 0; r < TT; ++r) s += lg[r][j];
@@ -165,30 +110,282 @@ router_kernel(const XT* __restrict__ x, const float* __restrict__ W_r,
     }
 }
 
+// ---------------------------------------------------------------- generic (fp32 x)
+
+template <typename XT, int EPT>
+__global__ void __launch_bounds__(NTHREADS)
+router_generic_kernel(const XT* __restrict__ x, const float* __restrict__ W_r,
+                      const float* __restrict__ logit_bias, int T, int d, int E, int K,
+                      int32_t* __restrict__ topk_idx, float* __restrict__ gates,
+                      float* __restrict__ logits_out, float* __restrict__ psum) {
+    constexpr int NP = EPT * 32;
+    __shared__ float xs[TT][KC + 1];
+    __shared__ float wsh[(NP * (KC + 1) > TT * (NP + 1)) ? NP * (KC + 1) : TT * (NP + 1)];
+    float (*wtile)[KC + 1] = reinterpret_cast<float (*)[KC + 1]>(wsh);
+    float (*lg)[NP + 1] = reinterpret_cast<float (*)[NP + 1]>(wsh);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t0 = blockIdx.x * TT;
+    float acc[4][EPT];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < EPT; ++b) acc[a][b] = 0.f;
+    for (int k0 = 0; k0 < d; k0 += KC) {
+#pragma unroll
+        for (int i = 0; i < (TT * KC) / NTHREADS; ++i) {
+            const int e = tid + i * NTHREADS;
+            const int r = e / KC, c = e % KC;
+            const int t = t0 + r;
+            xs[r][c] = (t < T) ? to_f<XT>(x[static_cast<size_t>(t) * d + k0 + c]) : 0.f;
+        }
+        for (int e = tid; e < NP * (KC / 4); e += NTHREADS) {
+            const int r = e / (KC / 4), c4 = e % (KC / 4);
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (r < E) v = *reinterpret_cast<const float4*>(W_r + static_cast<size_t>(r) * d + k0 + c4 * 4);
+            wtile[r][c4 * 4 + 0] = v.x;
+            wtile[r][c4 * 4 + 1] = v.y;
+            wtile[r][c4 * 4 + 2] = v.z;
+            wtile[r][c4 * 4 + 3] = v.w;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < KC; ++kk) {
+            float xv[4], wv[EPT];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) xv[a] = xs[warp * 4 + a][kk];
+#pragma unroll
+            for (int b = 0; b < EPT; ++b) wv[b] = wtile[lane + 32 * b][kk];
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < EPT; ++b) acc[a][b] = fmaf(xv[a], wv[b], acc[a][b]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < EPT; ++b) {
+            const int j = lane + 32 * b;
+            float v = -INFINITY;
+            if (j < E) v = acc[a][b] + (logit_bias ? logit_bias[j] : 0.f);
+            lg[warp * 4 + a][j] = v;
+        }
+    __syncthreads();
+    select_block<EPT>(wsh, t0, T, E, K, topk_idx, gates, logits_out, psum);
+}
+
+// ---------------------------------------------------------------- small N_r
+
+// After the call, v[i] of lane l holds the warp-wide sum of original index
+// l * (N / 32) + i, for i < N / 32 (a reduce-scatter in 5 shuffle rounds).
+template <int N>
+__device__ __forceinline__ void warp_reduce_scatter(float (&v)[N], int lane) {
+    static_assert(N >= 32 && (N & (N - 1)) == 0, "power of two >= 32");
+#pragma unroll
+    for (int s = 0; s < 5; ++s) {
+        const int o = 16 >> s;
+        const int half = (N >> s) / 2;
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+            const float send = upper ? v[i] : v[i + half];
+            const float keep = upper ? v[i + half] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+}
+
+template <typename XT, int NE, int RT>
+__global__ void __launch_bounds__(NTHREADS)
+router_small_kernel(const XT* __restrict__ x, const float* __restrict__ W_r,
+                    const float* __restrict__ logit_bias, int T, int d, int E, int K,
+                    int32_t* __restrict__ topk_idx, float* __restrict__ gates,
+                    float* __restrict__ logits_out, float* __restrict__ psum) {
+    extern __shared__ float4 wsm4[];                  // (NE, d) fp32, rows >= E zero
+    float* wsm = reinterpret_cast<float*>(wsm4);
+    __shared__ float lg[TT][32 + 1];
+    constexpr int VEC = sizeof(XT) == 2 ? 8 : 4;      // elements per 16-byte load
+    constexpr int NV = RT * NE;
+    static_assert(NV == 32 || NV == 64, "register tile");
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int t0 = blockIdx.x * TT;
+
+    for (int i = tid; i < NE * d / 4; i += NTHREADS) {
+        const int row = (i * 4) / d;
+        wsm4[i] = row < E ? reinterpret_cast<const float4*>(W_r)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    for (int i = tid; i < TT * 32; i += NTHREADS)
+        if ((i & 31) >= NE) lg[i >> 5][i & 31] = -INFINITY;
+    __syncthreads();
+
+#pragma unroll 1
+    for (int g = warp; g < TT / RT; g += 8) {
+        float acc[NV];
+#pragma unroll
+        for (int i = 0; i < NV; ++i) acc[i] = 0.f;
+        const XT* xr[RT];
+        bool ok[RT];
+#pragma unroll
+        for (int r = 0; r < RT; ++r) {
+            const int t = t0 + g * RT + r;
+            ok[r] = t < T;
+            xr[r] = x + static_cast<size_t>(ok[r] ? t : 0) * d;
+        }
+#pragma unroll 2
+        for (int k = lane * VEC; k < d; k += 32 * VEC) {
+            float xv[RT][VEC];
+#pragma unroll
+            for (int r = 0; r < RT; ++r) {
+                const uint4 raw = ok[r] ? __ldg(reinterpret_cast<const uint4*>(xr[r] + k)) : make_uint4(0, 0, 0, 0);
+                if (VEC == 8) {
+                    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float2 f = __bfloat1622float2(h2[q]);
+                        xv[r][2 * q] = f.x;
+                        xv[r][2 * q + 1] = f.y;
+                    }
+                } else {
+                    const float* f = reinterpret_cast<const float*>(&raw);
+#pragma unroll
+                    for (int q = 0; q < VEC; ++q) xv[r][q] = f[q];
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < NE; ++e) {
+                float w[VEC];
+#pragma unroll
+                for (int q = 0; q < VEC / 4; ++q) {
+                    const float4 w4 = *reinterpret_cast<const float4*>(wsm + static_cast<size_t>(e) * d + k + 4 * q);
+                    w[4 * q] = w4.x; w[4 * q + 1] = w4.y; w[4 * q + 2] = w4.z; w[4 * q + 3] = w4.w;
+                }
+#pragma unroll
+                for (int r = 0; r < RT; ++r)
+#pragma unroll
+                    for (int q = 0; q < VEC; ++q) acc[r * NE + e] = fmaf(xv[r][q], w[q], acc[r * NE + e]);
+            }
+        }
+        warp_reduce_scatter<NV>(acc, lane);
+#pragma unroll
+        for (int i = 0; i < NV / 32; ++i) {
+            const int vi = lane * (NV / 32) + i;
+            const int r = vi / NE, e = vi % NE;
+            lg[g * RT + r][e] = (e < E) ? acc[i] + (logit_bias ? logit_bias[e] : 0.f) : -INFINITY;
+        }
+    }
+    __syncthreads();
+    select_block<1>(&lg[0][0], t0, T, E, K, topk_idx, gates, logits_out, psum);
+}
+
+// ---------------------------------------------------------------- from precomputed logits
+
+template <int EPT>
+__global__ void __launch_bounds__(NTHREADS)
+router_select_kernel(const float* __restrict__ logits, const float* __restrict__ logit_bias, int T, int E, int K,
+                     int32_t* __restrict__ topk_idx, float* __restrict__ gates,
+                     float* __restrict__ logits_out, float* __restrict__ psum) {
+    constexpr int NP = EPT * 32;
+    __shared__ float lg[TT * (NP + 1)];
+    const int t0 = blockIdx.x * TT;
+    for (int i = threadIdx.x; i < TT * NP; i += NTHREADS) {
+        const int r = i / NP, j = i % NP;
+        const int t = t0 + r;
+        float v = -INFINITY;
+        if (j < E && t < T) v = logits[static_cast<size_t>(t) * E + j] + (logit_bias ? logit_bias[j] : 0.f);
+        lg[r * (NP + 1) + j] = v;
+    }
+    __syncthreads();
+    select_block<EPT>(lg, t0, T, E, K, topk_idx, gates, logits_out, psum);
+}
+
+// out[i] = sum_{s < ks} part[s * n + i], in split order.
+__global__ void __launch_bounds__(256)
+router_reduce_kernel(const float* __restrict__ part, int ks, size_t n, float* __restrict__ out) {
+    const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+    for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
+        float s = part[i];
+        for (int k = 1; k < ks; ++k) s += __ldg(part + static_cast<size_t>(k) * n + i);
+        out[i] = s;
+    }
+}
+
 template <typename XT>
-cudaError_t launch_t(const Dims& dm, const void* x, const float* W_r, const float* bias,
-                     int32_t* idx, float* gates, float* logits, float* psum, cudaStream_t st) {
+cudaError_t launch_generic(const Dims& dm, const void* x, const float* W_r, const float* bias,
+                           int32_t* idx, float* gates, float* logits, float* psum, cudaStream_t st) {
     const dim3 grid(dm.route_blocks), block(NTHREADS);
     const XT* xp = static_cast<const XT*>(x);
-    if (dm.E <= 32)
-        router_kernel<XT, 1><<<grid, block, 0, st>>>(xp, W_r, bias, dm.T, dm.d, dm.E, dm.K, idx, gates, logits, psum);
-    else if (dm.E <= 64)
-        router_kernel<XT, 2><<<grid, block, 0, st>>>(xp, W_r, bias, dm.T, dm.d, dm.E, dm.K, idx, gates, logits, psum);
-    else if (dm.E <= 128)
-        router_kernel<XT, 4><<<grid, block, 0, st>>>(xp, W_r, bias, dm.T, dm.d, dm.E, dm.K, idx, gates, logits, psum);
-    else
-        router_kernel<XT, 8><<<grid, block, 0, st>>>(xp, W_r, bias, dm.T, dm.d, dm.E, dm.K, idx, gates, logits, psum);
+#define MOE_GEN(EPT) router_generic_kernel<XT, EPT><<<grid, block, 0, st>>>(xp, W_r, bias, dm.T, dm.d, dm.E, dm.K, idx, gates, logits, psum)
+    if (dm.E <= 32) MOE_GEN(1);
+    else if (dm.E <= 64) MOE_GEN(2);
+    else if (dm.E <= 128) MOE_GEN(4);
+    else MOE_GEN(8);
+#undef MOE_GEN
     return cudaGetLastError();
+}
+
+template <typename XT, int NE, int RT>
+cudaError_t launch_small_t(const Dims& dm, const void* x, const float* W_r, const float* bias,
+                           int32_t* idx, float* gates, float* logits, float* psum, cudaStream_t st) {
+    const size_t smem = static_cast<size_t>(NE) * dm.d * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(router_small_kernel<XT, NE, RT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    router_small_kernel<XT, NE, RT><<<dm.route_blocks, NTHREADS, smem, st>>>(
+        static_cast<const XT*>(x), W_r, bias, dm.T, dm.d, dm.E, dm.K, idx, gates, logits, psum);
+    return cudaGetLastError();
+}
+
+template <typename XT>
+cudaError_t launch_small(const Dims& dm, const void* x, const float* W_r, const float* bias,
+                         int32_t* idx, float* gates, float* logits, float* psum, cudaStream_t st) {
+    if (dm.E <= 8) return launch_small_t<XT, 8, 4>(dm, x, W_r, bias, idx, gates, logits, psum, st);
+    if (dm.E <= 16) return launch_small_t<XT, 16, 4>(dm, x, W_r, bias, idx, gates, logits, psum, st);
+    return launch_small_t<XT, 32, 2>(dm, x, W_r, bias, idx, gates, logits, psum, st);
 }
 
 }  // namespace
 
+bool router_uses_small(const Dims& dm) {
+    const int ne = dm.E <= 8 ? 8 : (dm.E <= 16 ? 16 : 32);
+    return dm.E <= 32 && static_cast<size_t>(ne) * dm.d * 4 <= 160 * 1024;
+}
+
+bool router_uses_tc(const Dims& dm) {
+    return !router_uses_small(dm) && dm.dtype != MOE_F32;
+}
+
 cudaError_t launch_router(const Dims& dm, const void* x, const float* W_r, const float* logit_bias,
                           int32_t* topk_idx, float* gates, float* logits_out, float* psum,
-                          cudaStream_t st) {
-    if (dm.dtype == MOE_F32)
-        return launch_t<float>(dm, x, W_r, logit_bias, topk_idx, gates, logits_out, psum, st);
-    return launch_t<__nv_bfloat16>(dm, x, W_r, logit_bias, topk_idx, gates, logits_out, psum, st);
+                          const RouterScratch& rs, cudaStream_t st) {
+    if (router_uses_small(dm)) {
+        if (dm.dtype == MOE_F32)
+            return launch_small<float>(dm, x, W_r, logit_bias, topk_idx, gates, logits_out, psum, st);
+        return launch_small<__nv_bfloat16>(dm, x, W_r, logit_bias, topk_idx, gates, logits_out, psum, st);
+    }
+    if (!router_uses_tc(dm))
+        return launch_generic<float>(dm, x, W_r, logit_bias, topk_idx, gates, logits_out, psum, st);
+    const RouterTcPlan plan = router_tc_plan(dm);
+    cudaError_t e = launch_router_tc(dm, plan, x, W_r, rs.w3, rs.part, rs.status, st);
+    if (e != cudaSuccess) return e;
+    const float* logits = rs.part;
+    if (plan.ksplit > 1) {
+        const size_t n = static_cast<size_t>(dm.T) * dm.E;
+        int blocks = static_cast<int>((n + 255) / 256);
+        if (blocks > 4 * 148) blocks = 4 * 148;
+        router_reduce_kernel<<<blocks, 256, 0, st>>>(rs.part, plan.ksplit, n, rs.logits);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        logits = rs.logits;
+    }
+    const dim3 grid(dm.route_blocks), block(NTHREADS);
+#define MOE_SEL(EPT) router_select_kernel<EPT><<<grid, block, 0, st>>>(logits, logit_bias, dm.T, dm.E, dm.K, topk_idx, gates, logits_out, psum)
+    if (dm.E <= 32) MOE_SEL(1);
+    else if (dm.E <= 64) MOE_SEL(2);
+    else if (dm.E <= 128) MOE_SEL(4);
+    else MOE_SEL(8);
+#undef MOE_SEL
+    return cudaGetLastError();
 }
 
 }  // namespace moe

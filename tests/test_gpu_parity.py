@@ -26,6 +26,10 @@ CASES = {
     "bf16-k-equals-n": MoEShape("b4", 100, 128, 4, 4, 128, dtype=DTYPE_BF16),
     "bf16-single-expert": MoEShape("b5", 70, 128, 1, 1, 256, dtype=DTYPE_BF16),
     "bf16-one-token": MoEShape("b6", 1, 256, 8, 2, 256, n_shared=1, d_ff_shared=128, dtype=DTYPE_BF16),
+    "f32-generic-router": MoEShape("f32g", 100, 128, 40, 3, 128, dtype=DTYPE_F32),
+    "bf16-e24-small-router": MoEShape("b7", 300, 256, 24, 3, 256, dtype=DTYPE_BF16),
+    "bf16-e128-tc-router": MoEShape("b8", 600, 256, 128, 4, 128, n_shared=1, d_ff_shared=128,
+                                    dtype=DTYPE_BF16),
     "fp8-ragged-shared": MoEShape("f1", 300, 512, 16, 4, 256, n_shared=1, d_ff_shared=384, dtype=DTYPE_FP8),
     "fp8-decode-skewed": MoEShape("f2", 37, 1024, 256, 8, 256, n_shared=1, d_ff_shared=256,
                                   dtype=DTYPE_FP8, zipf_logit_bias=True),
