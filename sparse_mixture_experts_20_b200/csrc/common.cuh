@@ -274,4 +274,10 @@ __device__ __forceinline__ float silu_f32(float z) {
     return z / (1.0f + __expf(-z));
 }
 
+// z * sigmoid(z) with the reciprocal instead of a division (for z -> -inf
+// the exponential overflows to inf and the reciprocal gives 0).
+__device__ __forceinline__ float silu_fast(float z) {
+    return z * __frcp_rn(1.0f + __expf(-z));
+}
+
 }  // namespace moe

@@ -11,23 +11,31 @@
 // row (of A) and per column (of B) per 32 elements of K from tensor memory,
 // and the accumulator sums sa * sb * (a . b) over the whole K loop in fp32.
 //
-// Per CTA (320 threads, one CTA per SM), tiles of 128 rows x 128 weight rows:
-//   warp 0      TMA producer: A and B tiles of 128 rows x 128 bytes (one
-//               scale block of K) into a ring of 6 stages;
+// Tiles are 128 rows x 256 weight rows: one MMA instruction (K = 32) is then
+// about 128 tensor-core cycles of work, enough to hide the cost of issuing
+// it from a single thread.  The 256-column accumulator fills half of tensor
+// memory, so there is one accumulator; the epilogue releases it as soon as
+// it has read the last columns.
+//
+// Per CTA (320 threads, one CTA per SM):
+//   warp 0      TMA producer: A (128 rows x 128 bytes, one scale block of K)
+//               and B (256 rows x 128 bytes) into a ring of 4 stages;
 //   warp 1      MMA issuer: per stage 4 x tcgen05.mma (K = 32 each) with the
-//               scale factors of that stage, accumulating in one of two
-//               128-column TMEM buffers;
+//               scale factors of that stage;
 //   warps 2..5  epilogue: tcgen05.ld (thread = row), bias, SiLU and the
 //               per-row e4m3 re-quantisation of the hidden activation (one
-//               128-column scale block per row and tile, so the amax is
-//               thread-local), or bias and bf16 output;
-//   warps 6..9  scale-factor writers: per stage, load the 128 row scales of
-//               A and the block scale of B (prefetched 8 stages ahead),
-//               convert to UE8M0 and tcgen05.st them into a ring of 8
-//               tensor-memory slots.  Each slot holds, in every lane quadrant,
-//               lane m: columns c = 0..3 = the scale of row 32c + m (A) and of
-//               weight row 32c + m (B), each byte repeated for the four
-//               32-element sub-blocks of K.
+//               scale per row per 128 columns, so the amax is thread-local),
+//               or bias and bf16 output;
+//   warps 6..9  scale-factor writers: per stage, the 128 row scales of A and
+//               the two block scales of B (prefetched 8 stages ahead) as
+//               UE8M0, written with tcgen05.st into the stage's slot of
+//               tensor memory; they arrive on the stage's full barrier next to
+//               the TMA bytes, and wait on its empty barrier like the
+//               producer.  Slot layout, in every lane quadrant, lane m:
+//               columns c = 0..3 hold the scale of A row 32c + m, columns
+//               4 + c and 8 + c the scale of weight row 32c + m and
+//               128 + 32c + m, each byte repeated for the four 32-element
+//               sub-blocks of K.
 // Every wait is bounded (common.cuh).
 #include "ffn_common.cuh"
 
@@ -37,9 +45,11 @@ namespace {
 using namespace ffn;
 
 constexpr int NUM_THREADS = 320;
-constexpr int BN = 128, BK = 128, STAGES = 6, ACC_BUFS = 2, SF_SLOTS = 8, LOOKAHEAD = 8;
+constexpr int BN = 256, BK = 128, STAGES = 4, LOOKAHEAD = 8;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t SF_COL0 = ACC_BUFS * BN;          // scale-factor slots after the accumulators
+constexpr uint32_t SF_COL0 = BN;                     // scale-factor slots after the accumulator
+constexpr uint32_t SF_STRIDE = 16;                   // columns per stage slot (4 A + 8 B, padded)
+constexpr uint32_t FULL_ARRIVALS = 1 + 4;            // TMA expect_tx + one lane per scale-factor warp
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
 constexpr uint64_t kDrainTimeoutNs = 200000000ull;
 
@@ -49,8 +59,8 @@ struct Smem {
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
     static constexpr int OFF_BAR = OFF_B + STAGES * B_BYTES;
-    // full, empty [STAGES]; accf, acce [ACC_BUFS]; sff, sfe [SF_SLOTS]; drain
-    static constexpr int N_BARS = 2 * STAGES + 2 * ACC_BUFS + 2 * SF_SLOTS + 1;
+    // full, empty [STAGES]; accf, acce; drain
+    static constexpr int N_BARS = 2 * STAGES + 2 + 1;
     static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
     static constexpr int OFF_SEG = OFF_MISC + 16;
     static constexpr int TOTAL = OFF_SEG + SegTable::SEG_INTS * 4;
@@ -78,10 +88,8 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
     uint64_t* full = bars;
     uint64_t* empty = full + STAGES;
     uint64_t* accf = empty + STAGES;
-    uint64_t* acce = accf + ACC_BUFS;
-    uint64_t* sff = acce + ACC_BUFS;
-    uint64_t* sfe = sff + SF_SLOTS;
-    uint64_t* drain = sfe + SF_SLOTS;
+    uint64_t* acce = accf + 1;
+    uint64_t* drain = acce + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
     SegTable seg(reinterpret_cast<int*>(smem + L::OFF_SEG));
@@ -89,9 +97,9 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
 
     if (warp == 0) tmem_alloc<TMEM_COLS>(tmem_slot);
     if (warp == 1 && lane == 0) {
-        for (int i = 0; i < STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-        for (int i = 0; i < ACC_BUFS; ++i) { mbar_init(&accf[i], 1); mbar_init(&acce[i], 128); }
-        for (int i = 0; i < SF_SLOTS; ++i) { mbar_init(&sff[i], 128); mbar_init(&sfe[i], 1); }
+        for (int i = 0; i < STAGES; ++i) { mbar_init(&full[i], FULL_ARRIVALS); mbar_init(&empty[i], 1); }
+        mbar_init(accf, 1);
+        mbar_init(acce, 128);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -142,34 +150,30 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
         // ================= MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = make_idesc_mxf8(BM, BN);
-            int stage = 0, abuf = 0, sslot = 0;
-            uint32_t phase = 0, aphase = 0, sphase = 0;
+            int stage = 0;
+            uint32_t phase = 0, aphase = 0;
             bool ok = true, issued_any = false;
             for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
                 const TileInfo ti = decode_tile<BN, BK>(tile, p, seg, nseg);
-                if (!mbar_wait_bounded(&acce[abuf], aphase ^ 1u, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
+                if (!mbar_wait_bounded(acce, aphase ^ 1u, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * BN);
                 for (int kb = 0; kb < ti.kblocks; ++kb) {
                     if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
-                    if (!mbar_wait_bounded(&sff[sslot], sphase, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t adesc = smem_desc_k_sw128(smem + L::OFF_A + stage * L::A_BYTES);
                     const uint64_t bdesc = smem_desc_k_sw128(smem + L::OFF_B + stage * L::B_BYTES);
-                    const uint32_t sfa = tmem_base + SF_COL0 + static_cast<uint32_t>(sslot * 8);
+                    const uint32_t sfa = tmem_base + SF_COL0 + static_cast<uint32_t>(stage) * SF_STRIDE;
 #pragma unroll
                     for (int k = 0; k < 4; ++k)            // 4 x 32 e4m3 of K per stage
-                        umma_mxf8_bs(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, sfa, sfa + 4,
+                        umma_mxf8_bs(tmem_base, adesc + 2 * k, bdesc + 2 * k, idesc, sfa, sfa + 4,
                                      (kb > 0 || k > 0) ? 1u : 0u);
                     issued_any = true;
-                    umma_commit(&empty[stage]);
-                    umma_commit(&sfe[sslot]);
+                    umma_commit(&empty[stage]);             // frees the smem stage and its scale slot
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-                    if (++sslot == SF_SLOTS) { sslot = 0; sphase ^= 1u; }
                 }
                 if (!ok) break;
-                umma_commit(&accf[abuf]);
-                if (++abuf == ACC_BUFS) { abuf = 0; aphase ^= 1u; }
+                umma_commit(accf);
+                aphase ^= 1u;
             }
             if (!ok && issued_any) {
                 umma_commit(drain);
@@ -183,63 +187,72 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
         const int quad = warp & 3;
         const int r_local = quad * 32 + lane;
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
-        int abuf = 0;
         uint32_t aphase = 0;
         for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
             const TileInfo ti = decode_tile<BN, BK>(tile, p, seg, nseg);
             const GroupDev& g = p.g[ti.grp];
             const bool row_ok = r_local < ti.rows_left;
-            if (!warp_wait(&accf[abuf], aphase, abort_flag, p.status, p.timeout_ns, lane)) break;
+            if (!warp_wait(accf, aphase, abort_flag, p.status, p.timeout_ns, lane)) break;
+            aphase ^= 1u;
             tc_fence_after();
             const float* bias = g.bias + static_cast<size_t>(ti.mat) * g.N + ti.n0;
-            const uint32_t acc_col = static_cast<uint32_t>(abuf * BN);
             if (p.out_fp8) {
-                // first layer: bias + SiLU, then one e4m3 block of 128 columns per row
-                float v[BN];
+                // first layer: bias + SiLU, then one e4m3 block per 128 columns per row
+#pragma unroll 1
+                for (int h = 0; h < BN / 128; ++h) {
+                    float v[128];
 #pragma unroll
-                for (int c = 0; c < BN / 32; ++c) {
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(lane_base + acc_col + static_cast<uint32_t>(c * 32), r);
-                    tmem_ld_wait();
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t r[32];
+                        tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>(h * 128 + c * 32), r);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) v[c * 32 + j] = __uint_as_float(r[j]);
-                }
-                tc_fence_before();
-                mbar_arrive(&acce[abuf]);                    // accumulator copied out
-                if (row_ok) {
+                        for (int j = 0; j < 32; ++j) v[c * 32 + j] = __uint_as_float(r[j]);
+                    }
+                    if (h == BN / 128 - 1) {                 // accumulator fully read: release it
+                        tc_fence_before();
+                        mbar_arrive(acce);
+                    }
+                    const int n_blk = ti.n0 + h * 128;
+                    if (!row_ok || n_blk >= g.N) continue;
                     float amax = 0.f;
 #pragma unroll
-                    for (int j = 0; j < BN; ++j) {
-                        v[j] = silu_f32(v[j] + __ldg(bias + j));
+                    for (int j = 0; j < 128; ++j) {
+                        v[j] = silu_f32(v[j] + __ldg(bias + h * 128 + j));
                         amax = fmaxf(amax, fabsf(v[j]));
                     }
                     const float sc = pow2_scale_448(amax);
                     const float inv = 1.0f / sc;             // exact: sc is a power of two
-                    uint8_t* crow = static_cast<uint8_t*>(g.C) + static_cast<size_t>(ti.c_row + r_local) * g.N + ti.n0;
+                    uint8_t* crow = static_cast<uint8_t*>(g.C) + static_cast<size_t>(ti.c_row + r_local) * g.N + n_blk;
 #pragma unroll
-                    for (int q = 0; q < BN / 16; ++q) {
+                    for (int q = 0; q < 8; ++q) {
                         uint32_t w[4];
 #pragma unroll
-                        for (int h = 0; h < 4; ++h) {
-                            const int j = q * 16 + h * 4;
+                        for (int hh = 0; hh < 4; ++hh) {
+                            const int j = q * 16 + hh * 4;
                             const uint32_t lo = f32x2_to_e4m3x2(v[j] * inv, v[j + 1] * inv);
                             const uint32_t hi = f32x2_to_e4m3x2(v[j + 2] * inv, v[j + 3] * inv);
-                            w[h] = lo | (hi << 16);
+                            w[hh] = lo | (hi << 16);
                         }
                         reinterpret_cast<uint4*>(crow)[q] = make_uint4(w[0], w[1], w[2], w[3]);
                     }
-                    g.c_scales[static_cast<size_t>(ti.c_row + r_local) * (g.N / 128) + ti.n0 / 128] = sc;
+                    g.c_scales[static_cast<size_t>(ti.c_row + r_local) * (g.N / 128) + n_blk / 128] = sc;
                 }
             } else {
                 // second layer: bias, bf16 output
                 __nv_bfloat16* crow = static_cast<__nv_bfloat16*>(g.C) +
                                       static_cast<size_t>(ti.c_row + r_local) * g.N + ti.n0;
+                const int n_valid = min(BN, g.N - ti.n0);
 #pragma unroll 1
                 for (int c = 0; c < BN / 32; ++c) {
                     uint32_t r[32];
-                    tmem_ld_32x32b_x32(lane_base + acc_col + static_cast<uint32_t>(c * 32), r);
+                    tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>(c * 32), r);
                     tmem_ld_wait();
-                    if (row_ok) {
+                    if (c == BN / 32 - 1) {                  // accumulator fully read: release it
+                        tc_fence_before();
+                        mbar_arrive(acce);
+                    }
+                    if (row_ok && c * 32 < n_valid) {
                         uint32_t packed[16];
 #pragma unroll
                         for (int j = 0; j < 16; ++j) {
@@ -254,10 +267,7 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
                             dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
                     }
                 }
-                tc_fence_before();
-                mbar_arrive(&acce[abuf]);
             }
-            if (++abuf == ACC_BUFS) { abuf = 0; aphase ^= 1u; }
         }
     } else {
         // ================= scale-factor writers (warps 6..9)
@@ -276,7 +286,8 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
                 if (it.tile < total_tiles) it.ti = decode_tile<BN, BK>(it.tile, p, seg, nseg);
             }
         };
-        auto load = [&](const ItemIt& it, float (&a)[4], float& b) {
+        // A: the scales of rows 32c + lane; B: the two weight blocks of the tile
+        auto load = [&](const ItemIt& it, float (&a)[4], float (&b)[2]) {
             const GroupDev& g = p.g[it.ti.grp];
             const int kq = g.K / 128;
             const int rows_valid = min(BM, it.ti.rows_left);
@@ -285,18 +296,23 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
                 const int r = 32 * c + lane;
                 a[c] = (r < rows_valid) ? __ldg(g.a_scales + static_cast<size_t>(it.ti.a_row + r) * kq + it.kb) : 1.0f;
             }
-            b = __ldg(g.b_scales + (static_cast<size_t>(it.ti.mat) * (g.N / 128) + it.ti.n0 / 128) * kq + it.kb);
+            const int nb = g.N / 128;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int blk = it.ti.n0 / 128 + h;
+                b[h] = (blk < nb) ? __ldg(g.b_scales + (static_cast<size_t>(it.ti.mat) * nb + blk) * kq + it.kb) : 1.0f;
+            }
         };
         ItemIt cur, ahead;
         start(cur);
         start(ahead);
-        float ra[LOOKAHEAD][4], rb[LOOKAHEAD];
+        float ra[LOOKAHEAD][4], rb[LOOKAHEAD][2];
 #pragma unroll
         for (int j = 0; j < LOOKAHEAD; ++j) {
             if (valid(ahead)) { load(ahead, ra[j], rb[j]); advance(ahead); }
         }
-        int sslot = 0;
-        uint32_t sphase = 0;
+        int stage = 0;
+        uint32_t phase = 0;
         bool ok = true;
         while (ok && valid(cur)) {
 #pragma unroll
@@ -304,16 +320,19 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
                 if (!valid(cur)) break;
                 const uint32_t wa0 = ue8m0_x4(ra[j][0]), wa1 = ue8m0_x4(ra[j][1]);
                 const uint32_t wa2 = ue8m0_x4(ra[j][2]), wa3 = ue8m0_x4(ra[j][3]);
-                const uint32_t wb = ue8m0_x4(rb[j]);
+                const uint32_t wb0 = ue8m0_x4(rb[j][0]), wb1 = ue8m0_x4(rb[j][1]);
                 if (valid(ahead)) { load(ahead, ra[j], rb[j]); advance(ahead); }
-                if (!warp_wait(&sfe[sslot], sphase ^ 1u, abort_flag, p.status, p.timeout_ns, lane)) { ok = false; break; }
+                if (!warp_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, p.timeout_ns, lane)) { ok = false; break; }
                 tc_fence_after();
-                tmem_st_32x32b_x4(sf_base + static_cast<uint32_t>(sslot * 8), wa0, wa1, wa2, wa3);
-                tmem_st_32x32b_x4(sf_base + static_cast<uint32_t>(sslot * 8 + 4), wb, wb, wb, wb);
+                const uint32_t slot = sf_base + static_cast<uint32_t>(stage) * SF_STRIDE;
+                tmem_st_32x32b_x4(slot, wa0, wa1, wa2, wa3);
+                tmem_st_32x32b_x4(slot + 4, wb0, wb0, wb0, wb0);
+                tmem_st_32x32b_x4(slot + 8, wb1, wb1, wb1, wb1);
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(&sff[sslot]);
-                if (++sslot == SF_SLOTS) { sslot = 0; sphase ^= 1u; }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full[stage]);
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 advance(cur);
             }
         }

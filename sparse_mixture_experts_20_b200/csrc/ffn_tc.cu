@@ -7,13 +7,14 @@
 // segment list of ffn_common.cuh (routed experts from the device-side
 // dispatch offsets, then the shared experts), so the host never synchronises.
 //
-// Per CTA (192 threads, one CTA per SM):
+// Per CTA (320 threads, one CTA per SM):
 //   warp 0      TMA producer: A tile (128 rows x 64 bf16) and B tile
 //               (256 rows x 64 bf16), 128-byte swizzle, into a ring of 4
 //               shared-memory stages guarded by full/empty mbarriers;
 //   warp 1      MMA issuer: one thread issues tcgen05.mma (M=128, N=256, K=16)
 //               into tensor memory and frees each stage with tcgen05.commit;
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (thread = row),
+//   warps 2..9  epilogue: tcgen05.ld of the accumulator (thread = row; the
+//               warps of a lane quadrant split the 256 columns in halves),
 //               bias, SiLU, bf16 rounding and 16-byte stores.
 // Two 256-column accumulators in tensor memory let the epilogue of tile i
 // overlap the MMAs of tile i+1.  Rows of a tile past the end of its segment
@@ -30,7 +31,8 @@ namespace {
 
 using namespace ffn;
 
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;
+constexpr int EPI_THREADS = 256;
 constexpr int BN = 256, BK = 64, STAGES = 4, ACC_BUFS = 2;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;    // 2 s per wait
@@ -72,7 +74,7 @@ grouped_ffn_bf16_kernel(const __grid_constant__ TcParams p) {
     if (warp == 0) tmem_alloc<TMEM_COLS>(tmem_slot);
     if (warp == 1 && lane == 0) {
         for (int i = 0; i < STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-        for (int i = 0; i < ACC_BUFS; ++i) { mbar_init(&accf[i], 1); mbar_init(&acce[i], 128); }
+        for (int i = 0; i < ACC_BUFS; ++i) { mbar_init(&accf[i], 1); mbar_init(&acce[i], EPI_THREADS); }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -158,8 +160,9 @@ grouped_ffn_bf16_kernel(const __grid_constant__ TcParams p) {
         }
         __syncwarp();
     } else {
-        // ================= epilogue (warps 2..5; TMEM lane quadrant = warp % 4)
+        // ================= epilogue (warps 2..9; TMEM lane quadrant = warp % 4)
         const int quad = warp & 3;
+        const int half = (warp - 2) >> 2;                 // which 128 of the 256 columns
         const int r_local = quad * 32 + lane;
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
         int abuf = 0;
@@ -175,19 +178,31 @@ grouped_ffn_bf16_kernel(const __grid_constant__ TcParams p) {
                                   static_cast<size_t>(ti.c_row + r_local) * g.N + ti.n0;
             const float* bias = g.bias + static_cast<size_t>(ti.mat) * g.N + ti.n0;
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>(abuf * BN + c * 32), r);
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c0 = half * 4 + cc * 2;         // two 32-column chunks in flight
+                uint32_t r[2][32];
+                tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>(abuf * BN + c0 * 32), r[0]);
+                tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>(abuf * BN + c0 * 32 + 32), r[1]);
                 tmem_ld_wait();
-                if (row_ok && c * 32 < n_valid) {
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int c = c0 + u;
+                    if (!row_ok || c * 32 >= n_valid) continue;
                     uint32_t packed[16];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        float v0 = __uint_as_float(r[2 * j]) + __ldg(bias + c * 32 + 2 * j);
-                        float v1 = __uint_as_float(r[2 * j + 1]) + __ldg(bias + c * 32 + 2 * j + 1);
-                        if (p.silu) { v0 = silu_f32(v0); v1 = silu_f32(v1); }
-                        __nv_bfloat162 h2 = __floats2bfloat162_rn(v0, v1);
-                        packed[j] = *reinterpret_cast<uint32_t*>(&h2);
+                    for (int j4 = 0; j4 < 8; ++j4) {
+                        const float4 b4 = __ldg(reinterpret_cast<const float4*>(bias + c * 32) + j4);
+                        float v0 = __uint_as_float(r[u][4 * j4 + 0]) + b4.x;
+                        float v1 = __uint_as_float(r[u][4 * j4 + 1]) + b4.y;
+                        float v2 = __uint_as_float(r[u][4 * j4 + 2]) + b4.z;
+                        float v3 = __uint_as_float(r[u][4 * j4 + 3]) + b4.w;
+                        if (p.silu) {
+                            v0 = silu_fast(v0); v1 = silu_fast(v1); v2 = silu_fast(v2); v3 = silu_fast(v3);
+                        }
+                        __nv_bfloat162 h01 = __floats2bfloat162_rn(v0, v1);
+                        __nv_bfloat162 h23 = __floats2bfloat162_rn(v2, v3);
+                        packed[2 * j4] = *reinterpret_cast<uint32_t*>(&h01);
+                        packed[2 * j4 + 1] = *reinterpret_cast<uint32_t*>(&h23);
                     }
                     uint4* dst = reinterpret_cast<uint4*>(crow + c * 32);
 #pragma unroll
