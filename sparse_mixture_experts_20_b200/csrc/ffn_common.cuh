@@ -65,8 +65,9 @@ struct SegTable {
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 // Builds the table cooperatively (all threads of the block call it; ends with
-// the scan done by warp 0 -- the caller synchronises afterwards).
-template <int BN>
+// the scan done by warp 0 -- the caller synchronises afterwards).  A
+// scheduled tile covers MGROUP consecutive m-tiles (2 for CTA pairs).
+template <int BN, int MGROUP = 1>
 __device__ __forceinline__ int build_seg_table(const TcParams& p, SegTable& t, int nthreads) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n0segs = p.g[0].n_mats, n1segs = p.g[1].n_mats;
@@ -94,7 +95,7 @@ __device__ __forceinline__ int build_seg_table(const TcParams& p, SegTable& t, i
         t.arow[s] = arow;
         t.crow[s] = crow;
         t.mat[s] = packed;
-        t.start[s + 1] = ceil_div(rows, BM) * ceil_div(N, BN);     // tile count, scanned below
+        t.start[s + 1] = ceil_div(ceil_div(rows, BM), MGROUP) * ceil_div(N, BN);   // tile count, scanned below
     }
     __syncthreads();
     if (warp == 0) {                                                // inclusive scan of tile counts
@@ -115,8 +116,11 @@ __device__ __forceinline__ int build_seg_table(const TcParams& p, SegTable& t, i
     return nseg;
 }
 
-template <int BN, int BK>
-__device__ __forceinline__ TileInfo decode_tile(int tile, const TcParams& p, const SegTable& t, int nseg) {
+// Tile `tile` of the table; with MGROUP > 1 the m-tile is MGROUP * group + sub
+// (rows_left <= 0 when that m-tile lies past the segment's end).
+template <int BN, int BK, int MGROUP = 1>
+__device__ __forceinline__ TileInfo decode_tile(int tile, const TcParams& p, const SegTable& t, int nseg,
+                                                int sub = 0) {
     int lo = 0, hi = nseg - 1;                      // last s with start[s] <= tile
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -124,8 +128,8 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const TcParams& p, con
     }
     const int s = lo;
     const int local = tile - t.start[s];
-    const int mtiles = ceil_div(t.rows[s], BM);
-    const int nt = local / mtiles, mt = local % mtiles;
+    const int mgroups = ceil_div(ceil_div(t.rows[s], BM), MGROUP);
+    const int nt = local / mgroups, mt = (local % mgroups) * MGROUP + sub;
     TileInfo ti;
     ti.grp = t.mat[s] >> 16;
     ti.mat = t.mat[s] & 0xFFFF;

@@ -119,6 +119,9 @@ struct GemmArgs {
 
 cudaError_t launch_grouped_ffn_f32(const Dims& dm, const GemmArgs& a, cudaStream_t st);
 cudaError_t launch_grouped_ffn_bf16(const Dims& dm, const GemmArgs& a, cudaStream_t st);
+cudaError_t launch_grouped_ffn_bf16_pair(const Dims& dm, const GemmArgs& a, cudaStream_t st);
+// CTA-pair kernels are used unless the environment variable MOE_GEMM_PAIR is "0".
+bool gemm_pairs_enabled();
 cudaError_t launch_grouped_ffn_fp8(const Dims& dm, const GemmArgs& a, cudaStream_t st);
 
 cudaError_t launch_wait_selftest(int64_t timeout_ns, int32_t* status, cudaStream_t st);

@@ -196,8 +196,13 @@ int run_expert_ffn(const Dims& dm, const WsLayout& L, const void* x, const void*
         e = launch_grouped_ffn_f32(dm, g1, st);
         if (e == cudaSuccess) e = launch_grouped_ffn_f32(dm, g2, st);
     } else if (dm.dtype == MOE_BF16) {
-        e = launch_grouped_ffn_bf16(dm, g1, st);
-        if (e == cudaSuccess) e = launch_grouped_ffn_bf16(dm, g2, st);
+        if (gemm_pairs_enabled()) {
+            e = launch_grouped_ffn_bf16_pair(dm, g1, st);
+            if (e == cudaSuccess) e = launch_grouped_ffn_bf16_pair(dm, g2, st);
+        } else {
+            e = launch_grouped_ffn_bf16(dm, g1, st);
+            if (e == cudaSuccess) e = launch_grouped_ffn_bf16(dm, g2, st);
+        }
     } else {
         e = launch_grouped_ffn_fp8(dm, g1, st);
         if (e == cudaSuccess) e = launch_grouped_ffn_fp8(dm, g2, st);
