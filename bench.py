@@ -37,8 +37,12 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer tokens/s; grouped-GEMM TFLOP/s and HBM GB/s as % of B200 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-CPU_SAMPLE = {1: 64, 2: 256, 3: 256, 4: 64, 5: 128}     # oracle tokens per baseline sample
-REF_SAMPLE = {1: 64, 2: 32, 3: 64, 4: 16, 5: 32}         # oracle tokens per reference step
+# Oracle tokens per CPU-baseline sample (about 10-30 s of host work; the whole
+# batch where that fits) and per step of the reference arm (a fraction of a
+# second to a few seconds, so that a default --steps/--warmup run of the
+# reference arm ends within a few minutes).
+CPU_SAMPLE = {1: 64, 2: 4096, 3: 8192, 4: 16, 5: 64}
+REF_SAMPLE = {1: 64, 2: 32, 3: 64, 4: 1, 5: 4}
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -51,7 +55,24 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
+                    help="override a field of the workload shape (e.g. n_routed=64); for profiling "
+                         "reduced cases, never for the reported workload")
     return ap.parse_args()
+
+
+def workload(args):
+    from synthetic import CONFIGS
+    sh = CONFIGS[args.config]
+    if args.set:
+        kw = {}
+        for item in args.set:
+            k, v = item.split("=", 1)
+            cur = getattr(sh, k)
+            kw[k] = type(cur)(float(v)) if isinstance(cur, (int, float)) and not isinstance(cur, bool) else type(cur)(v)
+        sh = sh.replace(**kw)
+        sh = sh.replace(name=sh.name + " [" + ",".join(args.set) + "]")
+    return sh
 
 
 def load_peaks():
@@ -66,7 +87,8 @@ def workload_config(sh, seed, parallelism):
     return {"workload": sh.name, "T": sh.T, "d_model": sh.d_model, "n_routed": sh.n_routed,
             "top_k": sh.top_k, "d_ff": sh.d_ff, "n_shared": sh.n_shared, "d_ff_shared": sh.d_ff_shared,
             "capacity_factor": sh.capacity_factor, "seed": seed, "parallelism": parallelism,
-            "l2": "flushed between timed steps (256 MiB write)"}
+            "l2": ("n/a (host oracle)" if parallelism == "cpu"
+                   else "flushed between timed steps (256 MiB write)")}
 
 
 def dtype_name(sh):
@@ -132,7 +154,20 @@ class ClockSampler:
 # ----------------------------------------------------------------------------- oracle timing
 
 def oracle_inputs_on_host(inp):
-    return {k: (None if v is None else v.detach().cpu()) for k, v in inp.items()}
+    """The inputs as the oracle reads them: on the host, fp32/bf16 values
+    widened to fp64 numpy once (exact) so that the timed oracle calls do not
+    re-convert the weights each step; FP8 codes stay as stored (their decode
+    and block scaling are part of what the oracle computes)."""
+    import torch
+    out = {}
+    for k, v in inp.items():
+        if v is None:
+            out[k] = None
+        elif v.dtype in (torch.float32, torch.bfloat16, torch.float16):
+            out[k] = v.detach().to("cpu", torch.float64).numpy()
+        else:
+            out[k] = v.detach().cpu()
+    return out
 
 
 def time_oracle(sh, host_inp, n_tokens, seed):
@@ -181,25 +216,42 @@ def ffn_bytes(sh, kept):
     return float(w + act), touched
 
 
-def traffic_from_profile(kernel_src_hash, cid):
-    """dram bytes per FFN launch pair from the committed ncu summary, valid only
-    while the kernel source is unchanged since the capture."""
+CSRC = os.path.join(ROOT, "sparse_mixture_experts_20_b200", "csrc")
+
+
+def ffn_kernel(sh):
+    """(kernel name, source files) of the grouped FFN kernel the library runs
+    for this dtype (the bf16 CTA-pair kernel unless MOE_GEMM_PAIR=0)."""
+    if sh.dtype == 0:
+        return "ffn_f32_kernel", ["ffn_f32.cu"]
+    if sh.dtype == 2:
+        return "grouped_ffn_fp8_kernel", ["ffn_fp8.cu", "ffn_common.cuh", "common.cuh"]
+    if os.environ.get("MOE_GEMM_PAIR", "1") == "0":
+        return "grouped_ffn_bf16_kernel", ["ffn_tc.cu", "ffn_common.cuh", "common.cuh"]
+    return "grouped_ffn_bf16_pair_kernel", ["ffn_tc2.cu", "ffn_common.cuh", "common.cuh"]
+
+
+def src_hash(files):
+    h = hashlib.sha1()
+    for f in files:
+        h.update(open(os.path.join(CSRC, f), "rb").read())
+    return h.hexdigest()
+
+
+def traffic_from_profile(workload_name, kernel, sha):
+    """DRAM bytes (read + write) of the grouped FFN launches of one step, from
+    the committed ncu summary; None unless it was captured on this workload
+    with the kernel sources unchanged since."""
     p = os.path.join(ROOT, "profiles", "grouped_ffn_traffic.json")
     if not os.path.exists(p):
         return None
     try:
-        d = json.load(open(p))
-        e = d.get(str(cid))
-        if e and e.get("ffn_tc_sha1") == kernel_src_hash:
-            return e.get("dram_bytes_per_step")
+        for e in json.load(open(p)).get("entries", []):
+            if e.get("workload") == workload_name and e.get("kernel") == kernel and e.get("src_sha1") == sha:
+                return e.get("dram_bytes_per_step")
     except Exception:
         return None
     return None
-
-
-def ffn_src_hash():
-    src = os.path.join(ROOT, "sparse_mixture_experts_20_b200", "csrc", "ffn_tc.cu")
-    return hashlib.sha1(open(src, "rb").read()).hexdigest()
 
 
 def run_ours(args):
@@ -220,7 +272,7 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    sh = CONFIGS[args.config]
+    sh = workload(args)
     M.lib()
     inp = make_inputs(sh, seed=args.seed + rank, device=dev)
     cfg = M.make_config(sh)
@@ -245,7 +297,6 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     n_stage = 5
-    launches_per_step = 1 + 3 + 2 + 1 + 1
 
     def step(ev):
         ev[0].record(stream)
@@ -279,10 +330,12 @@ def run_ours(args):
     barrier()
     torch.cuda.synchronize(dev)
     sampler.mark()
+    launches0 = M.moe_kernel_launches()
     for k in range(args.steps):
         flush.zero_()
         step(evs[k])
     torch.cuda.synchronize(dev)
+    launches = M.moe_kernel_launches() - launches0
     sampler.mark()
     barrier()
     stage_ms = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(n_stage)]
@@ -341,10 +394,11 @@ def run_ours(args):
         ach = fbytes / (ffn_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(ach / peaks["hbm_gbs"], 4)}
-    roof["kernel"] = "grouped_ffn_tc_kernel (first + second layer launches, per step)"
+    kname, kfiles = ffn_kernel(sh)
+    roof["kernel"] = f"{kname} (both launches of a step: first and second layer)"
     roof["peak_source"] = (f"{peak_src} ({'bf16 burst x2 nominal fp8/bf16 ratio' if fp8 else 'bf16 burst'})"
                            if roof["bound"] == "tensor" else f"{peak_src} HBM copy")
-    roof["traffic"] = traffic_from_profile(ffn_src_hash(), args.config)
+    roof["traffic"] = traffic_from_profile(sh.name, kname, src_hash(kfiles))
     roof["algorithmic"] = {"flops": flops, "bytes": fbytes, "experts_touched": touched}
 
     n_tok = T * world * args.steps
@@ -363,7 +417,7 @@ def run_ours(args):
         "e2e": {"value": round(T * world * args.steps / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(inp["x"].numel() * inp["x"].element_size()),
                 "d2h_bytes_per_step": int(T * d * (4 if sh.dtype == 0 else 2) + 4)},
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": launches,
         "routing": {"max_load": int(counts.max()), "mean_load": float(counts.mean()),
                     "experts_touched": int((counts > 0).sum()), "dropped": int(counts.sum() - kept.sum())},
         "device_status": status,
@@ -374,7 +428,8 @@ def run_ours(args):
         n, dt = time_oracle(sh, host, CPU_SAMPLE[args.config], args.seed)
         line["cpu_baseline"] = {"value": round(n / dt, 3), "unit": "tokens/s", "cores": oracle_threads(),
                                 "kind": "oracle",
-                                "sample": f"{n} of {T} tokens (routing of all {T}), fp64 numpy, {dt:.1f} s"}
+                                "sample": f"{n} of {T} tokens (routing of all {T}), fp64 numpy, {dt:.1f} s; "
+                                          "fp32/bf16 inputs widened to fp64 once before timing"}
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
@@ -388,8 +443,8 @@ def run_reference(args):
     if rank != 0:
         return
     import torch
-    from synthetic import CONFIGS, make_inputs
-    sh = CONFIGS[args.config]
+    from synthetic import make_inputs
+    sh = workload(args)
     gen_dev = "cuda" if torch.cuda.is_available() else "cpu"
     host = oracle_inputs_on_host(make_inputs(sh, seed=args.seed, device=gen_dev))
     n_tok = REF_SAMPLE[args.config]
@@ -402,7 +457,8 @@ def run_reference(args):
         total_n += n
     value = total_n / total_t
     cores = oracle_threads()
-    sample = f"{n_tok} of {sh.T} tokens per step (routing of all {sh.T}), fp64 numpy"
+    sample = (f"{n_tok} of {sh.T} tokens per step (routing of all {sh.T}), fp64 numpy, "
+              "fp32/bf16 inputs widened to fp64 once before timing")
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1000 * total_t / args.steps, 2),

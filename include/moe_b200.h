@@ -140,6 +140,13 @@ MOE_EXPORT int moe_last_cuda_error(void);
 /* Human-readable name of a MOE_* status code (static string). */
 MOE_EXPORT const char* moe_status_string(int status);
 
+/* Number of CUDA kernels this library has launched in this process, on every
+ * device and stream, since it was loaded (a launch counts when it is issued,
+ * whether or not it later fails).  Thread-safe; read it before and after a
+ * sequence of calls to learn how many kernels the sequence launched.  Not a
+ * step of the method: bookkeeping for benchmarks. */
+MOE_EXPORT uint64_t moe_kernel_launches(void);
+
 /* ---- stage 1: router ------------------------------------------------------
  * l[t,j] = sum_i x[t,i] W_r[j,i] (+ logit_bias[j]) in fp32; s = softmax(l);
  * topk_idx[t,k] = the K largest l (ties -> lower j), descending;

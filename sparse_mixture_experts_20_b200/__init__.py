@@ -34,7 +34,7 @@ EXPORTED = (
     "moe_workspace_size", "moe_buffer_rows", "moe_workspace_init", "moe_get_device_status",
     "moe_last_cuda_error", "moe_status_string", "moe_route", "moe_dispatch", "moe_expert_ffn",
     "moe_combine", "moe_balance_stats", "moe_layer_forward", "moe_selftest_wait_timeout",
-    "moe_dispatch_noalloc",
+    "moe_dispatch_noalloc", "moe_kernel_launches",
 )
 
 
@@ -87,11 +87,13 @@ def lib() -> ctypes.CDLL:
             "moe_layer_forward": [cfgp] + [P] * 24,
             "moe_selftest_wait_timeout": [cfgp, ctypes.c_int64, P, P],
             "moe_dispatch_noalloc": [cfgp, P, P, P, P, P, P, P, P, P, P],
+            "moe_kernel_launches": [],
         }
+        restype = {"moe_status_string": ctypes.c_char_p, "moe_kernel_launches": ctypes.c_uint64}
         for name, args in sig.items():
             fn = getattr(L, name)
             fn.argtypes = args
-            fn.restype = ctypes.c_char_p if name == "moe_status_string" else I
+            fn.restype = restype.get(name, I)
         _LIB = L
     return _LIB
 
@@ -156,6 +158,11 @@ def moe_get_device_status(cfg, ws, stream=None, clear: bool = False) -> int:
     _check(lib().moe_get_device_status(ctypes.byref(cfg), _p(ws), _stream(stream), ctypes.byref(st),
                                        1 if clear else 0), "moe_get_device_status")
     return st.value
+
+
+def moe_kernel_launches() -> int:
+    """Kernels the library has launched in this process since it was loaded."""
+    return int(lib().moe_kernel_launches())
 
 
 def moe_route(cfg, x, W_r, logit_bias, topk_idx, gates, logits_out, ws, stream=None):

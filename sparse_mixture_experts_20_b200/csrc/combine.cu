@@ -129,12 +129,14 @@ cudaError_t launch_combine(const Dims& dm, const void* y, const float* gates,
     threads = (threads + 31) / 32 * 32;
     if (f32) combine_kernel<true><<<dm.T, threads, 0, st>>>(y, gates, slot_row, dm.T, dm.d, dm.K, dm.S, dm.r_cap, out);
     else combine_kernel<false><<<dm.T, threads, 0, st>>>(y, gates, slot_row, dm.T, dm.d, dm.K, dm.S, dm.r_cap, out);
+    count_launches();
     return cudaGetLastError();
 }
 
 cudaError_t launch_balance(const Dims& dm, const int32_t* counts, const float* psum,
                            float* f, float* P, float* loss, cudaStream_t st) {
     balance_kernel<<<1, 256, 0, st>>>(counts, psum, dm.route_blocks, dm.T, dm.E, dm.K, dm.alpha, f, P, loss);
+    count_launches();
     return cudaGetLastError();
 }
 

@@ -250,6 +250,7 @@ cudaError_t launch_dispatch(const Dims& dm, const void* x, const int32_t* topk_i
     else if (dm.dtype == MOE_BF16) MOE_SCATTER(1);
     else MOE_SCATTER(2);
 #undef MOE_SCATTER
+    count_launches(3);
     return cudaGetLastError();
 }
 

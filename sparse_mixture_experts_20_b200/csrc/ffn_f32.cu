@@ -138,6 +138,7 @@ cudaError_t launch_grouped_ffn_f32(const Dims& dm, const GemmArgs& a, cudaStream
     p.silu = a.silu;
     const int mt_bound = (dm.r_cap + FBM - 1) / FBM + dm.E + dm.S * ((dm.T + FBM - 1) / FBM);
     ffn_f32_kernel<<<dim3(mt_bound, ntiles), 256, 0, st>>>(p);
+    count_launches();
     return cudaGetLastError();
 }
 

@@ -235,6 +235,7 @@ cudaError_t launch_grouped_ffn_bf16(const Dims&, const GemmArgs& a, cudaStream_t
     cudaError_t e = cudaFuncSetAttribute(grouped_ffn_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     grouped_ffn_bf16_kernel<<<device_sm_count(), NUM_THREADS, smem, st>>>(p);
+    count_launches();
     return cudaGetLastError();
 }
 

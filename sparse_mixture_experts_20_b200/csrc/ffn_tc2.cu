@@ -263,6 +263,7 @@ cudaError_t launch_grouped_ffn_bf16_pair(const Dims&, const GemmArgs& a, cudaStr
     if (clusters < 1) return cudaErrorLaunchOutOfResources;
     cfg.gridDim = dim3(2 * clusters);
     e = cudaLaunchKernelEx(&cfg, grouped_ffn_bf16_pair_kernel, p);
+    count_launches();
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }

@@ -134,4 +134,7 @@ int device_sm_count();
 // Records a failed CUDA call for moe_last_cuda_error() on this thread.
 void note_cuda_error(int err);
 
+// Adds n to the process-wide kernel launch counter (moe_kernel_launches).
+void count_launches(int n = 1);
+
 }  // namespace moe

@@ -1,6 +1,7 @@
 // C ABI of the MoE layer library: argument checks, workspace layout and the
 // stage sequence.  Every entry point validates on the host before launching
 // anything, and returns a MOE_* status; no C++ exception crosses the ABI.
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include "common.cuh"
@@ -249,8 +250,12 @@ __global__ void wait_selftest_kernel(int64_t timeout_ns, int32_t* status) {
 
 void note_cuda_error(int err) { g_last_cuda_error = err; }
 
+static std::atomic<uint64_t> g_kernel_launches{0};
+void count_launches(int n) { g_kernel_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+
 cudaError_t launch_wait_selftest(int64_t timeout_ns, int32_t* status, cudaStream_t st) {
     wait_selftest_kernel<<<1, 32, 0, st>>>(timeout_ns, status);
+    count_launches();
     return cudaGetLastError();
 }
 
@@ -306,6 +311,8 @@ int moe_get_device_status(const moe_config* cfg, void* ws, void* stream, int32_t
 }
 
 int moe_last_cuda_error(void) { return g_last_cuda_error; }
+
+uint64_t moe_kernel_launches(void) { return moe::g_kernel_launches.load(std::memory_order_relaxed); }
 
 const char* moe_status_string(int status) {
     switch (status) {

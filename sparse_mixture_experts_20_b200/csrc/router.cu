@@ -321,6 +321,7 @@ cudaError_t launch_generic(const Dims& dm, const void* x, const float* W_r, cons
     else if (dm.E <= 128) MOE_GEN(4);
     else MOE_GEN(8);
 #undef MOE_GEN
+    count_launches();
     return cudaGetLastError();
 }
 
@@ -333,6 +334,7 @@ cudaError_t launch_small_t(const Dims& dm, const void* x, const float* W_r, cons
     if (e != cudaSuccess) return e;
     router_small_kernel<XT, NE, RT><<<dm.route_blocks, NTHREADS, smem, st>>>(
         static_cast<const XT*>(x), W_r, bias, dm.T, dm.d, dm.E, dm.K, idx, gates, logits, psum);
+    count_launches();
     return cudaGetLastError();
 }
 
@@ -374,6 +376,7 @@ cudaError_t launch_router(const Dims& dm, const void* x, const float* W_r, const
         int blocks = static_cast<int>((n + 255) / 256);
         if (blocks > 4 * 148) blocks = 4 * 148;
         router_reduce_kernel<<<blocks, 256, 0, st>>>(rs.part, plan.ksplit, n, rs.logits);
+        count_launches();
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         logits = rs.logits;
@@ -385,6 +388,7 @@ cudaError_t launch_router(const Dims& dm, const void* x, const float* W_r, const
     else if (dm.E <= 128) MOE_SEL(4);
     else MOE_SEL(8);
 #undef MOE_SEL
+    count_launches();
     return cudaGetLastError();
 }
 

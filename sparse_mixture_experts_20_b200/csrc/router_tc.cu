@@ -208,6 +208,7 @@ cudaError_t launch_bn(const Dims& dm, const RouterTcPlan& plan, const RouterTcPa
     cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     router_tc_kernel<BN><<<dim3(plan.mt, plan.nt, plan.ksplit), RTHREADS, smem, st>>>(p);
+    count_launches();
     return cudaGetLastError();
 }
 
@@ -239,6 +240,7 @@ cudaError_t launch_router_tc(const Dims& dm, const RouterTcPlan& plan, const voi
     int blocks = static_cast<int>((n + 255) / 256);
     if (blocks > 4 * 148) blocks = 4 * 148;
     router_split_kernel<<<blocks, 256, 0, st>>>(W_r, dm.E, dm.d, static_cast<__nv_bfloat16*>(w3));
+    count_launches();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     RouterTcParams p;

@@ -111,6 +111,7 @@ def test_unsupported_shapes_rejected(bad):
 
 def test_null_pointers_rejected_without_launch():
     L = M.lib()
+    launches_before = M.moe_kernel_launches()
     cfg = M.make_config(T=64, d_model=128, n_routed=8, top_k=2, d_ff=256)
     c = ctypes.byref(cfg)
     assert L.moe_route(c, None, None, None, None, None, None, None, None) == M.MOE_ERR_INVALID_ARG
@@ -122,6 +123,8 @@ def test_null_pointers_rejected_without_launch():
     # misaligned workspace / inputs (fake, never dereferenced)
     assert L.moe_route(c, 0x1000, 0x1000, None, 0x1000, 0x1000, None, 0x1001, None) == M.MOE_ERR_INVALID_ARG
     assert L.moe_route(c, 0x1008, 0x1000, None, 0x1000, 0x1000, None, 0x1000, None) == M.MOE_ERR_INVALID_ARG
+    # every rejection happened on the host, before any kernel was launched
+    assert M.moe_kernel_launches() == launches_before
 
 
 def test_fp8_requires_scales():

@@ -46,14 +46,20 @@ def test_stage_and_layer_parity(name):
     require_gpu()
     sh = CASES[name]
     inp = TL.gpu_inputs(sh, seed=1234)
+    n0 = M.moe_kernel_launches()
     o = TL.run_stages(sh, inp)
+    n_stages = M.moe_kernel_launches() - n0
     assert o["status"] == 0
     rt_prod = TL.check_routing(sh, inp, o)
     TL.check_dispatch(sh, inp, o, rt_prod)
     TL.check_expert_ffn(sh, inp, o, rt_prod)
     TL.check_combine(sh, o, rt_prod)
+    n1 = M.moe_kernel_launches()
     lay = TL.run_layer(sh, inp)
+    n_layer = M.moe_kernel_launches() - n1
     assert lay["status"] == 0
+    # router >= 1, dispatch 3, two grouped GEMMs, combine, balance
+    assert n_layer == n_stages >= 8, (n_layer, n_stages)
     # the fused entry point runs the same kernels in the same order
     assert torch.equal(lay["out"], o["out"])
     assert torch.equal(lay["topk_idx"], o["topk_idx"])
