@@ -83,6 +83,25 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def max_over_ranks(ms, world, device=None):
+    """The largest of the ranks' times (every rank returns it); the job is as
+    slow as its slowest replica.  Works on the nccl (CUDA tensor) and gloo
+    (CPU tensor) backends."""
+    if world <= 1:
+        return float(ms)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank_step, world, steps, total_ms):
+    """Whole-job tokens/s: the tokens of all ranks over all timed steps,
+    divided by the (max-over-ranks) time of those steps."""
+    return tokens_per_rank_step * world * steps / (total_ms * 1e-3)
+
+
 def workload_config(sh, seed, parallelism):
     return {"workload": sh.name, "T": sh.T, "d_model": sh.d_model, "n_routed": sh.n_routed,
             "top_k": sh.top_k, "d_ff": sh.d_ff, "n_shared": sh.n_shared, "d_ff_shared": sh.d_ff_shared,
@@ -341,11 +360,7 @@ def run_ours(args):
     stage_ms = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(n_stage)]
                          for k in range(args.steps)])
     step_ms = stage_ms.sum(axis=1)
-    total_ms = float(step_ms.sum())
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(float(step_ms.sum()), world, dev)
     kept = b["kept"].cpu().numpy()
     counts = b["counts"].cpu().numpy()
     status = M.moe_get_device_status(cfg, ws)
@@ -372,11 +387,7 @@ def run_ours(args):
         e2e_ev[k][1].record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    e2e_ms = float(sum(a.elapsed_time(c) for a, c in e2e_ev))
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(float(sum(a.elapsed_time(c) for a, c in e2e_ev)), world, dev)
     clocks = sampler.stop()
 
     peaks, peak_src = load_peaks()
@@ -401,8 +412,7 @@ def run_ours(args):
     roof["traffic"] = traffic_from_profile(sh.name, kname, src_hash(kfiles))
     roof["algorithmic"] = {"flops": flops, "bytes": fbytes, "experts_touched": touched}
 
-    n_tok = T * world * args.steps
-    value = n_tok / (total_ms * 1e-3)
+    value = job_throughput(T, world, args.steps, total_ms)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
@@ -414,7 +424,7 @@ def run_ours(args):
                       enumerate(["route", "dispatch", "expert_ffn", "combine", "balance"])},
         "grouped_gemm_tflops": round(flops / (ffn_ms * 1e-3) / 1e12, 1),
         "roofline": roof,
-        "e2e": {"value": round(T * world * args.steps / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+        "e2e": {"value": round(job_throughput(T, world, args.steps, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(inp["x"].numel() * inp["x"].element_size()),
                 "d2h_bytes_per_step": int(T * d * (4 if sh.dtype == 0 else 2) + 4)},
         "gpu_launches": launches,

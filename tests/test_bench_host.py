@@ -1,0 +1,115 @@
+"""Host logic of bench.py, on CPU: the cross-rank reduction of the replica
+path on two gloo ranks, the whole-job throughput, the workload overrides,
+the roofline arithmetic and the traffic table lookup."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from synthetic import CONFIGS  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, times, out_dir):
+    import datetime
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        t = bench.max_over_ranks(times[rank], world)
+        v = bench.job_throughput(4096, world, 10, t)
+        with open(os.path.join(out_dir, f"r{rank}.json"), "w") as f:
+            json.dump({"t": t, "v": v}, f)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2])
+def test_replica_timing_is_max_over_ranks_gloo(tmp_path, world):
+    times = [3.25, 5.5]
+    mp.start_processes(_rank_main, args=(world, _free_port(), times, str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    res = [json.load(open(tmp_path / f"r{r}.json")) for r in range(world)]
+    for r in res:
+        assert r["t"] == max(times)                       # every rank sees the slowest replica
+        assert r["v"] == pytest.approx(4096 * world * 10 / (max(times) * 1e-3))
+
+
+def test_single_rank_needs_no_process_group():
+    assert bench.max_over_ranks(2.0, 1) == 2.0
+    assert bench.job_throughput(128, 1, 4, 2.0) == pytest.approx(128 * 4 / 2e-3)
+
+
+def test_reference_arm_other_ranks_exit_without_output():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "0"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_set_overrides_build_a_reduced_case():
+    args = bench.argparse.Namespace(config=4, set=["n_routed=64", "T=1024"])
+    sh = bench.workload(args)
+    assert (sh.n_routed, sh.T, sh.d_model, sh.top_k) == (64, 1024, 7168, 8)
+    assert sh.name.endswith("[n_routed=64,T=1024]")
+    assert bench.workload(bench.argparse.Namespace(config=2, set=[])) == CONFIGS[2]
+
+
+def test_roofline_work_per_step_closed_forms():
+    import numpy as np
+    sh = CONFIGS[2]
+    kept = np.full(sh.n_routed, sh.T * sh.top_k // sh.n_routed)
+    R = int(kept.sum())
+    assert bench.algorithmic_ffn(sh, R) == 4.0 * sh.d_model * sh.d_ff * R
+    b, touched = bench.ffn_bytes(sh, kept)
+    d, f = sh.d_model, sh.d_ff
+    weights = sh.n_routed * (2 * d * f * 2 + 4 * (f + d))
+    act = R * d * 2 + 2 * R * f * 2 + R * d * 2
+    assert touched == sh.n_routed and b == weights + act
+    # FP8: one byte per weight plus the fp32 block scales
+    sh4 = CONFIGS[4]
+    kept4 = np.zeros(sh4.n_routed, dtype=np.int64)
+    kept4[:3] = 10
+    b4, t4 = bench.ffn_bytes(sh4, kept4)
+    d, f, S, T = sh4.d_model, sh4.d_ff, sh4.n_shared, sh4.T
+    w4 = 3 * (2 * d * f + 4 * (f + d)) + S * (2 * d * sh4.d_ff_shared + 4 * (sh4.d_ff_shared + d))
+    w4 += 3 * 2 * (d // 128) * (f // 128) * 4 + S * 2 * (d // 128) * (sh4.d_ff_shared // 128) * 4
+    R4 = 30
+    act4 = (R4 + S * T) * d + 2 * (R4 * f + S * T * sh4.d_ff_shared) + (R4 + S * T) * d * 2
+    assert t4 == 3 and b4 == w4 + act4
+
+
+def test_traffic_lookup_requires_the_captured_sources():
+    p = os.path.join(ROOT, "profiles", "grouped_ffn_traffic.json")
+    entries = json.load(open(p))["entries"]
+    assert entries
+    for e in entries:
+        assert bench.traffic_from_profile(e["workload"], e["kernel"], e["src_sha1"]) == e["dram_bytes_per_step"]
+        assert bench.traffic_from_profile(e["workload"], e["kernel"], "0" * 40) is None
+        assert bench.traffic_from_profile(e["workload"] + " other", e["kernel"], e["src_sha1"]) is None
+
+
+def test_ffn_kernel_follows_dtype_and_pair_switch(monkeypatch):
+    monkeypatch.delenv("MOE_GEMM_PAIR", raising=False)
+    assert bench.ffn_kernel(CONFIGS[1])[0] == "ffn_f32_kernel"
+    assert bench.ffn_kernel(CONFIGS[2])[0] == "grouped_ffn_bf16_pair_kernel"
+    assert bench.ffn_kernel(CONFIGS[4])[0] == "grouped_ffn_fp8_kernel"
+    monkeypatch.setenv("MOE_GEMM_PAIR", "0")
+    assert bench.ffn_kernel(CONFIGS[2])[0] == "grouped_ffn_bf16_kernel"
+    for cid in (1, 2, 4):
+        for f in bench.ffn_kernel(CONFIGS[cid])[1]:
+            assert os.path.exists(os.path.join(bench.CSRC, f))
