@@ -235,6 +235,29 @@ def ffn_bytes(sh, kept):
     return float(w + act), touched
 
 
+def stage_bytes(sh, kept):
+    """Algorithmic HBM bytes per step of the memory-bound stages: every
+    operand read once and every result written once.
+      route:    x, W_r (fp32), the logit bias, topk_idx + gates, the partial
+                sums of s per 32-token block
+      dispatch: topk_idx, x once, the dispatched rows (+ FP8 scales, + the
+                quantised x of the shared experts), the slot maps
+      combine:  the kept routed rows and the shared rows of y, gates and
+                slot map, the layer output"""
+    T, d, E, K, S = sh.T, sh.d_model, sh.n_routed, sh.top_k, sh.n_shared
+    bx = {0: 4, 1: 2, 2: 2}[sh.dtype]          # x / y / out element bytes
+    bq = {0: 4, 1: 2, 2: 1}[sh.dtype]          # dispatched row element bytes
+    R = int(kept.sum())
+    route = T * d * bx + E * d * 4 + (E * 4 if sh.zipf_logit_bias else 0) + T * K * 8 + ((T + 31) // 32) * E * 4
+    disp = T * K * 4 + T * d * bx + R * d * bq + T * K * 4 + R * 4 + (2 * E + 1) * 4
+    if sh.dtype == 2:
+        disp += R * (d // 128) * 4
+        if S > 0:
+            disp += T * d + T * (d // 128) * 4
+    comb = R * d * bx + S * T * d * bx + T * K * 8 + T * d * bx
+    return {"route": float(route), "dispatch": float(disp), "combine": float(comb)}
+
+
 CSRC = os.path.join(ROOT, "sparse_mixture_experts_20_b200", "csrc")
 
 
@@ -412,6 +435,13 @@ def run_ours(args):
     roof["traffic"] = traffic_from_profile(sh.name, kname, src_hash(kfiles))
     roof["algorithmic"] = {"flops": flops, "bytes": fbytes, "experts_touched": touched}
 
+    sb = stage_bytes(sh, kept)
+    stages_hbm = {}
+    for i, name in enumerate(["route", "dispatch", "expert_ffn", "combine", "balance"]):
+        if name in sb:
+            ms_i = float(stage_ms[:, i].mean())
+            gbs = sb[name] / (ms_i * 1e-3) / 1e9
+            stages_hbm[name] = {"bytes": sb[name], "gbs": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4)}
     value = job_throughput(T, world, args.steps, total_ms)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -423,6 +453,7 @@ def run_ours(args):
         "stages_ms": {n: round(float(stage_ms[:, i].mean()), 4) for i, n in
                       enumerate(["route", "dispatch", "expert_ffn", "combine", "balance"])},
         "grouped_gemm_tflops": round(flops / (ffn_ms * 1e-3) / 1e12, 1),
+        "stages_hbm": stages_hbm,
         "roofline": roof,
         "e2e": {"value": round(job_throughput(T, world, args.steps, e2e_ms), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(inp["x"].numel() * inp["x"].element_size()),

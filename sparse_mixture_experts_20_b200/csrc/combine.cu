@@ -6,10 +6,10 @@
 // BF16 combine.  "エキスパート並列（Expert Parallelism）" §推論フロー step 5:
 // results return to their token (on one GPU: a gather).
 //
-// combine_kernel: block per token; each thread owns 16 bytes of the output
-// row, gathers the token's kept expert rows (ascending k) with 16-byte loads,
-// accumulates g * y in fp32, adds the shared experts' rows (ascending s) and
-// rounds once.
+// combine_kernel: warp(s) per token; each lane owns 16-byte chunks of the
+// output row, gathers the token's kept expert rows (loads issued together,
+// accumulated in ascending k) with 16-byte loads, accumulates g * y in fp32,
+// adds the shared experts' rows (ascending s) and rounds once.
 // balance_kernel: one block; fixed-order reductions, so f, P and the loss are
 // bit-reproducible.
 #include "common.cuh"
@@ -18,63 +18,69 @@
 namespace moe {
 namespace {
 
-constexpr int MAXK = 16;
 
-template <bool F32>
-__global__ void __launch_bounds__(1024)
+constexpr int CB_WARPS = 8;       // warps per combine block
+
+// W warps per token (W = 1 for large batches, up to 8 for small ones).  Lanes
+// 0..K-1 read the token's slot rows and gates and broadcast them; each lane
+// then owns 16-byte chunks of the output row: it issues the loads of all the
+// token's kept rows for a chunk before accumulating them in ascending k
+// (then the shared rows in ascending s) in fp32, and rounds once.
+template <bool F32, int KT>           // KT >= K: register slots for the token's rows
+__global__ void __launch_bounds__(32 * CB_WARPS, KT <= 8 ? 4 : 2)
 combine_kernel(const void* __restrict__ y_, const float* __restrict__ gates,
                const int32_t* __restrict__ slot_row, int T, int d, int K, int S, int r_cap,
-               void* __restrict__ out_) {
-    __shared__ int rows_s[MAXK];
-    __shared__ float g_s[MAXK];
-    const int t = blockIdx.x, tid = threadIdx.x;
-    if (tid < K) {
-        rows_s[tid] = slot_row[static_cast<size_t>(t) * K + tid];
-        g_s[tid] = gates[static_cast<size_t>(t) * K + tid];
-    }
-    __syncthreads();
-    if (F32) {
-        const float* y = static_cast<const float*>(y_);
-        for (int c = tid; c < d / 4; c += blockDim.x) {
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int k = 0; k < K; ++k) {
-                const int r = rows_s[k];
-                if (r < 0) continue;
-                const float g = g_s[k];
-                const float4 v = reinterpret_cast<const float4*>(y + static_cast<size_t>(r) * d)[c];
-                acc.x = fmaf(g, v.x, acc.x); acc.y = fmaf(g, v.y, acc.y);
-                acc.z = fmaf(g, v.z, acc.z); acc.w = fmaf(g, v.w, acc.w);
-            }
-            for (int s = 0; s < S; ++s) {
-                const float4 v = reinterpret_cast<const float4*>(
-                    y + (static_cast<size_t>(r_cap) + static_cast<size_t>(s) * T + t) * d)[c];
-                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-            }
-            reinterpret_cast<float4*>(static_cast<float*>(out_) + static_cast<size_t>(t) * d)[c] = acc;
-        }
-    } else {
-        const __nv_bfloat16* y = static_cast<const __nv_bfloat16*>(y_);
-        for (int c = tid; c < d / 8; c += blockDim.x) {
-            float acc[8];
+               void* __restrict__ out_, int wpt) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int t = blockIdx.x * (CB_WARPS / wpt) + warp / wpt;
+    const int sub = warp % wpt;
+    if (t >= T) return;
+    const int my_row = lane < K ? slot_row[static_cast<size_t>(t) * K + lane] : -1;
+    const float my_g = lane < K ? gates[static_cast<size_t>(t) * K + lane] : 0.f;
+    int rows[KT];
+    float g[KT];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-            for (int k = 0; k < K; ++k) {
-                const int r = rows_s[k];
-                if (r < 0) continue;
-                const float g = g_s[k];
-                const uint4 raw = __ldg(reinterpret_cast<const uint4*>(y + static_cast<size_t>(r) * d) + c);
-                const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+    for (int k = 0; k < KT; ++k) {
+        rows[k] = __shfl_sync(0xffffffffu, my_row, k);
+        g[k] = __shfl_sync(0xffffffffu, my_g, k);
+    }
+    const int nchunks = d / (F32 ? 4 : 8);
+    const uint4* y = static_cast<const uint4*>(y_);          // rows of nchunks 16-byte chunks
+    uint4* out = static_cast<uint4*>(out_) + static_cast<size_t>(t) * nchunks;
+    for (int c = sub * 32 + lane; c < nchunks; c += 32 * wpt) {
+        uint4 raw[KT];
+#pragma unroll
+        for (int k = 0; k < KT; ++k)
+            raw[k] = (k < K && rows[k] >= 0) ? __ldg(y + static_cast<size_t>(rows[k]) * nchunks + c)
+                                             : make_uint4(0, 0, 0, 0);
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+        for (int k = 0; k < KT; ++k) {
+            if (k >= K || rows[k] < 0) continue;
+            if (F32) {
+                const float* f = reinterpret_cast<const float*>(&raw[k]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[i] = fmaf(g[k], f[i], acc[i]);
+            } else {
+                const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[k]);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const float2 f = __bfloat1622float2(h2[i]);
-                    acc[2 * i] = fmaf(g, f.x, acc[2 * i]);
-                    acc[2 * i + 1] = fmaf(g, f.y, acc[2 * i + 1]);
+                    acc[2 * i] = fmaf(g[k], f.x, acc[2 * i]);
+                    acc[2 * i + 1] = fmaf(g[k], f.y, acc[2 * i + 1]);
                 }
             }
-            for (int s = 0; s < S; ++s) {
-                const uint4 raw = __ldg(reinterpret_cast<const uint4*>(
-                    y + (static_cast<size_t>(r_cap) + static_cast<size_t>(s) * T + t) * d) + c);
-                const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+        }
+        for (int s = 0; s < S; ++s) {
+            const uint4 v = __ldg(y + (static_cast<size_t>(r_cap) + static_cast<size_t>(s) * T + t) * nchunks + c);
+            if (F32) {
+                const float* f = reinterpret_cast<const float*>(&v);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[i] += f[i];
+            } else {
+                const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const float2 f = __bfloat1622float2(h2[i]);
@@ -82,15 +88,20 @@ combine_kernel(const void* __restrict__ y_, const float* __restrict__ gates,
                     acc[2 * i + 1] += f.y;
                 }
             }
-            uint4 o;
+        }
+        uint4 o;
+        if (F32) {
+            o = make_uint4(__float_as_uint(acc[0]), __float_as_uint(acc[1]), __float_as_uint(acc[2]),
+                           __float_as_uint(acc[3]));
+        } else {
             uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 __nv_bfloat162 v = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
                 ow[i] = *reinterpret_cast<uint32_t*>(&v);
             }
-            reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out_) + static_cast<size_t>(t) * d)[c] = o;
         }
+        out[c] = o;
     }
 }
 
@@ -124,11 +135,20 @@ balance_kernel(const int32_t* __restrict__ counts, const float* __restrict__ psu
 cudaError_t launch_combine(const Dims& dm, const void* y, const float* gates,
                            const int32_t* slot_row, void* out, cudaStream_t st) {
     const bool f32 = dm.dtype == MOE_F32;
-    int threads = dm.d / (f32 ? 4 : 8);
-    if (threads > 1024) threads = 1024;
-    threads = (threads + 31) / 32 * 32;
-    if (f32) combine_kernel<true><<<dm.T, threads, 0, st>>>(y, gates, slot_row, dm.T, dm.d, dm.K, dm.S, dm.r_cap, out);
-    else combine_kernel<false><<<dm.T, threads, 0, st>>>(y, gates, slot_row, dm.T, dm.d, dm.K, dm.S, dm.r_cap, out);
+    int wpt = 1;                              // enough warps in flight to fill the GPU at small T
+    while (wpt < CB_WARPS && static_cast<long long>(dm.T) * wpt < 148LL * 32) wpt *= 2;
+    const int blocks = (dm.T + CB_WARPS / wpt - 1) / (CB_WARPS / wpt);
+#define MOE_COMBINE(F, KT) combine_kernel<F, KT><<<blocks, 32 * CB_WARPS, 0, st>>>(          \
+        y, gates, slot_row, dm.T, dm.d, dm.K, dm.S, dm.r_cap, out, wpt)
+#define MOE_COMBINE_K(F)                                                                         \
+    if (dm.K <= 2) MOE_COMBINE(F, 2);                                                            \
+    else if (dm.K <= 4) MOE_COMBINE(F, 4);                                                       \
+    else if (dm.K <= 8) MOE_COMBINE(F, 8);                                                       \
+    else MOE_COMBINE(F, 16)
+    if (f32) { MOE_COMBINE_K(true); }
+    else { MOE_COMBINE_K(false); }
+#undef MOE_COMBINE_K
+#undef MOE_COMBINE
     count_launches();
     return cudaGetLastError();
 }

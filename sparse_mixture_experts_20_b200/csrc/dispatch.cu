@@ -15,9 +15,9 @@
 //   2. scan_kernel   : one block; per expert, prefix sums of popcounts over
 //      words -> word_base[word][j] (slots of j in earlier words), counts,
 //      kept = min(counts, C), offsets = exclusive scan of kept.
-//   3. scatter_kernel: block per token; thread k < K finds the slot's rank
+//   3. scatter_kernel: warp per token; lane k < K finds the slot's rank
 //      (word_base + popcount of the lower lanes' bits), keeps it if rank < C,
-//      writes slot_row / row_slot; then the block copies (bf16/fp32) or
+//      writes slot_row / row_slot; then the warp copies (bf16/fp32) or
 //      quantises to e4m3 (FP8) the token's row into each kept destination
 //      with 16-byte accesses.
 #include "common.cuh"
@@ -131,98 +131,132 @@ scan_kernel(const uint32_t* __restrict__ bitmap, int E, int t_words, int capacit
     }
 }
 
+constexpr int SC_WARPS = 8;       // warps per scatter block
+
+// W warps per token (W = 1 for large batches; up to 8 when there are too few
+// tokens to fill the GPU).  Lanes 0..K-1 resolve the token's K slots to destination
+// rows (rank = word_base + popcount of the earlier tokens' bits of the word);
+// the rows are broadcast with shuffles and the warp copies (bf16 / fp32) or
+// quantises to e4m3 (FP8) the token's row into every kept destination with
+// 16-byte (8-byte for e4m3) accesses.  The first loads of the row are issued
+// before the slot resolution, so the two latencies overlap.
 template <int MODE>   // 0: fp32 copy, 1: bf16 copy, 2: bf16 -> e4m3 + 1x128 scales
-__global__ void __launch_bounds__(1024)
+__global__ void __launch_bounds__(32 * SC_WARPS)
 scatter_kernel(const void* __restrict__ x_, const int32_t* __restrict__ topk_idx,
                const uint32_t* __restrict__ bitmap, const int32_t* __restrict__ word_base,
                const int32_t* __restrict__ offsets, int T, int d, int E, int K, int capacity,
                int r_cap, int shared_copy, int32_t* __restrict__ slot_row,
                int32_t* __restrict__ row_slot, void* __restrict__ x_disp_,
-               float* __restrict__ x_disp_scales) {
-    __shared__ int rows_s[MAXK];
-    const int t = blockIdx.x;
-    const int tid = threadIdx.x;
-    if (tid < K) {
-        int ids[MAXK];
-        for (int k = 0; k < K; ++k) ids[k] = topk_idx[static_cast<size_t>(t) * K + k];
-        int row = -1;
-        if (slot_valid(ids, tid, E)) {
-            const int j = ids[tid];
-            const int w = t >> 5;
-            const uint32_t below = bitmap[static_cast<size_t>(w) * E + j] & ((1u << (t & 31)) - 1u);
-            const int rank = word_base[static_cast<size_t>(w) * E + j] + __popc(below);
-            if (capacity < 0 || rank < capacity) row = offsets[j] + rank;
-        }
-        rows_s[tid] = row;
-        slot_row[static_cast<size_t>(t) * K + tid] = row;
-        if (row >= 0) row_slot[row] = t * K + tid;
+               float* __restrict__ x_disp_scales, int wpt) {
+    constexpr int PF = 4;                                  // 16-byte chunks per lane in flight
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int t = blockIdx.x * (SC_WARPS / wpt) + warp / wpt;
+    const int sub = warp % wpt;                            // this warp's share of the row
+    if (t >= T) return;
+    const int lane0 = sub * 32 + lane;                     // chunk of the first round
+    const int stride = 32 * wpt;                           // chunks between rounds
+    const int nchunks = d / (MODE == 0 ? 4 : 8);           // 16-byte chunks of the source row
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(x_) +
+                                                      static_cast<size_t>(t) * d * (MODE == 0 ? 4 : 2));
+    uint4 pre[PF];
+#pragma unroll
+    for (int u = 0; u < PF; ++u) {
+        const int c = lane0 + stride * u;
+        pre[u] = c < nchunks ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
     }
-    __syncthreads();
-    if (MODE == 0) {
-        const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(x_) + static_cast<size_t>(t) * d);
-        for (int c = tid; c < d / 4; c += blockDim.x) {
-            const float4 v = src[c];
-            for (int k = 0; k < K; ++k) {
-                const int r = rows_s[k];
-                if (r >= 0) reinterpret_cast<float4*>(static_cast<float*>(x_disp_) + static_cast<size_t>(r) * d)[c] = v;
-            }
+    // ---- slot resolution (lane k: slot k)
+    const int my_id = lane < K ? topk_idx[static_cast<size_t>(t) * K + lane] : -1;
+    int row = -1;
+    {
+        bool valid = lane < K && my_id >= 0 && my_id < E;
+        for (int q = 0; q < K; ++q) {                      // repeated by an earlier slot?
+            const int other = __shfl_sync(0xffffffffu, my_id, q);
+            if (q < lane && other == my_id) valid = false;
         }
-    } else if (MODE == 1) {
-        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x_) + static_cast<size_t>(t) * d);
-        for (int c = tid; c < d / 8; c += blockDim.x) {
-            const uint4 v = src[c];
-            for (int k = 0; k < K; ++k) {
-                const int r = rows_s[k];
-                if (r >= 0) reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(x_disp_) + static_cast<size_t>(r) * d)[c] = v;
+        if (valid) {
+            const int w = t >> 5;
+            const uint32_t below = bitmap[static_cast<size_t>(w) * E + my_id] & ((1u << (t & 31)) - 1u);
+            const int rank = word_base[static_cast<size_t>(w) * E + my_id] + __popc(below);
+            if (capacity < 0 || rank < capacity) row = offsets[my_id] + rank;
+        }
+        if (lane < K && sub == 0) {
+            slot_row[static_cast<size_t>(t) * K + lane] = row;
+            if (row >= 0) row_slot[row] = t * K + lane;
+        }
+    }
+    int rows[MAXK + 1];
+#pragma unroll
+    for (int k = 0; k < MAXK; ++k) rows[k] = __shfl_sync(0xffffffffu, row, k);
+    rows[MAXK] = (MODE == 2 && shared_copy) ? r_cap + t : -1;
+    if (MODE != 2) {
+        uint4* dst0 = static_cast<uint4*>(x_disp_);
+        const size_t row_chunks = static_cast<size_t>(nchunks);
+        for (int base = 0; base < nchunks; base += stride * PF) {
+            uint4 v[PF];
+#pragma unroll
+            for (int u = 0; u < PF; ++u) {
+                const int c = base + lane0 + stride * u;
+                v[u] = base == 0 ? pre[u] : (c < nchunks ? __ldg(src + c) : make_uint4(0, 0, 0, 0));
+            }
+#pragma unroll
+            for (int k = 0; k < MAXK; ++k) {
+                if (k >= K) break;
+                const int r = rows[k];
+                if (r < 0) continue;
+#pragma unroll
+                for (int u = 0; u < PF; ++u) {
+                    const int c = base + lane0 + stride * u;
+                    if (c < nchunks) dst0[static_cast<size_t>(r) * row_chunks + c] = v[u];
+                }
             }
         }
     } else {
-        // 16 consecutive threads own one 128-column block (8 values each);
-        // blockDim is a multiple of 16 and d a multiple of 128.
-        const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x_) + static_cast<size_t>(t) * d);
+        // 16 consecutive lanes own one 128-column block (8 values each); d is
+        // a multiple of 128, so a 16-lane group is always entirely in range
         uint8_t* xd = static_cast<uint8_t*>(x_disp_);
         const int nq = d / 128;
-        const int nchunks = d / 8;
-        // every lane runs every round so that the 16-lane shuffles are full-warp
-        for (int base = 0; base < nchunks; base += blockDim.x) {
-            const int c = base + tid;
-            const bool act = c < nchunks;
-            float v[8];
-            if (act) {
-                const uint4 raw = src[c];
-                const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+        for (int base = 0; base < nchunks; base += stride * PF) {
+            uint4 raw[PF];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float2 f = __bfloat1622float2(h2[i]);
-                    v[2 * i] = f.x;
-                    v[2 * i + 1] = f.y;
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] = 0.f;
+            for (int u = 0; u < PF; ++u) {
+                const int c = base + lane0 + stride * u;
+                raw[u] = base == 0 ? pre[u] : (c < nchunks ? __ldg(src + c) : make_uint4(0, 0, 0, 0));
             }
-            float amax = 0.f;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+            for (int u = 0; u < PF; ++u) {
+                const int c = base + lane0 + stride * u;
+                float v[8];
+                const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[u]);
 #pragma unroll
-            for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off, 16));
-            if (!act) continue;
-            const float sc = pow2_scale_448(amax);
-            const float inv = 1.0f / sc;                     // exact: power of two
-            uint2 q;
-            q.x = static_cast<uint32_t>(f32x2_to_e4m3x2(v[0] * inv, v[1] * inv)) |
-                  (static_cast<uint32_t>(f32x2_to_e4m3x2(v[2] * inv, v[3] * inv)) << 16);
-            q.y = static_cast<uint32_t>(f32x2_to_e4m3x2(v[4] * inv, v[5] * inv)) |
-                  (static_cast<uint32_t>(f32x2_to_e4m3x2(v[6] * inv, v[7] * inv)) << 16);
-            const int blk = c >> 4;
-            const bool lead = (c & 15) == 0;
-            for (int k = 0; k <= K; ++k) {
-                int r;
-                if (k < K) r = rows_s[k];
-                else r = shared_copy ? r_cap + t : -1;
-                if (r < 0) continue;
-                reinterpret_cast<uint2*>(xd + static_cast<size_t>(r) * d)[c] = q;
-                if (lead) x_disp_scales[static_cast<size_t>(r) * nq + blk] = sc;
+                for (int i2 = 0; i2 < 4; ++i2) {
+                    const float2 f = __bfloat1622float2(h2[i2]);
+                    v[2 * i2] = f.x;
+                    v[2 * i2 + 1] = f.y;
+                }
+                float amax = 0.f;
+#pragma unroll
+                for (int i2 = 0; i2 < 8; ++i2) amax = fmaxf(amax, fabsf(v[i2]));
+#pragma unroll
+                for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off, 16));
+                if (c >= nchunks) continue;
+                const float sc = pow2_scale_448(amax);
+                const float inv = 1.0f / sc;                     // exact: power of two
+                uint2 q;
+                q.x = static_cast<uint32_t>(f32x2_to_e4m3x2(v[0] * inv, v[1] * inv)) |
+                      (static_cast<uint32_t>(f32x2_to_e4m3x2(v[2] * inv, v[3] * inv)) << 16);
+                q.y = static_cast<uint32_t>(f32x2_to_e4m3x2(v[4] * inv, v[5] * inv)) |
+                      (static_cast<uint32_t>(f32x2_to_e4m3x2(v[6] * inv, v[7] * inv)) << 16);
+                const int blk = c >> 4;
+                const bool lead = (c & 15) == 0;
+#pragma unroll
+                for (int k = 0; k <= MAXK; ++k) {
+                    if (k < MAXK && k >= K) continue;
+                    const int r = rows[k];
+                    if (r < 0) continue;
+                    reinterpret_cast<uint2*>(xd + static_cast<size_t>(r) * d)[c] = q;
+                    if (lead) x_disp_scales[static_cast<size_t>(r) * nq + blk] = sc;
+                }
             }
         }
     }
@@ -237,15 +271,15 @@ cudaError_t launch_dispatch(const Dims& dm, const void* x, const int32_t* topk_i
                             int32_t* status, cudaStream_t st) {
     bitmap_kernel<<<(dm.t_words + 7) / 8, 256, 0, st>>>(topk_idx, dm.T, dm.E, dm.K, dm.t_words, bitmap, status);
     scan_kernel<<<1, 1024, 0, st>>>(bitmap, dm.E, dm.t_words, dm.capacity, word_base, counts, kept, offsets);
-    const int vec = dm.dtype == MOE_F32 ? 4 : 8;
-    int threads = dm.d / vec;
-    if (threads > 1024) threads = 1024;
-    if (dm.dtype == MOE_FP8_E4M3_BLOCK) threads = threads / 16 * 16;
-    threads = (threads + 31) / 32 * 32;
     const int shared_copy = (dm.dtype == MOE_FP8_E4M3_BLOCK && dm.S > 0) ? 1 : 0;
-#define MOE_SCATTER(MODE) scatter_kernel<MODE><<<dm.T, threads, 0, st>>>(                 \
+    // warps per token: enough warps in flight to fill the GPU at small T
+    int wpt = 1;
+    while (wpt < SC_WARPS && static_cast<long long>(dm.T) * wpt < 148LL * 32) wpt *= 2;
+    const int tpb = SC_WARPS / wpt;
+    const int blocks = (dm.T + tpb - 1) / tpb;
+#define MOE_SCATTER(MODE) scatter_kernel<MODE><<<blocks, 32 * SC_WARPS, 0, st>>>(          \
         x, topk_idx, bitmap, word_base, offsets, dm.T, dm.d, dm.E, dm.K, dm.capacity,      \
-        dm.r_cap, shared_copy, slot_row, row_slot, x_disp, x_disp_scales)
+        dm.r_cap, shared_copy, slot_row, row_slot, x_disp, x_disp_scales, wpt)
     if (dm.dtype == MOE_F32) MOE_SCATTER(0);
     else if (dm.dtype == MOE_BF16) MOE_SCATTER(1);
     else MOE_SCATTER(2);

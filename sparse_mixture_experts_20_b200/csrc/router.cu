@@ -6,9 +6,10 @@
 //
 // The logits come from one of three producers, chosen by shape:
 //   * router_small_kernel (N_r <= 32 and W_r fits in shared memory): W_r is
-//     staged once per block; each warp takes 4 (or 2) tokens, lanes split the
-//     model dimension with 16-byte loads of x, and a reduce-scatter over the
-//     lanes leaves each lane with whole dot products.  x is read once.
+//     staged once per block by bulk asynchronous copies (one per expert row,
+//     completed on an mbarrier); each warp takes 4 (or 2) tokens, lanes split
+//     the model dimension with 16-byte loads of x, and a reduce-scatter over
+//     the lanes leaves each lane with whole dot products.  x is read once.
 //   * the tensor-core router (router_tc.cu, bf16 x, larger N_r): W_r split into
 //     three bf16 planes, one tcgen05 GEMM with K = 3 d, partial logits per K
 //     split summed here by router_reduce_kernel;
@@ -196,28 +197,52 @@ __device__ __forceinline__ void warp_reduce_scatter(float (&v)[N], int lane) {
     }
 }
 
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned)
+// from global to this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 :: "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
+constexpr uint64_t kStageWaitNs = 2000000000ull;
+
 template <typename XT, int NE, int RT>
 __global__ void __launch_bounds__(NTHREADS)
 router_small_kernel(const XT* __restrict__ x, const float* __restrict__ W_r,
                     const float* __restrict__ logit_bias, int T, int d, int E, int K,
                     int32_t* __restrict__ topk_idx, float* __restrict__ gates,
-                    float* __restrict__ logits_out, float* __restrict__ psum) {
+                    float* __restrict__ logits_out, float* __restrict__ psum, int32_t* status) {
     extern __shared__ float4 wsm4[];                  // (NE, d) fp32, rows >= E zero
     float* wsm = reinterpret_cast<float*>(wsm4);
     __shared__ float lg[TT][32 + 1];
+    __shared__ __align__(8) uint64_t wbar;
+    __shared__ int abort_s;
     constexpr int VEC = sizeof(XT) == 2 ? 8 : 4;      // elements per 16-byte load
     constexpr int NV = RT * NE;
     static_assert(NV == 32 || NV == 64, "register tile");
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int t0 = blockIdx.x * TT;
 
-    for (int i = tid; i < NE * d / 4; i += NTHREADS) {
-        const int row = (i * 4) / d;
-        wsm4[i] = row < E ? reinterpret_cast<const float4*>(W_r)[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    if (tid == 0) {
+        abort_s = 0;
+        mbar_init(&wbar, 1);
+        fence_mbar_init();
+        // rows 0..E-1 of W_r, d * 4 bytes each, land asynchronously
+        mbar_arrive_expect_tx(&wbar, static_cast<uint32_t>(E) * d * 4);
+        for (int e = 0; e < E; ++e)
+            bulk_copy_g2s(wsm + static_cast<size_t>(e) * d, W_r + static_cast<size_t>(e) * d,
+                          static_cast<uint32_t>(d) * 4, &wbar);
     }
+    for (int i = E * d / 4 + tid; i < NE * d / 4; i += NTHREADS) wsm4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int i = tid; i < TT * 32; i += NTHREADS)
         if ((i & 31) >= NE) lg[i >> 5][i & 31] = -INFINITY;
     __syncthreads();
+    if (!mbar_wait_bounded(&wbar, 0, &abort_s, status, kStageWaitNs)) {
+        // the copies never completed (reported in the status word): leave the
+        // outputs of this block unwritten rather than compute on garbage
+        return;
+    }
 
 #pragma unroll 1
     for (int g = warp; g < TT / RT; g += 8) {
@@ -232,7 +257,7 @@ router_small_kernel(const XT* __restrict__ x, const float* __restrict__ W_r,
             ok[r] = t < T;
             xr[r] = x + static_cast<size_t>(ok[r] ? t : 0) * d;
         }
-#pragma unroll 2
+#pragma unroll 4
         for (int k = lane * VEC; k < d; k += 32 * VEC) {
             float xv[RT][VEC];
 #pragma unroll
@@ -327,23 +352,25 @@ cudaError_t launch_generic(const Dims& dm, const void* x, const float* W_r, cons
 
 template <typename XT, int NE, int RT>
 cudaError_t launch_small_t(const Dims& dm, const void* x, const float* W_r, const float* bias,
-                           int32_t* idx, float* gates, float* logits, float* psum, cudaStream_t st) {
+                           int32_t* idx, float* gates, float* logits, float* psum, int32_t* status,
+                           cudaStream_t st) {
     const size_t smem = static_cast<size_t>(NE) * dm.d * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(router_small_kernel<XT, NE, RT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     router_small_kernel<XT, NE, RT><<<dm.route_blocks, NTHREADS, smem, st>>>(
-        static_cast<const XT*>(x), W_r, bias, dm.T, dm.d, dm.E, dm.K, idx, gates, logits, psum);
+        static_cast<const XT*>(x), W_r, bias, dm.T, dm.d, dm.E, dm.K, idx, gates, logits, psum, status);
     count_launches();
     return cudaGetLastError();
 }
 
 template <typename XT>
 cudaError_t launch_small(const Dims& dm, const void* x, const float* W_r, const float* bias,
-                         int32_t* idx, float* gates, float* logits, float* psum, cudaStream_t st) {
-    if (dm.E <= 8) return launch_small_t<XT, 8, 4>(dm, x, W_r, bias, idx, gates, logits, psum, st);
-    if (dm.E <= 16) return launch_small_t<XT, 16, 4>(dm, x, W_r, bias, idx, gates, logits, psum, st);
-    return launch_small_t<XT, 32, 2>(dm, x, W_r, bias, idx, gates, logits, psum, st);
+                         int32_t* idx, float* gates, float* logits, float* psum, int32_t* status,
+                         cudaStream_t st) {
+    if (dm.E <= 8) return launch_small_t<XT, 8, 4>(dm, x, W_r, bias, idx, gates, logits, psum, status, st);
+    if (dm.E <= 16) return launch_small_t<XT, 16, 4>(dm, x, W_r, bias, idx, gates, logits, psum, status, st);
+    return launch_small_t<XT, 32, 2>(dm, x, W_r, bias, idx, gates, logits, psum, status, st);
 }
 
 }  // namespace
@@ -362,8 +389,9 @@ cudaError_t launch_router(const Dims& dm, const void* x, const float* W_r, const
                           const RouterScratch& rs, cudaStream_t st) {
     if (router_uses_small(dm)) {
         if (dm.dtype == MOE_F32)
-            return launch_small<float>(dm, x, W_r, logit_bias, topk_idx, gates, logits_out, psum, st);
-        return launch_small<__nv_bfloat16>(dm, x, W_r, logit_bias, topk_idx, gates, logits_out, psum, st);
+            return launch_small<float>(dm, x, W_r, logit_bias, topk_idx, gates, logits_out, psum, rs.status, st);
+        return launch_small<__nv_bfloat16>(dm, x, W_r, logit_bias, topk_idx, gates, logits_out, psum, rs.status,
+                                           st);
     }
     if (!router_uses_tc(dm))
         return launch_generic<float>(dm, x, W_r, logit_bias, topk_idx, gates, logits_out, psum, st);

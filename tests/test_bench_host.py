@@ -113,3 +113,15 @@ def test_ffn_kernel_follows_dtype_and_pair_switch(monkeypatch):
     for cid in (1, 2, 4):
         for f in bench.ffn_kernel(CONFIGS[cid])[1]:
             assert os.path.exists(os.path.join(bench.CSRC, f))
+
+
+def test_stage_bytes_closed_forms():
+    import numpy as np
+    sh = CONFIGS[2]
+    T, d, E, K = sh.T, sh.d_model, sh.n_routed, sh.top_k
+    kept = np.full(E, T * K // E)
+    R = T * K
+    b = bench.stage_bytes(sh, kept)
+    assert b["route"] == T * d * 2 + E * d * 4 + T * K * 8 + (T // 32) * E * 4
+    assert b["dispatch"] == T * K * 4 + T * d * 2 + R * d * 2 + T * K * 4 + R * 4 + (2 * E + 1) * 4
+    assert b["combine"] == R * d * 2 + T * K * 8 + T * d * 2
