@@ -8,7 +8,8 @@
 // a 256 x 256 x 16 block, with A rows 0..127 in the first CTA's shared memory
 // and rows 128..255 in the second's, and weight rows split the same way.  Per
 // SM that halves the weight bytes moved into shared memory and the number of
-// MMA instructions issued, so a stage holds 32 KB and the ring 6 stages.
+// MMA instructions issued.  A stage holds 128 columns of K (two 128-byte
+// swizzle atoms, 64 KB per CTA) and the ring 3 stages.
 //
 // A scheduled tile is a pair of 128-row m-tiles of one segment (the second
 // may lie past the segment's end; its rows are computed and not stored) and
@@ -35,14 +36,17 @@ constexpr int NUM_THREADS = 320;
 constexpr int EPI_WARPS = 8;
 constexpr int BN = 256;            // weight rows per pair tile (128 per CTA)
 constexpr int BN_HALF = BN / 2;
-constexpr int BK = 64, STAGES = 6, ACC_BUFS = 2;
+constexpr int SUB = 2;                 // 128-byte swizzle atoms of K per stage
+constexpr int BK = 64 * SUB, STAGES = 3, ACC_BUFS = 2;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
 constexpr uint64_t kDrainTimeoutNs = 200000000ull;
 
 struct Smem {
-    static constexpr int A_BYTES = BM * 128;        // 128 rows x 64 bf16
-    static constexpr int B_BYTES = BN_HALF * 128;   // 128 weight rows x 64 bf16
+    static constexpr int A_SUB = BM * 128;          // 128 rows x 64 bf16 (one swizzle atom of K)
+    static constexpr int B_SUB = BN_HALF * 128;     // 128 weight rows x 64 bf16
+    static constexpr int A_BYTES = SUB * A_SUB;
+    static constexpr int B_BYTES = SUB * B_SUB;
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
     static constexpr int OFF_BAR = OFF_B + STAGES * B_BYTES;
@@ -106,10 +110,14 @@ grouped_ffn_bf16_pair_kernel(const __grid_constant__ TcParams p) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
                     const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
                     if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (L::A_BYTES + L::B_BYTES));
-                    tma_load_2d_pair(smem + L::OFF_A + stage * L::A_BYTES, &p.a_map[ti.grp], bar0,
-                                     kb * BK, ti.a_row);
-                    tma_load_3d_pair(smem + L::OFF_B + stage * L::B_BYTES, &p.b_map[ti.grp], bar0,
-                                     kb * BK, ti.n0 + static_cast<int>(rank) * BN_HALF, ti.mat);
+#pragma unroll
+                    for (int s = 0; s < SUB; ++s) {
+                        // a K range past the end reads zeros (the MMA then adds nothing)
+                        tma_load_2d_pair(smem + L::OFF_A + stage * L::A_BYTES + s * L::A_SUB, &p.a_map[ti.grp], bar0,
+                                         kb * BK + s * 64, ti.a_row);
+                        tma_load_3d_pair(smem + L::OFF_B + stage * L::B_BYTES + s * L::B_SUB, &p.b_map[ti.grp], bar0,
+                                         kb * BK + s * 64, ti.n0 + static_cast<int>(rank) * BN_HALF, ti.mat);
+                    }
                     ++issued;
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
@@ -137,11 +145,15 @@ grouped_ffn_bf16_pair_kernel(const __grid_constant__ TcParams p) {
                 for (int kb = 0; kb < ti.kblocks; ++kb) {
                     if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
                     tc_fence_after();
-                    const uint64_t adesc = smem_desc_k_sw128(smem + L::OFF_A + stage * L::A_BYTES);
-                    const uint64_t bdesc = smem_desc_k_sw128(smem + L::OFF_B + stage * L::B_BYTES);
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        umma_f16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                    for (int s = 0; s < SUB; ++s) {
+                        const uint64_t adesc = smem_desc_k_sw128(smem + L::OFF_A + stage * L::A_BYTES + s * L::A_SUB);
+                        const uint64_t bdesc = smem_desc_k_sw128(smem + L::OFF_B + stage * L::B_BYTES + s * L::B_SUB);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            umma_f16_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc,
+                                          (kb > 0 || s > 0 || k > 0) ? 1u : 0u);
+                    }
                     issued_any = true;
                     umma_commit_pair(&empty[stage], 0x3);   // stage free in both CTAs
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
