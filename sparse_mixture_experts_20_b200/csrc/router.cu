@@ -7,9 +7,11 @@
 // The logits come from one of three producers, chosen by shape:
 //   * router_small_kernel (N_r <= 32 and W_r fits in shared memory): W_r is
 //     staged once per block by bulk asynchronous copies (one per expert row,
-//     completed on an mbarrier); each warp takes 4 (or 2) tokens, lanes split
-//     the model dimension with 16-byte loads of x, and a reduce-scatter over
-//     the lanes leaves each lane with whole dot products.  x is read once.
+//     completed on an mbarrier); each warp takes 4 (or 2) tokens and one half
+//     of the model dimension (16 warps), lanes split it with 16-byte loads of
+//     x, a reduce-scatter over the lanes leaves each lane with whole partial
+//     dot products, and the two halves are added in a fixed order.  x is read
+//     once.
 //   * the tensor-core router (router_tc.cu, bf16 x, larger N_r): W_r split into
 //     three bf16 planes, one tcgen05 GEMM with K = 3 d, partial logits per K
 //     split summed here by router_reduce_kernel;
@@ -36,7 +38,7 @@ template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v
 // lg: TT rows of EPT*32 (+1 pad) logits with the bias already added and -inf
 // in padded expert columns.  Rows of tokens >= T are ignored.  Overwrites lg
 // with s.
-template <int EPT>
+template <int EPT, int NW = NTHREADS / 32>       // NW: warps of the calling block
 __device__ __forceinline__ void select_block(float* lg_raw, int t0, int T, int E, int K,
                                              int32_t* __restrict__ topk_idx, float* __restrict__ gates,
                                              float* __restrict__ logits_out, float* __restrict__ psum) {
@@ -44,8 +46,8 @@ __device__ __forceinline__ void select_block(float* lg_raw, int t0, int T, int E
     float (*lg)[NP + 1] = reinterpret_cast<float (*)[NP + 1]>(lg_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 #pragma unroll 1
-    for (int i = 0; i < TT / 8; ++i) {
-        const int r = warp + 8 * i;
+    for (int i = 0; i < TT / NW; ++i) {
+        const int r = warp + NW * i;
         const int t = t0 + r;
         if (t >= T) {                                 // zero s so psum ignores it
 #pragma unroll
@@ -104,7 +106,7 @@ __device__ __forceinline__ void select_block(float* lg_raw, int t0, int T, int E
         }
     }
     __syncthreads();
-    for (int j = tid; j < E; j += NTHREADS) {
+    for (int j = tid; j < E; j += NW * 32) {
         float s = 0.f;
         for (int r = 0; r < TT; ++r) s += lg[r][j];
         psum[static_cast<size_t>(blockIdx.x) * E + j] = s;
@@ -207,8 +209,15 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
 
 constexpr uint64_t kStageWaitNs = 2000000000ull;
 
+// Warps of the small router: two groups of 8 (one per half of the model
+// dimension) when a warp's register tile is 32 accumulators, else one group.
+template <int NE, int RT> struct SmallCfg {
+    static constexpr int GROUPS = (RT * NE == 32) ? 2 : 1;
+    static constexpr int WARPS = 8 * GROUPS;
+};
+
 template <typename XT, int NE, int RT>
-__global__ void __launch_bounds__(NTHREADS)
+__global__ void __launch_bounds__(SmallCfg<NE, RT>::WARPS * 32)
 router_small_kernel(const XT* __restrict__ x, const float* __restrict__ W_r,
                     const float* __restrict__ logit_bias, int T, int d, int E, int K,
                     int32_t* __restrict__ topk_idx, float* __restrict__ gates,
@@ -216,8 +225,11 @@ router_small_kernel(const XT* __restrict__ x, const float* __restrict__ W_r,
     extern __shared__ float4 wsm4[];                  // (NE, d) fp32, rows >= E zero
     float* wsm = reinterpret_cast<float*>(wsm4);
     __shared__ float lg[TT][32 + 1];
+    __shared__ float lgp[2][TT][32 + 1];              // partial logits of the two halves of d
     __shared__ __align__(8) uint64_t wbar;
     __shared__ int abort_s;
+    constexpr int GROUPS = SmallCfg<NE, RT>::GROUPS;
+    constexpr int NT = SmallCfg<NE, RT>::WARPS * 32;
     constexpr int VEC = sizeof(XT) == 2 ? 8 : 4;      // elements per 16-byte load
     constexpr int NV = RT * NE;
     static_assert(NV == 32 || NV == 64, "register tile");
@@ -234,8 +246,8 @@ router_small_kernel(const XT* __restrict__ x, const float* __restrict__ W_r,
             bulk_copy_g2s(wsm + static_cast<size_t>(e) * d, W_r + static_cast<size_t>(e) * d,
                           static_cast<uint32_t>(d) * 4, &wbar);
     }
-    for (int i = E * d / 4 + tid; i < NE * d / 4; i += NTHREADS) wsm4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int i = tid; i < TT * 32; i += NTHREADS)
+    for (int i = E * d / 4 + tid; i < NE * d / 4; i += NT) wsm4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = tid; i < TT * 32; i += NT)
         if ((i & 31) >= NE) lg[i >> 5][i & 31] = -INFINITY;
     __syncthreads();
     if (!mbar_wait_bounded(&wbar, 0, &abort_s, status, kStageWaitNs)) {
@@ -244,8 +256,13 @@ router_small_kernel(const XT* __restrict__ x, const float* __restrict__ W_r,
         return;
     }
 
+    // with two groups, warps 0..7 take columns [0, d/2) of every token and
+    // warps 8..15 the rest
+    const int half = warp >> 3, wg = warp & 7;
+    const int k_begin = GROUPS == 2 ? half * (d / 2) : 0;
+    const int k_end = (GROUPS == 2 && half == 0) ? d / 2 : d;
 #pragma unroll 1
-    for (int g = warp; g < TT / RT; g += 8) {
+    for (int g = wg; g < TT / RT; g += 8) {
         float acc[NV];
 #pragma unroll
         for (int i = 0; i < NV; ++i) acc[i] = 0.f;
@@ -258,7 +275,7 @@ router_small_kernel(const XT* __restrict__ x, const float* __restrict__ W_r,
             xr[r] = x + static_cast<size_t>(ok[r] ? t : 0) * d;
         }
 #pragma unroll 4
-        for (int k = lane * VEC; k < d; k += 32 * VEC) {
+        for (int k = k_begin + lane * VEC; k < k_end; k += 32 * VEC) {
             float xv[RT][VEC];
 #pragma unroll
             for (int r = 0; r < RT; ++r) {
@@ -295,12 +312,17 @@ router_small_kernel(const XT* __restrict__ x, const float* __restrict__ W_r,
 #pragma unroll
         for (int i = 0; i < NV / 32; ++i) {
             const int vi = lane * (NV / 32) + i;
-            const int r = vi / NE, e = vi % NE;
-            lg[g * RT + r][e] = (e < E) ? acc[i] + (logit_bias ? logit_bias[e] : 0.f) : -INFINITY;
+            lgp[half][g * RT + vi / NE][vi % NE] = acc[i];
         }
     }
     __syncthreads();
-    select_block<1>(&lg[0][0], t0, T, E, K, topk_idx, gates, logits_out, psum);
+    for (int i = tid; i < TT * NE; i += NT) {         // the two halves, in a fixed order
+        const int r = i / NE, e = i % NE;
+        const float l = GROUPS == 2 ? lgp[0][r][e] + lgp[1][r][e] : lgp[0][r][e];
+        lg[r][e] = (e < E) ? l + (logit_bias ? logit_bias[e] : 0.f) : -INFINITY;
+    }
+    __syncthreads();
+    select_block<1, SmallCfg<NE, RT>::WARPS>(&lg[0][0], t0, T, E, K, topk_idx, gates, logits_out, psum);
 }
 
 // ---------------------------------------------------------------- from precomputed logits
@@ -358,7 +380,7 @@ cudaError_t launch_small_t(const Dims& dm, const void* x, const float* W_r, cons
     cudaError_t e = cudaFuncSetAttribute(router_small_kernel<XT, NE, RT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    router_small_kernel<XT, NE, RT><<<dm.route_blocks, NTHREADS, smem, st>>>(
+    router_small_kernel<XT, NE, RT><<<dm.route_blocks, SmallCfg<NE, RT>::WARPS * 32, smem, st>>>(
         static_cast<const XT*>(x), W_r, bias, dm.T, dm.d, dm.E, dm.K, idx, gates, logits, psum, status);
     count_launches();
     return cudaGetLastError();
