@@ -11,9 +11,10 @@
 // MMA instructions issued.  A stage holds 128 columns of K (two 128-byte
 // swizzle atoms, 64 KB per CTA) and the ring 3 stages.
 //
-// A scheduled tile is a pair of 128-row m-tiles of one segment (the second
-// may lie past the segment's end; its rows are computed and not stored) and
-// one 256-wide n-tile.  Each CTA loads its own A rows and its half of the
+// A scheduled tile is a pair of 128-row m-tiles of one segment and one
+// 256-wide n-tile; when a segment has an odd number of m-tiles its last one
+// runs alone as an M = 128 pair MMA (64 rows per CTA), so no MMA work is spent
+// on a whole empty m-tile.  Each CTA loads its own A rows and its half of the
 // weight rows; both TMA loads signal the first CTA's stage barrier, where the
 // single MMA-issuing thread of the pair waits.  tcgen05.commit with a CTA
 // mask releases the stage in both CTAs and announces a finished accumulator
@@ -57,6 +58,41 @@ struct Smem {
     static constexpr int TOTAL = OFF_SEG + SegTable::SEG_INTS * 4;
     static constexpr int ALLOC = TOTAL + 1024;
 };
+
+// Tile `tile` for CTA `rank` of the pair.  A segment of r rows has
+// ceil(r / 128) m-tiles, scheduled two at a time (M = 256: 128 rows per CTA).
+// An odd last m-tile is scheduled alone as an M = 128 pair MMA: 64 rows per
+// CTA, whose accumulator uses 128 tensor-memory columns: lanes 0..63 hold
+// output columns 0..127 of the 64 rows, lanes 64..127 columns 128..255 of the
+// same rows.
+struct PairTile {
+    TileInfo ti;
+    bool m128;
+};
+
+__device__ __forceinline__ PairTile decode_pair(int tile, const TcParams& p, const SegTable& t, int nseg, int rank) {
+    int lo = 0, hi = nseg - 1;                      // last s with start[s] <= tile
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (t.start[mid] <= tile) lo = mid; else hi = mid - 1;
+    }
+    const int s = lo;
+    const int local = tile - t.start[s];
+    const int mtiles = ceil_div(t.rows[s], BM);
+    const int mgroups = ceil_div(mtiles, 2);
+    const int nt = local / mgroups, g = local % mgroups;
+    PairTile pt;
+    pt.m128 = (2 * g + 1 == mtiles);
+    const int off = g * 2 * BM + rank * (pt.m128 ? BM / 2 : BM);
+    pt.ti.grp = t.mat[s] >> 16;
+    pt.ti.mat = t.mat[s] & 0xFFFF;
+    pt.ti.rows_left = t.rows[s] - off;
+    pt.ti.a_row = t.arow[s] + off;
+    pt.ti.c_row = t.crow[s] + off;
+    pt.ti.n0 = nt * BN;
+    pt.ti.kblocks = ceil_div(p.g[pt.ti.grp].K, BK);
+    return pt;
+}
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_ffn_bf16_pair_kernel(const __grid_constant__ TcParams p) {
@@ -105,7 +141,9 @@ grouped_ffn_bf16_pair_kernel(const __grid_constant__ TcParams p) {
             uint32_t phase = 0;
             bool ok = true;
             for (int tile = pair_id; tile < total_tiles && ok; tile += n_pairs) {
-                const TileInfo ti = decode_tile<BN, BK, 2>(tile, p, seg, nseg, static_cast<int>(rank));
+                // an M = 128 tile loads 128 rows from its 64-row offset; the
+                // MMA reads the first 64
+                const TileInfo ti = decode_pair(tile, p, seg, nseg, static_cast<int>(rank)).ti;
                 for (int kb = 0; kb < ti.kblocks; ++kb) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
                     const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
@@ -133,12 +171,15 @@ grouped_ffn_bf16_pair_kernel(const __grid_constant__ TcParams p) {
     } else if (warp == 1) {
         // ================= MMA issuer (first CTA of the pair)
         if (rank == 0 && lane == 0) {
-            constexpr uint32_t idesc = make_idesc(1, 2 * BM, BN);
+            constexpr uint32_t idesc256 = make_idesc(1, 2 * BM, BN);
+            constexpr uint32_t idesc128 = make_idesc(1, BM, BN);
             int stage = 0, abuf = 0;
             uint32_t phase = 0, aphase = 0;
             bool ok = true, issued_any = false;
             for (int tile = pair_id; tile < total_tiles && ok; tile += n_pairs) {
-                const TileInfo ti = decode_tile<BN, BK, 2>(tile, p, seg, nseg, 0);
+                const PairTile pt = decode_pair(tile, p, seg, nseg, 0);
+                const TileInfo& ti = pt.ti;
+                const uint32_t idesc = pt.m128 ? idesc128 : idesc256;
                 if (!mbar_wait_bounded(&acce[abuf], aphase ^ 1u, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * BN);
@@ -178,30 +219,38 @@ grouped_ffn_bf16_pair_kernel(const __grid_constant__ TcParams p) {
         int abuf = 0;
         uint32_t aphase = 0;
         for (int tile = pair_id; tile < total_tiles; tile += n_pairs) {
-            const TileInfo ti = decode_tile<BN, BK, 2>(tile, p, seg, nseg, static_cast<int>(rank));
+            const PairTile pt = decode_pair(tile, p, seg, nseg, static_cast<int>(rank));
+            const TileInfo& ti = pt.ti;
             const GroupDev& g = p.g[ti.grp];
-            const bool row_ok = r_local < ti.rows_left;
+            // M = 256: quadrant = 32 rows, warp half = 128 columns (4 chunks);
+            // M = 128: quadrants 0, 1 = rows 0..63 of columns 0..127, quadrants
+            // 2, 3 = the same rows of columns 128..255; warp half = 64 columns
+            const int r_loc = pt.m128 ? (quad & 1) * 32 + lane : r_local;
+            const int n_base = (pt.m128 && quad >= 2) ? 128 : 0;
+            const int chunk0 = pt.m128 ? half * 2 : half * 4;
+            const int n_iter = pt.m128 ? 1 : 2;
+            const bool row_ok = r_loc < ti.rows_left;
             const int n_valid = min(BN, g.N - ti.n0);
             if (!warp_wait(&accf[abuf], aphase, abort_flag, p.status, p.timeout_ns, lane)) break;
             tc_fence_after();
             __nv_bfloat16* crow = static_cast<__nv_bfloat16*>(g.C) +
-                                  static_cast<size_t>(ti.c_row + r_local) * g.N + ti.n0;
+                                  static_cast<size_t>(ti.c_row + r_loc) * g.N + ti.n0;
             const float* bias = g.bias + static_cast<size_t>(ti.mat) * g.N + ti.n0;
 #pragma unroll 1
-            for (int cc = 0; cc < 2; ++cc) {
-                const int c0 = half * 4 + cc * 2;
+            for (int cc = 0; cc < n_iter; ++cc) {
+                const int c0 = chunk0 + cc * 2;
                 uint32_t r[2][32];
                 tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>(abuf * BN + c0 * 32), r[0]);
                 tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>(abuf * BN + c0 * 32 + 32), r[1]);
                 tmem_ld_wait();
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
-                    const int c = c0 + u;
-                    if (!row_ok || c * 32 >= n_valid) continue;
+                    const int col = n_base + (c0 + u) * 32;     // output column within the tile
+                    if (!row_ok || col >= n_valid) continue;
                     uint32_t packed[16];
 #pragma unroll
                     for (int j4 = 0; j4 < 8; ++j4) {
-                        const float4 b4 = __ldg(reinterpret_cast<const float4*>(bias + c * 32) + j4);
+                        const float4 b4 = __ldg(reinterpret_cast<const float4*>(bias + col) + j4);
                         float v0 = __uint_as_float(r[u][4 * j4 + 0]) + b4.x;
                         float v1 = __uint_as_float(r[u][4 * j4 + 1]) + b4.y;
                         float v2 = __uint_as_float(r[u][4 * j4 + 2]) + b4.z;
@@ -214,7 +263,7 @@ grouped_ffn_bf16_pair_kernel(const __grid_constant__ TcParams p) {
                         packed[2 * j4] = *reinterpret_cast<uint32_t*>(&h01);
                         packed[2 * j4 + 1] = *reinterpret_cast<uint32_t*>(&h23);
                     }
-                    uint4* dst = reinterpret_cast<uint4*>(crow + c * 32);
+                    uint4* dst = reinterpret_cast<uint4*>(crow + col);
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
                         dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
