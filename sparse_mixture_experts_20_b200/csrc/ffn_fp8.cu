@@ -218,7 +218,7 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
                     float amax = 0.f;
 #pragma unroll
                     for (int j = 0; j < 128; ++j) {
-                        v[j] = silu_f32(v[j] + __ldg(bias + h * 128 + j));
+                        v[j] = silu_fast(v[j] + __ldg(bias + h * 128 + j));
                         amax = fmaxf(amax, fabsf(v[j]));
                     }
                     const float sc = pow2_scale_448(amax);
