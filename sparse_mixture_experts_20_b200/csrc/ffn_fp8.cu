@@ -13,16 +13,20 @@
 //
 // Tiles are 128 rows x 256 weight rows: one MMA instruction (K = 32) is then
 // about 128 tensor-core cycles of work, enough to hide the cost of issuing
-// it from a single thread.  The 256-column accumulator fills half of tensor
-// memory, so there is one accumulator; the epilogue releases it as soon as
-// it has read the last columns.
+// it from a single thread.  Two 256-column accumulators and the scale-factor
+// slots do not fit in the 512 columns of tensor memory, so the accumulators
+// overlap: buffer 0 is columns 0..255, buffer 1 columns 192..447, scale slots
+// 448..511.  The epilogue drains a tile's 64 overlapping columns first and
+// says so on the `ovl` barrier; the MMA of the next tile (in the other
+// buffer) starts then, while the epilogue finishes the rest.
 //
 // Per CTA (320 threads, one CTA per SM):
 //   warp 0      TMA producer: A (128 rows x 128 bytes, one scale block of K)
 //               and B (256 rows x 128 bytes) into a ring of 4 stages;
 //   warp 1      MMA issuer: per stage 4 x tcgen05.mma (K = 32 each) with the
 //               scale factors of that stage;
-//   warps 2..5  epilogue: tcgen05.ld (thread = row), bias, SiLU and the
+//   warps 2..5  epilogue: tcgen05.ld (thread = row; the overlapping columns
+//               first), bias, SiLU and the
 //               per-row e4m3 re-quantisation of the hidden activation (one
 //               scale per row per 128 columns, so the amax is thread-local),
 //               or bias and bf16 output;
@@ -47,11 +51,14 @@ using namespace ffn;
 constexpr int NUM_THREADS = 320;
 constexpr int BN = 256, BK = 128, STAGES = 4, LOOKAHEAD = 8;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t SF_COL0 = BN;                     // scale-factor slots after the accumulator
+constexpr uint32_t ACC1_COL = 192;                   // buffer 1; columns 192..255 shared with buffer 0
+constexpr uint32_t SF_COL0 = ACC1_COL + BN;          // scale-factor slots after the accumulators
 constexpr uint32_t SF_STRIDE = 16;                   // columns per stage slot (4 A + 8 B, padded)
 constexpr uint32_t FULL_ARRIVALS = 1 + 4;            // TMA expect_tx + one lane per scale-factor warp
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
 constexpr uint64_t kDrainTimeoutNs = 200000000ull;
+static_assert(SF_COL0 + STAGES * SF_STRIDE <= TMEM_COLS, "tensor memory budget");
+static_assert(BN - ACC1_COL == 64, "the epilogue drains two 32-column chunks first");
 
 struct Smem {
     static constexpr int A_BYTES = BM * 128;
@@ -59,8 +66,8 @@ struct Smem {
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
     static constexpr int OFF_BAR = OFF_B + STAGES * B_BYTES;
-    // full, empty [STAGES]; accf, acce; drain
-    static constexpr int N_BARS = 2 * STAGES + 2 + 1;
+    // full, empty [STAGES]; accf, acce [2]; ovl; drain
+    static constexpr int N_BARS = 2 * STAGES + 4 + 2;
     static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
     static constexpr int OFF_SEG = OFF_MISC + 16;
     static constexpr int TOTAL = OFF_SEG + SegTable::SEG_INTS * 4;
@@ -88,8 +95,9 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
     uint64_t* full = bars;
     uint64_t* empty = full + STAGES;
     uint64_t* accf = empty + STAGES;
-    uint64_t* acce = accf + 1;
-    uint64_t* drain = acce + 1;
+    uint64_t* acce = accf + 2;
+    uint64_t* ovl = acce + 2;
+    uint64_t* drain = ovl + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
     SegTable seg(reinterpret_cast<int*>(smem + L::OFF_SEG));
@@ -98,8 +106,8 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
     if (warp == 0) tmem_alloc<TMEM_COLS>(tmem_slot);
     if (warp == 1 && lane == 0) {
         for (int i = 0; i < STAGES; ++i) { mbar_init(&full[i], FULL_ARRIVALS); mbar_init(&empty[i], 1); }
-        mbar_init(accf, 1);
-        mbar_init(acce, 128);
+        for (int i = 0; i < 2; ++i) { mbar_init(&accf[i], 1); mbar_init(&acce[i], 128); }
+        mbar_init(ovl, 128);
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -150,13 +158,20 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
         // ================= MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc = make_idesc_mxf8(BM, BN);
-            int stage = 0;
-            uint32_t phase = 0, aphase = 0;
-            bool ok = true, issued_any = false;
+            int stage = 0, abuf = 0;
+            uint32_t phase = 0, aph0 = 0, aph1 = 0, ovl_ph = 0;
+            bool ok = true, issued_any = false, first = true;
             for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
                 const TileInfo ti = decode_tile<BN, BK>(tile, p, seg, nseg);
-                if (!mbar_wait_bounded(acce, aphase ^ 1u, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
+                // the previous tile's overlapping columns drained ...
+                if (!first && !mbar_wait_bounded(ovl, ovl_ph, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
+                if (!first) ovl_ph ^= 1u;
+                first = false;
+                // ... and this buffer's tile from two tiles back fully drained
+                uint32_t& aph = abuf ? aph1 : aph0;
+                if (!mbar_wait_bounded(&acce[abuf], aph ^ 1u, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
                 tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (abuf ? ACC1_COL : 0u);
                 for (int kb = 0; kb < ti.kblocks; ++kb) {
                     if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
                     tc_fence_after();
@@ -165,15 +180,16 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
                     const uint32_t sfa = tmem_base + SF_COL0 + static_cast<uint32_t>(stage) * SF_STRIDE;
 #pragma unroll
                     for (int k = 0; k < 4; ++k)            // 4 x 32 e4m3 of K per stage
-                        umma_mxf8_bs(tmem_base, adesc + 2 * k, bdesc + 2 * k, idesc, sfa, sfa + 4,
+                        umma_mxf8_bs(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, sfa, sfa + 4,
                                      (kb > 0 || k > 0) ? 1u : 0u);
                     issued_any = true;
                     umma_commit(&empty[stage]);             // frees the smem stage and its scale slot
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
-                umma_commit(accf);
-                aphase ^= 1u;
+                umma_commit(&accf[abuf]);
+                aph ^= 1u;
+                abuf ^= 1;
             }
             if (!ok && issued_any) {
                 umma_commit(drain);
@@ -187,32 +203,38 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
         const int quad = warp & 3;
         const int r_local = quad * 32 + lane;
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
-        uint32_t aphase = 0;
+        int abuf = 0;
+        uint32_t fph0 = 0, fph1 = 0;
         for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
             const TileInfo ti = decode_tile<BN, BK>(tile, p, seg, nseg);
             const GroupDev& g = p.g[ti.grp];
             const bool row_ok = r_local < ti.rows_left;
-            if (!warp_wait(accf, aphase, abort_flag, p.status, p.timeout_ns, lane)) break;
-            aphase ^= 1u;
+            uint32_t& fph = abuf ? fph1 : fph0;
+            if (!warp_wait(&accf[abuf], fph, abort_flag, p.status, p.timeout_ns, lane)) break;
+            fph ^= 1u;
             tc_fence_after();
+            // this tile's accumulator; its overlapping columns are 192..255 of
+            // buffer 0 (the second half) or 0..63 of buffer 1 (the first half)
+            const uint32_t acc = lane_base + (abuf ? ACC1_COL : 0u);
             const float* bias = g.bias + static_cast<size_t>(ti.mat) * g.N + ti.n0;
             if (p.out_fp8) {
-                // first layer: bias + SiLU, then one e4m3 block per 128 columns per row
+                // first layer: bias + SiLU, then one e4m3 block per 128 columns
+                // per row; the half holding the overlap goes first
 #pragma unroll 1
-                for (int h = 0; h < BN / 128; ++h) {
+                for (int hi = 0; hi < BN / 128; ++hi) {
+                    const int h = abuf ? hi : (BN / 128 - 1 - hi);
                     float v[128];
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         uint32_t r[32];
-                        tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>(h * 128 + c * 32), r);
+                        tmem_ld_32x32b_x32(acc + static_cast<uint32_t>(h * 128 + c * 32), r);
                         tmem_ld_wait();
 #pragma unroll
                         for (int j = 0; j < 32; ++j) v[c * 32 + j] = __uint_as_float(r[j]);
                     }
-                    if (h == BN / 128 - 1) {                 // accumulator fully read: release it
-                        tc_fence_before();
-                        mbar_arrive(acce);
-                    }
+                    tc_fence_before();
+                    if (hi == 0) mbar_arrive(ovl);               // overlap read: the next tile may start
+                    else mbar_arrive(&acce[abuf]);               // accumulator fully read: release it
                     const int n_blk = ti.n0 + h * 128;
                     if (!row_ok || n_blk >= g.N) continue;
                     float amax = 0.f;
@@ -239,18 +261,22 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
                     g.c_scales[static_cast<size_t>(ti.c_row + r_local) * (g.N / 128) + n_blk / 128] = sc;
                 }
             } else {
-                // second layer: bias, bf16 output
+                // second layer: bias, bf16 output; the two overlapping chunks first
                 __nv_bfloat16* crow = static_cast<__nv_bfloat16*>(g.C) +
                                       static_cast<size_t>(ti.c_row + r_local) * g.N + ti.n0;
                 const int n_valid = min(BN, g.N - ti.n0);
 #pragma unroll 1
-                for (int c = 0; c < BN / 32; ++c) {
+                for (int ci = 0; ci < BN / 32; ++ci) {
+                    const int c = abuf ? ci : (ci + 6) & 7;
                     uint32_t r[32];
-                    tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>(c * 32), r);
+                    tmem_ld_32x32b_x32(acc + static_cast<uint32_t>(c * 32), r);
                     tmem_ld_wait();
-                    if (c == BN / 32 - 1) {                  // accumulator fully read: release it
+                    if (ci == 1) {                               // overlap read: the next tile may start
                         tc_fence_before();
-                        mbar_arrive(acce);
+                        mbar_arrive(ovl);
+                    } else if (ci == BN / 32 - 1) {              // accumulator fully read: release it
+                        tc_fence_before();
+                        mbar_arrive(&acce[abuf]);
                     }
                     if (row_ok && c * 32 < n_valid) {
                         uint32_t packed[16];
@@ -268,6 +294,7 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
                     }
                 }
             }
+            abuf ^= 1;
         }
     } else {
         // ================= scale-factor writers (warps 6..9)
