@@ -345,6 +345,14 @@ __device__ __forceinline__ float pow2_scale_448(float amax) {
     return __uint_as_float(static_cast<uint32_t>(k + 127) << 23);
 }
 
+// 1 / s for a power of two s = 2^k, k in [-126, 127], exactly and without a
+// division: the exponent field of 2^-k is 254 minus that of s; 2^-127 is the
+// one subnormal result.
+__device__ __forceinline__ float inv_pow2(float s) {
+    const uint32_t e = (__float_as_uint(s) >> 23) & 0xFFu;
+    return e < 254u ? __uint_as_float((254u - e) << 23) : __uint_as_float(0x00400000u);
+}
+
 __device__ __forceinline__ float silu_f32(float z) {
     return z / (1.0f + __expf(-z));
 }

@@ -241,7 +241,7 @@ scatter_kernel(const void* __restrict__ x_, const int32_t* __restrict__ topk_idx
                 for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off, 16));
                 if (c >= nchunks) continue;
                 const float sc = pow2_scale_448(amax);
-                const float inv = 1.0f / sc;                     // exact: power of two
+                const float inv = inv_pow2(sc);                  // exact: power of two
                 uint2 q;
                 q.x = static_cast<uint32_t>(f32x2_to_e4m3x2(v[0] * inv, v[1] * inv)) |
                       (static_cast<uint32_t>(f32x2_to_e4m3x2(v[2] * inv, v[3] * inv)) << 16);

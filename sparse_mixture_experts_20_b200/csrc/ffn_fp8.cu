@@ -238,13 +238,19 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
                     const int n_blk = ti.n0 + h * 128;
                     if (!row_ok || n_blk >= g.N) continue;
                     float amax = 0.f;
+                    const float4* b4 = reinterpret_cast<const float4*>(bias + h * 128);
 #pragma unroll
-                    for (int j = 0; j < 128; ++j) {
-                        v[j] = silu_fast(v[j] + __ldg(bias + h * 128 + j));
-                        amax = fmaxf(amax, fabsf(v[j]));
+                    for (int j4 = 0; j4 < 32; ++j4) {
+                        const float4 b = __ldg(b4 + j4);
+                        v[4 * j4 + 0] = silu_fast(v[4 * j4 + 0] + b.x);
+                        v[4 * j4 + 1] = silu_fast(v[4 * j4 + 1] + b.y);
+                        v[4 * j4 + 2] = silu_fast(v[4 * j4 + 2] + b.z);
+                        v[4 * j4 + 3] = silu_fast(v[4 * j4 + 3] + b.w);
+                        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[4 * j4]), fabsf(v[4 * j4 + 1])),
+                                                 fmaxf(fabsf(v[4 * j4 + 2]), fabsf(v[4 * j4 + 3]))));
                     }
                     const float sc = pow2_scale_448(amax);
-                    const float inv = 1.0f / sc;             // exact: sc is a power of two
+                    const float inv = inv_pow2(sc);          // exact: sc is a power of two
                     uint8_t* crow = static_cast<uint8_t*>(g.C) + static_cast<size_t>(ti.c_row + r_local) * g.N + n_blk;
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
@@ -280,12 +286,16 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
                     }
                     if (row_ok && c * 32 < n_valid) {
                         uint32_t packed[16];
+                        const float4* b4 = reinterpret_cast<const float4*>(bias + c * 32);
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) {
-                            __nv_bfloat162 h2 = __floats2bfloat162_rn(
-                                __uint_as_float(r[2 * j]) + __ldg(bias + c * 32 + 2 * j),
-                                __uint_as_float(r[2 * j + 1]) + __ldg(bias + c * 32 + 2 * j + 1));
-                            packed[j] = *reinterpret_cast<uint32_t*>(&h2);
+                        for (int j4 = 0; j4 < 8; ++j4) {
+                            const float4 b = __ldg(b4 + j4);
+                            __nv_bfloat162 lo = __floats2bfloat162_rn(__uint_as_float(r[4 * j4 + 0]) + b.x,
+                                                                      __uint_as_float(r[4 * j4 + 1]) + b.y);
+                            __nv_bfloat162 hi = __floats2bfloat162_rn(__uint_as_float(r[4 * j4 + 2]) + b.z,
+                                                                      __uint_as_float(r[4 * j4 + 3]) + b.w);
+                            packed[2 * j4] = *reinterpret_cast<uint32_t*>(&lo);
+                            packed[2 * j4 + 1] = *reinterpret_cast<uint32_t*>(&hi);
                         }
                         uint4* dst = reinterpret_cast<uint4*>(crow + c * 32);
 #pragma unroll
