@@ -254,5 +254,65 @@ class MoELayer:
                           self.topk_idx, self.gates, self.counts, self.ws, stream)
         return self.out, self.f, self.P, self.loss
 
+    def _forward_into(self, x, out, loss, stream=None):
+        w = self.w
+        g = lambda k: w.get(k)  # noqa: E731
+        moe_layer_forward(self.cfg, x, g("W_r"), g("logit_bias"), g("W1"), g("W1_scales"), g("b1"),
+                          g("W2"), g("W2_scales"), g("b2"), g("Ws1"), g("Ws1_scales"), g("bs1"),
+                          g("Ws2"), g("Ws2_scales"), g("bs2"), out, self.f, self.P, loss,
+                          self.topk_idx, self.gates, self.counts, self.ws, stream)
+
+    def forward_host_batches(self, x_hosts, out_hosts, loss_hosts, between=None):
+        """Runs the layer on consecutive batches that live in pinned host
+        memory and writes each batch's output and loss back to host memory.
+
+        Batch k's host->device copy runs on a copy-in stream and its
+        device->host copies on a copy-out stream, so they overlap the compute
+        of batches k-1 and k+1 (device inputs and outputs are double-buffered;
+        events order the three streams).  `between`, if given, is called on
+        the compute stream before each batch.  Returns the (start, end) CUDA
+        events that bracket the whole run: the first input copy to the last
+        output copy.  f, P, topk_idx, gates and counts hold the last batch's."""
+        import torch
+        dev = self.device
+        n = len(x_hosts)
+        assert len(out_hosts) == n and len(loss_hosts) == n
+        cur = torch.cuda.current_stream(dev)
+        s_in = torch.cuda.Stream(device=dev)
+        s_out = torch.cuda.Stream(device=dev)
+        x_dev = [torch.empty_like(x_hosts[0], device=dev) for _ in range(2)]
+        out_dev = [torch.empty_like(self.out) for _ in range(2)]
+        loss_dev = [torch.empty_like(self.loss) for _ in range(2)]
+        ev = lambda: torch.cuda.Event()  # noqa: E731
+        in_ready = [ev(), ev()]
+        computed = [ev(), ev()]
+        copied_out = [ev(), ev()]
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s_in.wait_stream(cur)
+        s_out.wait_stream(cur)
+        start.record(s_in)
+        for k in range(n):
+            b = k & 1
+            with torch.cuda.stream(s_in):
+                if k >= 2:
+                    s_in.wait_event(computed[b])            # x_dev[b] no longer read
+                x_dev[b].copy_(x_hosts[k], non_blocking=True)
+                in_ready[b].record(s_in)
+            cur.wait_event(in_ready[b])
+            if k >= 2:
+                cur.wait_event(copied_out[b])               # out_dev[b] already copied back
+            if between is not None:
+                between()
+            self._forward_into(x_dev[b], out_dev[b], loss_dev[b], stream=cur)
+            computed[b].record(cur)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(computed[b])
+                out_hosts[k].copy_(out_dev[b], non_blocking=True)
+                loss_hosts[k].copy_(loss_dev[b], non_blocking=True)
+                copied_out[b].record(s_out)
+        end.record(s_out)
+        cur.wait_stream(s_out)
+        return start, end
+
     def device_status(self, clear: bool = False) -> int:
         return moe_get_device_status(self.cfg, self.ws, clear=clear)

@@ -137,3 +137,24 @@ def test_layer_is_deterministic():
     a = TL.run_layer(sh, inp)
     b = TL.run_layer(sh, inp)
     assert torch.equal(a["out"], b["out"]) and torch.equal(a["P"], b["P"]) and torch.equal(a["loss"], b["loss"])
+
+
+def test_host_batches_pipeline_matches_forward():
+    """MoELayer.forward_host_batches (copies on their own streams, double
+    buffers) returns, for every batch, exactly what forward() returns."""
+    require_gpu()
+    sh = CASES["bf16-ragged-shared-cap"]
+    inp = TL.gpu_inputs(sh, seed=7)
+    layer = M.MoELayer(M.make_config(sh), inp, device=inp["x"].device)
+    gen = torch.Generator().manual_seed(11)
+    xs = [torch.randn(sh.T, sh.d_model, generator=gen).to(torch.bfloat16).pin_memory() for _ in range(5)]
+    outs = [torch.empty(sh.T, sh.d_model, dtype=torch.bfloat16).pin_memory() for _ in range(5)]
+    losses = [torch.empty(1, dtype=torch.float32).pin_memory() for _ in range(5)]
+    layer.forward_host_batches(xs, outs, losses)
+    torch.cuda.synchronize()
+    assert layer.device_status() == 0
+    for k in range(5):
+        out, _, _, loss = layer.forward(xs[k].to(inp["x"].device))
+        torch.cuda.synchronize()
+        assert torch.equal(outs[k], out.cpu()), k
+        assert torch.equal(losses[k], loss.cpu()), k
