@@ -45,6 +45,7 @@ masked) gives the same output; brute-force top-K over all K-subsets on tiny
 inputs; the C(8,2) = 28 and C(16,2) = 120 selected-set counts; active-parameter
 fraction K/N_r; balance loss closed forms (uniform routing gives alpha, a
 collapsed router gives alpha * N_r); the first C tokens kept under capacity;
+hand-computed capacities (including fp32 values of the capacity factor);
 the e4m3 and bf16 rounding against torch's conversions.  The expert FFN
 arithmetic beyond these is pinned only through the dense limit.
 """

@@ -335,3 +335,18 @@ def test_fp8_layer_dense_limit():
     y = F.linear(q_rows(h), deq_w(inp["W2"][0], inp["W2_scales"][0]), inp["b2"][0].double())
     y = y.to(torch.bfloat16).double()   # single rounding: y is one expert with gate 1
     assert np.array_equal(out, y.numpy())
+
+
+@pytest.mark.parametrize("T,K,N,cf,expected", [
+    (8192, 8, 64, 1.25, 1280),   # DeepSeekMoE-style workload: 1.25 * 8192 * 8 / 64 exactly
+    (203, 2, 6, 1.0, 68),        # 406 / 6 = 67.67 -> 68
+    (777, 2, 8, 1.1, 214),       # fp32(1.1) = 1.10000002384...; * 194.25 = 213.675 -> 214
+    (6, 1, 3, 0.5, 1),           # exactly 1: no rounding up
+    (10, 1, 1, 0.1, 2),          # fp32(0.1) = 0.10000000149... > 0.1: 1.0000000149 -> 2
+    (64, 2, 8, 0.0, None),       # no capacity limit
+    (64, 2, 8, -1.0, None),
+])
+def test_capacity_hand_computed_values(T, K, N, cf, expected):
+    """[TopK] §解決策2: C = ceil(cf * T * K / N_r) on the fp32 value of cf
+    (the value the C interface receives); expected values worked by hand."""
+    assert O.capacity_of(T, K, N, cf) == expected
