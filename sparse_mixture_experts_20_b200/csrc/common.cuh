@@ -66,10 +66,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // completed.  Returns false when *abort_flag became non-zero (another role of
 // the block gave up) or when timeout_ns elapsed; in the latter case it sets
 // *abort_flag and records MOE_DEV_TIMEOUT in *status.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
-                                                  volatile int* abort_flag,
-                                                  int32_t* status, uint64_t timeout_ns) {
-    if (mbar_try_wait(bar, parity)) return true;
+// The spin is out of line so that the many call sites of a warp-specialised
+// kernel do not each carry a copy of it (instruction-cache pressure); the
+// first try stays inline.
+static __device__ __noinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                   int32_t* status, uint64_t timeout_ns) {
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -82,6 +83,13 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
             }
         }
     }
+}
+
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
+                                                  volatile int* abort_flag,
+                                                  int32_t* status, uint64_t timeout_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return mbar_wait_spin(bar, parity, abort_flag, status, timeout_ns);
 }
 
 // ---------------------------------------------------------------- TMA

@@ -350,28 +350,33 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
         }
         int stage = 0;
         uint32_t phase = 0;
-        bool ok = true;
-        while (ok && valid(cur)) {
+#pragma unroll 1
+        while (valid(cur)) {
+            // the oldest prefetched scales; the ring shifts by one (register
+            // moves only, so the loop body exists once)
+            const uint32_t wa0 = ue8m0_x4(ra[0][0]), wa1 = ue8m0_x4(ra[0][1]);
+            const uint32_t wa2 = ue8m0_x4(ra[0][2]), wa3 = ue8m0_x4(ra[0][3]);
+            const uint32_t wb0 = ue8m0_x4(rb[0][0]), wb1 = ue8m0_x4(rb[0][1]);
 #pragma unroll
-            for (int j = 0; j < LOOKAHEAD; ++j) {
-                if (!valid(cur)) break;
-                const uint32_t wa0 = ue8m0_x4(ra[j][0]), wa1 = ue8m0_x4(ra[j][1]);
-                const uint32_t wa2 = ue8m0_x4(ra[j][2]), wa3 = ue8m0_x4(ra[j][3]);
-                const uint32_t wb0 = ue8m0_x4(rb[j][0]), wb1 = ue8m0_x4(rb[j][1]);
-                if (valid(ahead)) { load(ahead, ra[j], rb[j]); advance(ahead); }
-                if (!warp_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, p.timeout_ns, lane)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t slot = sf_base + static_cast<uint32_t>(stage) * SF_STRIDE;
-                tmem_st_32x32b_x4(slot, wa0, wa1, wa2, wa3);
-                tmem_st_32x32b_x4(slot + 4, wb0, wb0, wb0, wb0);
-                tmem_st_32x32b_x4(slot + 8, wb1, wb1, wb1, wb1);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&full[stage]);
-                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-                advance(cur);
+            for (int j = 0; j + 1 < LOOKAHEAD; ++j) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) ra[j][c] = ra[j + 1][c];
+                rb[j][0] = rb[j + 1][0];
+                rb[j][1] = rb[j + 1][1];
             }
+            if (valid(ahead)) { load(ahead, ra[LOOKAHEAD - 1], rb[LOOKAHEAD - 1]); advance(ahead); }
+            if (!warp_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, p.timeout_ns, lane)) break;
+            tc_fence_after();
+            const uint32_t slot = sf_base + static_cast<uint32_t>(stage) * SF_STRIDE;
+            tmem_st_32x32b_x4(slot, wa0, wa1, wa2, wa3);
+            tmem_st_32x32b_x4(slot + 4, wb0, wb0, wb0, wb0);
+            tmem_st_32x32b_x4(slot + 8, wb1, wb1, wb1, wb1);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&full[stage]);
+            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            advance(cur);
         }
     }
 
