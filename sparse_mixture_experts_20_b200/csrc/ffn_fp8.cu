@@ -31,7 +31,7 @@
 //               scale per row per 128 columns, so the amax is thread-local),
 //               or bias and bf16 output;
 //   warps 6..9  scale-factor writers: per stage, the 128 row scales of A and
-//               the two block scales of B (prefetched 8 stages ahead) as
+//               the two block scales of B (prefetched 4 stages ahead) as
 //               UE8M0, written with tcgen05.st into the stage's slot of
 //               tensor memory; they arrive on the stage's full barrier next to
 //               the TMA bytes, and wait on its empty barrier like the
@@ -49,7 +49,7 @@ namespace {
 using namespace ffn;
 
 constexpr int NUM_THREADS = 320;
-constexpr int BN = 256, BK = 128, STAGES = 4, LOOKAHEAD = 8;
+constexpr int BN = 256, BK = 128, STAGES = 4, LOOKAHEAD = 4;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC1_COL = 192;                   // buffer 1; columns 192..255 shared with buffer 0
 constexpr uint32_t SF_COL0 = ACC1_COL + BN;          // scale-factor slots after the accumulators

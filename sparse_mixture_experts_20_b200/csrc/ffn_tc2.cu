@@ -59,7 +59,9 @@ struct Smem {
     static constexpr int ALLOC = TOTAL + 1024;
 };
 
-// Tile `tile` for CTA `rank` of the pair.  A segment of r rows has
+// Tile `tile` for CTA `rank` of the pair (a last n-tile with at most 128
+// valid columns runs as an N = 128 pair MMA, 64 weight rows per CTA).  A
+// segment of r rows has
 // ceil(r / 128) m-tiles, scheduled two at a time (M = 256: 128 rows per CTA).
 // An odd last m-tile is scheduled alone as an M = 128 pair MMA: 64 rows per
 // CTA, whose accumulator uses 128 tensor-memory columns: lanes 0..63 hold
@@ -68,6 +70,7 @@ struct Smem {
 struct PairTile {
     TileInfo ti;
     bool m128;
+    bool n128;      // last n-tile with at most 128 valid columns: an N = 128 MMA
 };
 
 __device__ __forceinline__ PairTile decode_pair(int tile, const TcParams& p, const SegTable& t, int nseg, int rank) {
@@ -91,6 +94,8 @@ __device__ __forceinline__ PairTile decode_pair(int tile, const TcParams& p, con
     pt.ti.c_row = t.crow[s] + off;
     pt.ti.n0 = nt * BN;
     pt.ti.kblocks = ceil_div(p.g[pt.ti.grp].K, BK);
+    // (not combined with M = 128, whose accumulator layout folds N)
+    pt.n128 = !pt.m128 && p.g[pt.ti.grp].N - pt.ti.n0 <= BN_HALF;
     return pt;
 }
 
@@ -143,7 +148,10 @@ grouped_ffn_bf16_pair_kernel(const __grid_constant__ TcParams p) {
             for (int tile = pair_id; tile < total_tiles && ok; tile += n_pairs) {
                 // an M = 128 tile loads 128 rows from its 64-row offset; the
                 // MMA reads the first 64
-                const TileInfo ti = decode_pair(tile, p, seg, nseg, static_cast<int>(rank)).ti;
+                const PairTile pt = decode_pair(tile, p, seg, nseg, static_cast<int>(rank));
+                const TileInfo& ti = pt.ti;
+                // an N = 128 tile: each CTA holds 64 weight rows (the box reads 128)
+                const int b_row = ti.n0 + static_cast<int>(rank) * (pt.n128 ? BN_HALF / 2 : BN_HALF);
                 for (int kb = 0; kb < ti.kblocks; ++kb) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
                     const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
@@ -154,7 +162,7 @@ grouped_ffn_bf16_pair_kernel(const __grid_constant__ TcParams p) {
                         tma_load_2d_pair(smem + L::OFF_A + stage * L::A_BYTES + s * L::A_SUB, &p.a_map[ti.grp], bar0,
                                          kb * BK + s * 64, ti.a_row);
                         tma_load_3d_pair(smem + L::OFF_B + stage * L::B_BYTES + s * L::B_SUB, &p.b_map[ti.grp], bar0,
-                                         kb * BK + s * 64, ti.n0 + static_cast<int>(rank) * BN_HALF, ti.mat);
+                                         kb * BK + s * 64, b_row, ti.mat);
                     }
                     ++issued;
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -173,13 +181,14 @@ grouped_ffn_bf16_pair_kernel(const __grid_constant__ TcParams p) {
         if (rank == 0 && lane == 0) {
             constexpr uint32_t idesc256 = make_idesc(1, 2 * BM, BN);
             constexpr uint32_t idesc128 = make_idesc(1, BM, BN);
+            constexpr uint32_t idesc256n = make_idesc(1, 2 * BM, BN_HALF);
             int stage = 0, abuf = 0;
             uint32_t phase = 0, aphase = 0;
             bool ok = true, issued_any = false;
             for (int tile = pair_id; tile < total_tiles && ok; tile += n_pairs) {
                 const PairTile pt = decode_pair(tile, p, seg, nseg, 0);
                 const TileInfo& ti = pt.ti;
-                const uint32_t idesc = pt.m128 ? idesc128 : idesc256;
+                const uint32_t idesc = pt.m128 ? idesc128 : (pt.n128 ? idesc256n : idesc256);
                 if (!mbar_wait_bounded(&acce[abuf], aphase ^ 1u, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * BN);
@@ -227,8 +236,10 @@ grouped_ffn_bf16_pair_kernel(const __grid_constant__ TcParams p) {
             // 2, 3 = the same rows of columns 128..255; warp half = 64 columns
             const int r_loc = pt.m128 ? (quad & 1) * 32 + lane : r_local;
             const int n_base = (pt.m128 && quad >= 2) ? 128 : 0;
-            const int chunk0 = pt.m128 ? half * 2 : half * 4;
-            const int n_iter = pt.m128 ? 1 : 2;
+            // (an N = 128 tile: 128 columns, 64 per warp half, like M = 128)
+            const bool narrow = pt.m128 || pt.n128;
+            const int chunk0 = narrow ? half * 2 : half * 4;
+            const int n_iter = narrow ? 1 : 2;
             const bool row_ok = r_loc < ti.rows_left;
             const int n_valid = min(BN, g.N - ti.n0);
             if (!warp_wait(&accf[abuf], aphase, abort_flag, p.status, p.timeout_ns, lane)) break;
