@@ -444,6 +444,10 @@ def run_ours(args):
     roof["peak_source"] = (f"{peak_src} ({'bf16 burst x2 nominal fp8/bf16 ratio' if fp8 else 'bf16 burst'})"
                            if roof["bound"] == "tensor" else f"{peak_src} HBM copy")
     roof["traffic"] = traffic_from_profile(sh.name, kname, src_hash(kfiles))
+    # the nominal B200 peaks the targets are written against (dense bf16
+    # 2.25 PF, fp8 4.5 PF, HBM 8 TB/s), beside the measured ones
+    spec = (4500.0 if fp8 else 2250.0) if roof["bound"] == "tensor" else 8000.0
+    roof["frac_of_spec_peak"] = round(roof["achieved"] / spec, 4)
     if roof["bound"] == "tensor":
         # a dense GEMM at the 1 kW power cap runs below the burst clock: the
         # sustained measured peak, for context
