@@ -304,21 +304,40 @@ def balance_stats(counts: np.ndarray, s: np.ndarray, K: int, alpha: float):
 def route(shape, inputs, logits: Optional[np.ndarray] = None):
     """Router, top-K, gates, plan and balance statistics for all T tokens.
 
+    A per-expert bias b is used in one of two ways (shape.bias_mode):
+      0  added to the logits: s, top-K, gates and P all see l + b (the decode
+         workload's skew);
+      1  selection only ([TopK] §解決策3, auxiliary-loss-free balancing: a
+         per-expert bias steers which experts are chosen, the loss is not
+         changed): top-K on l + b, while s, the gates and P use the unbiased
+         l.  The pages give no formula; this is the plainest reading.
+
     `logits`, when given, replaces the oracle's own fp64 logits as the
     selection keys (used to check the product's routing bit-exactly on its own
-    fp32 logits); s and P still come from the oracle's fp64 logits."""
+    fp32 logits -- those are l + b in mode 0 and l in mode 1, to which the
+    bias is then added in fp32 as the kernel does); s and P still come from
+    the oracle's fp64 logits."""
     x = to_f64(inputs["x"])
     lb = inputs.get("logit_bias")
-    l64 = router_logits(x, to_f64(inputs["W_r"]), None if lb is None else to_f64(lb))
+    mode = getattr(shape, "bias_mode", 0)
+    sel_bias = None if (lb is None or mode != 1) else to_f64(lb)
+    l64 = router_logits(x, to_f64(inputs["W_r"]), None if (lb is None or mode == 1) else to_f64(lb))
     s = softmax(l64)
-    keys = l64 if logits is None else np.asarray(logits, np.float64)
+    keys64 = l64 if sel_bias is None else l64 + sel_bias[None, :]
+    if logits is None:
+        keys = keys64
+    elif sel_bias is None:
+        keys = np.asarray(logits, np.float64)
+    else:
+        b32 = np.asarray(to_f64(lb), np.float32)
+        keys = (np.asarray(logits, np.float32) + b32[None, :]).astype(np.float64)
     idx = topk_select(keys, shape.top_k)
     g = gates_of(s, idx)
     C = capacity_of(shape.T, shape.top_k, shape.n_routed, shape.capacity_factor)
     plan = dispatch_plan(idx, shape.n_routed, C)
     f, P, L = balance_stats(plan["counts"], s, shape.top_k, shape.alpha)
     return {"logits": l64, "s": s, "idx": idx, "gates": g, "C": C, "plan": plan,
-            "f": f, "P": P, "loss": L, "gap": topk_gap(l64, shape.top_k)}
+            "f": f, "P": P, "loss": L, "gap": topk_gap(keys64, shape.top_k)}
 
 
 def expert_weights(inputs, prefix: str, e: int, fp8: bool):

@@ -46,6 +46,11 @@ class MoEShape:
     alpha: float = 0.01
     dtype: int = DTYPE_BF16
     zipf_logit_bias: bool = False
+    # how the per-expert bias is used: 0 = added to the logits (softmax, top-K,
+    # gates and P all see it); 1 = selection only (top-K on logits + bias,
+    # softmax, gates and P on the unbiased logits)
+    bias_mode: int = 0
+    selection_bias: bool = False   # draw a N(0, 0.5^2) per-expert bias
 
     def replace(self, **kw) -> "MoEShape":
         return dataclasses.replace(self, **kw)
@@ -138,6 +143,8 @@ def make_inputs(shape: MoEShape, seed: int = 0, device="cpu",
     if shape.zipf_logit_bias:
         rank = torch.randperm(E, generator=gen, device=device).to(torch.float64) + 1.0
         out["logit_bias"] = (1.5 * torch.log(1.0 / rank)).float()
+    elif shape.selection_bias:
+        out["logit_bias"] = _normal(gen, (E,), 0.5, device)
     if route_only:
         return out
     bias_std = 0.1  # N(0, 0.01): variance 0.01

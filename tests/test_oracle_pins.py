@@ -350,3 +350,44 @@ def test_capacity_hand_computed_values(T, K, N, cf, expected):
     """[TopK] §解決策2: C = ceil(cf * T * K / N_r) on the fp32 value of cf
     (the value the C interface receives); expected values worked by hand."""
     assert O.capacity_of(T, K, N, cf) == expected
+
+
+# ---------------------------------------------------------------------------
+# Selection-only bias ([TopK] §解決策3: auxiliary-loss-free balancing steers
+# the choice of experts with a per-expert bias without changing the loss).
+
+
+def _one_token(bias, mode):
+    from synthetic import MoEShape
+    sh = MoEShape("t", 1, 1, 4, 2, 64, bias_mode=mode, dtype=0)
+    inp = {"x": np.array([[1.0]]), "W_r": np.array([[2.0], [1.0], [0.0], [-1.0]]),
+           "logit_bias": None if bias is None else np.asarray(bias, np.float64)}
+    return O.route(sh, inp)
+
+
+def test_selection_bias_hand_computed():
+    """l = [2, 1, 0, -1], b = [0, 0, 0, 10]: expert 3 is chosen first
+    (key 9), expert 0 second (key 2); the gates come from the unbiased
+    softmax: g = [e^-1, e^2] / (e^-1 + e^2) = [1/(1+e^3), e^3/(1+e^3)]."""
+    r = _one_token([0.0, 0.0, 0.0, 10.0], 1)
+    assert r["idx"].tolist() == [[3, 0]]
+    assert r["gates"][0, 0] == pytest.approx(0.04742587317756678, rel=1e-14)
+    assert r["gates"][0, 1] == pytest.approx(0.9525741268224334, rel=1e-14)
+    # P is the unbiased softmax of the single token
+    e = np.exp(np.array([2.0, 1.0, 0.0, -1.0]))
+    assert np.allclose(r["P"], e / e.sum(), rtol=0, atol=1e-15)
+
+
+def test_logit_bias_mode_uses_biased_softmax():
+    """Same numbers with the bias in the logits: keys and softmax both see
+    l + b = [2, 1, 0, 9], so g = [e^9, e^2] / (e^9 + e^2)."""
+    r = _one_token([0.0, 0.0, 0.0, 10.0], 0)
+    assert r["idx"].tolist() == [[3, 0]]
+    assert r["gates"][0, 0] == pytest.approx(1.0 / (1.0 + math.exp(-7.0)), rel=1e-14)
+
+
+def test_selection_bias_zero_changes_nothing():
+    a = _one_token([0.0, 0.0, 0.0, 0.0], 1)
+    b = _one_token(None, 0)
+    assert a["idx"].tolist() == b["idx"].tolist() == [[0, 1]]
+    assert np.array_equal(a["gates"], b["gates"]) and np.array_equal(a["P"], b["P"])
