@@ -107,7 +107,18 @@ typedef struct {
     float   capacity_factor; /* 0 = no capacity limit                             */
     float   alpha;           /* balance weight (the pages recommend 0.01)         */
     int32_t dtype;           /* MOE_F32 | MOE_BF16 | MOE_FP8_E4M3_BLOCK           */
+    int32_t bias_mode;       /* how logit_bias is used (see MOE_BIAS_*)           */
 } moe_config;
+
+/* bias_mode.  MOE_BIAS_LOGITS: the per-expert bias is added to the router
+ * logits, so softmax, top-K, gates and P all see it.  MOE_BIAS_SELECTION:
+ * the bias enters only the top-K keys (l + b); softmax, gates and P use the
+ * unbiased logits -- the auxiliary-loss-free balancing of "Sparse MoE
+ * Top-Kルーティング" §解決策3, where a per-expert bias steers which experts
+ * are chosen without changing the loss (the pages give no formula; this is
+ * the plainest reading).  logits_out holds the softmax logits (l + b, or l). */
+#define MOE_BIAS_LOGITS     0
+#define MOE_BIAS_SELECTION  1
 
 /* ---- sizing helpers (host only, no GPU work) ------------------------------ */
 
@@ -148,8 +159,9 @@ MOE_EXPORT const char* moe_status_string(int status);
 MOE_EXPORT uint64_t moe_kernel_launches(void);
 
 /* ---- stage 1: router ------------------------------------------------------
- * l[t,j] = sum_i x[t,i] W_r[j,i] (+ logit_bias[j]) in fp32; s = softmax(l);
- * topk_idx[t,k] = the K largest l (ties -> lower j), descending;
+ * l[t,j] = sum_i x[t,i] W_r[j,i] (+ logit_bias[j] with MOE_BIAS_LOGITS) in
+ * fp32; s = softmax(l); topk_idx[t,k] = the K largest keys l (+ logit_bias[j]
+ * with MOE_BIAS_SELECTION, added in fp32), ties -> lower j, descending;
  * gates[t,k] = s[t,topk_idx[t,k]] / sum_k' s[t,topk_idx[t,k']].
  * Also writes per-block partial sums of s into ws for moe_balance_stats.
  *   x          (T, d_model) fp32 (MOE_F32) or bf16

@@ -29,6 +29,7 @@ MOE_ERR_DEVICE_TIMEOUT = 5
 MOE_DEV_BAD_ROUTING = 0x1
 MOE_DEV_TIMEOUT = 0x2
 MOE_F32, MOE_BF16, MOE_FP8_E4M3_BLOCK = 0, 1, 2
+MOE_BIAS_LOGITS, MOE_BIAS_SELECTION = 0, 1
 
 EXPORTED = (
     "moe_workspace_size", "moe_buffer_rows", "moe_workspace_init", "moe_get_device_status",
@@ -43,7 +44,7 @@ class moe_config(ctypes.Structure):
         ("T", ctypes.c_int32), ("d_model", ctypes.c_int32), ("n_routed", ctypes.c_int32),
         ("top_k", ctypes.c_int32), ("d_ff", ctypes.c_int32), ("n_shared", ctypes.c_int32),
         ("d_ff_shared", ctypes.c_int32), ("capacity_factor", ctypes.c_float),
-        ("alpha", ctypes.c_float), ("dtype", ctypes.c_int32),
+        ("alpha", ctypes.c_float), ("dtype", ctypes.c_int32), ("bias_mode", ctypes.c_int32),
     ]
 
 
@@ -100,8 +101,8 @@ def lib() -> ctypes.CDLL:
 
 def make_config(shape=None, **kw) -> moe_config:
     """moe_config from any object with the fields T, d_model, n_routed, top_k,
-    d_ff, n_shared, d_ff_shared, capacity_factor, alpha, dtype (keyword
-    arguments override)."""
+    d_ff, n_shared, d_ff_shared, capacity_factor, alpha, dtype, bias_mode
+    (keyword arguments override)."""
     fields = [f for f, _ in moe_config._fields_]
     vals = {f: getattr(shape, f) for f in fields if shape is not None and hasattr(shape, f)}
     vals.update(kw)
@@ -110,6 +111,7 @@ def make_config(shape=None, **kw) -> moe_config:
     vals.setdefault("capacity_factor", 0.0)
     vals.setdefault("alpha", 0.01)
     vals.setdefault("dtype", MOE_BF16)
+    vals.setdefault("bias_mode", MOE_BIAS_LOGITS)
     return moe_config(**{f: vals[f] for f in fields})
 
 

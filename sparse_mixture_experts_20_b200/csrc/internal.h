@@ -38,6 +38,7 @@ struct Dims {
     int x_disp_rows;
     int y_rows;
     int dtype;
+    int bias_mode;  // 0: logit_bias enters the logits; 1: only the top-K keys
     float alpha;
     int route_blocks;
     int t_words;

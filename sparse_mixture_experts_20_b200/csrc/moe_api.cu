@@ -58,6 +58,7 @@ int validate(const moe_config* cfg, Dims* dm) {
     if (!std::isfinite(c.capacity_factor) || c.capacity_factor < 0.f || !std::isfinite(c.alpha))
         return MOE_ERR_INVALID_ARG;
     if (c.dtype != MOE_F32 && c.dtype != MOE_BF16 && c.dtype != MOE_FP8_E4M3_BLOCK) return MOE_ERR_INVALID_ARG;
+    if (c.bias_mode != MOE_BIAS_LOGITS && c.bias_mode != MOE_BIAS_SELECTION) return MOE_ERR_INVALID_ARG;
     if (c.n_routed > 256 || c.top_k > 16 || c.n_shared > 8) return MOE_ERR_UNSUPPORTED;
     const int q = c.dtype == MOE_FP8_E4M3_BLOCK ? 128 : 64;
     if (c.d_model % q || c.d_ff % q || (c.n_shared > 0 && c.d_ff_shared % q)) return MOE_ERR_UNSUPPORTED;
@@ -72,6 +73,7 @@ int validate(const moe_config* cfg, Dims* dm) {
     dm->S = c.n_shared;
     dm->dffs = c.n_shared > 0 ? c.d_ff_shared : 0;
     dm->dtype = c.dtype;
+    dm->bias_mode = c.bias_mode;
     dm->alpha = c.alpha;
     dm->capacity = capacity_of(c.capacity_factor, c.T, c.top_k, c.n_routed);
     long long rcap = static_cast<long long>(c.T) * c.top_k;

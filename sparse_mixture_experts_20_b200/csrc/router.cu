@@ -35,13 +35,16 @@ template <typename XT> __device__ __forceinline__ float to_f(XT v);
 template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
 template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
 
-// lg: TT rows of EPT*32 (+1 pad) logits with the bias already added and -inf
-// in padded expert columns.  Rows of tokens >= T are ignored.  Overwrites lg
-// with s.
+// lg: TT rows of EPT*32 (+1 pad) softmax logits (any logit bias already
+// added) and -inf in padded expert columns.  Rows of tokens >= T are ignored.
+// Overwrites lg with s.  sel_bias (or nullptr): a per-expert bias that enters
+// only the top-K keys (auxiliary-loss-free balancing, "Sparse MoE Top-K
+// ルーティング" §解決策3); softmax, gates and the partial sums of s stay on lg.
 template <int EPT, int NW = NTHREADS / 32>       // NW: warps of the calling block
 __device__ __forceinline__ void select_block(float* lg_raw, int t0, int T, int E, int K,
                                              int32_t* __restrict__ topk_idx, float* __restrict__ gates,
-                                             float* __restrict__ logits_out, float* __restrict__ psum) {
+                                             float* __restrict__ logits_out, float* __restrict__ psum,
+                                             const float* __restrict__ sel_bias) {
     constexpr int NP = EPT * 32;
     float (*lg)[NP + 1] = reinterpret_cast<float (*)[NP + 1]>(lg_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -62,6 +65,13 @@ __device__ __forceinline__ void select_block(float* lg_raw, int t0, int T, int E
             for (int b = 0; b < EPT; ++b)
                 if (lane + 32 * b < E) logits_out[static_cast<size_t>(t) * E + lane + 32 * b] = v[b];
         }
+        // selection keys: the logits, plus the selection-only bias if any
+        float kv[EPT];
+#pragma unroll
+        for (int b = 0; b < EPT; ++b) {
+            const int j = lane + 32 * b;
+            kv[b] = (sel_bias != nullptr && j < E) ? v[b] + __ldg(sel_bias + j) : v[b];
+        }
         uint32_t taken = 0;
         float vmax = 0.f, sel_v = 0.f;
         int sel_j = 0;
@@ -72,7 +82,7 @@ __device__ __forceinline__ void select_block(float* lg_raw, int t0, int T, int E
             for (int b = 0; b < EPT; ++b) {
                 const int j = lane + 32 * b;
                 const bool ok = j < E && !((taken >> b) & 1u);
-                if (ok && (v[b] > bv || (v[b] == bv && j < bj))) { bv = v[b]; bj = j; }
+                if (ok && (kv[b] > bv || (kv[b] == bv && j < bj))) { bv = kv[b]; bj = j; }
             }
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) {
@@ -80,9 +90,26 @@ __device__ __forceinline__ void select_block(float* lg_raw, int t0, int T, int E
                 const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
                 if (ov > bv || (ov == bv && oj < bj)) { bv = ov; bj = oj; }
             }
+            if (sel_bias != nullptr) {
+                // the winner's softmax logit (its key includes the bias)
+                float ub = v[0];
+#pragma unroll
+                for (int b = 1; b < EPT; ++b)
+                    if (b == (bj >> 5)) ub = v[b];
+                bv = __shfl_sync(0xffffffffu, ub, bj & 31);
+            }
             if (k == 0) vmax = bv;
             if ((bj & 31) == lane) taken |= 1u << (bj >> 5);
             if (lane == k) { sel_v = bv; sel_j = bj; }
+        }
+        if (sel_bias != nullptr) {                    // the softmax maximum over all experts
+            float m = -INFINITY;
+#pragma unroll
+            for (int b = 0; b < EPT; ++b)
+                if (lane + 32 * b < E) m = fmaxf(m, v[b]);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+            vmax = m;
         }
         float e_sum = 0.f;
 #pragma unroll
@@ -120,7 +147,8 @@ __global__ void __launch_bounds__(NTHREADS)
 router_generic_kernel(const XT* __restrict__ x, const float* __restrict__ W_r,
                       const float* __restrict__ logit_bias, int T, int d, int E, int K,
                       int32_t* __restrict__ topk_idx, float* __restrict__ gates,
-                      float* __restrict__ logits_out, float* __restrict__ psum) {
+                      float* __restrict__ logits_out, float* __restrict__ psum,
+                      const float* __restrict__ sel_bias) {
     constexpr int NP = EPT * 32;
     __shared__ float xs[TT][KC + 1];
     __shared__ float wsh[(NP * (KC + 1) > TT * (NP + 1)) ? NP * (KC + 1) : TT * (NP + 1)];
@@ -175,7 +203,7 @@ router_generic_kernel(const XT* __restrict__ x, const float* __restrict__ W_r,
             lg[warp * 4 + a][j] = v;
         }
     __syncthreads();
-    select_block<EPT>(wsh, t0, T, E, K, topk_idx, gates, logits_out, psum);
+    select_block<EPT>(wsh, t0, T, E, K, topk_idx, gates, logits_out, psum, sel_bias);
 }
 
 // ---------------------------------------------------------------- small N_r
@@ -221,7 +249,8 @@ __global__ void __launch_bounds__(SmallCfg<NE, RT>::WARPS * 32)
 router_small_kernel(const XT* __restrict__ x, const float* __restrict__ W_r,
                     const float* __restrict__ logit_bias, int T, int d, int E, int K,
                     int32_t* __restrict__ topk_idx, float* __restrict__ gates,
-                    float* __restrict__ logits_out, float* __restrict__ psum, int32_t* status) {
+                    float* __restrict__ logits_out, float* __restrict__ psum, int32_t* status,
+                    const float* __restrict__ sel_bias) {
     extern __shared__ float4 wsm4[];                  // (NE, d) fp32, rows >= E zero
     float* wsm = reinterpret_cast<float*>(wsm4);
     __shared__ float lg[TT][32 + 1];
@@ -322,7 +351,7 @@ router_small_kernel(const XT* __restrict__ x, const float* __restrict__ W_r,
         lg[r][e] = (e < E) ? l + (logit_bias ? logit_bias[e] : 0.f) : -INFINITY;
     }
     __syncthreads();
-    select_block<1, SmallCfg<NE, RT>::WARPS>(&lg[0][0], t0, T, E, K, topk_idx, gates, logits_out, psum);
+    select_block<1, SmallCfg<NE, RT>::WARPS>(&lg[0][0], t0, T, E, K, topk_idx, gates, logits_out, psum, sel_bias);
 }
 
 // ---------------------------------------------------------------- from precomputed logits
@@ -331,7 +360,8 @@ template <int EPT>
 __global__ void __launch_bounds__(NTHREADS)
 router_select_kernel(const float* __restrict__ logits, const float* __restrict__ logit_bias, int T, int E, int K,
                      int32_t* __restrict__ topk_idx, float* __restrict__ gates,
-                     float* __restrict__ logits_out, float* __restrict__ psum) {
+                     float* __restrict__ logits_out, float* __restrict__ psum,
+                     const float* __restrict__ sel_bias) {
     constexpr int NP = EPT * 32;
     __shared__ float lg[TT * (NP + 1)];
     const int t0 = blockIdx.x * TT;
@@ -343,7 +373,7 @@ router_select_kernel(const float* __restrict__ logits, const float* __restrict__
         lg[r * (NP + 1) + j] = v;
     }
     __syncthreads();
-    select_block<EPT>(lg, t0, T, E, K, topk_idx, gates, logits_out, psum);
+    select_block<EPT>(lg, t0, T, E, K, topk_idx, gates, logits_out, psum, sel_bias);
 }
 
 // out[i] = sum_{s < ks} part[s * n + i], in split order.
@@ -359,10 +389,11 @@ router_reduce_kernel(const float* __restrict__ part, int ks, size_t n, float* __
 
 template <typename XT>
 cudaError_t launch_generic(const Dims& dm, const void* x, const float* W_r, const float* bias,
-                           int32_t* idx, float* gates, float* logits, float* psum, cudaStream_t st) {
+                           int32_t* idx, float* gates, float* logits, float* psum, const float* sel_bias,
+                           cudaStream_t st) {
     const dim3 grid(dm.route_blocks), block(NTHREADS);
     const XT* xp = static_cast<const XT*>(x);
-#define MOE_GEN(EPT) router_generic_kernel<XT, EPT><<<grid, block, 0, st>>>(xp, W_r, bias, dm.T, dm.d, dm.E, dm.K, idx, gates, logits, psum)
+#define MOE_GEN(EPT) router_generic_kernel<XT, EPT><<<grid, block, 0, st>>>(xp, W_r, bias, dm.T, dm.d, dm.E, dm.K, idx, gates, logits, psum, sel_bias)
     if (dm.E <= 32) MOE_GEN(1);
     else if (dm.E <= 64) MOE_GEN(2);
     else if (dm.E <= 128) MOE_GEN(4);
@@ -375,13 +406,13 @@ cudaError_t launch_generic(const Dims& dm, const void* x, const float* W_r, cons
 template <typename XT, int NE, int RT>
 cudaError_t launch_small_t(const Dims& dm, const void* x, const float* W_r, const float* bias,
                            int32_t* idx, float* gates, float* logits, float* psum, int32_t* status,
-                           cudaStream_t st) {
+                           const float* sel_bias, cudaStream_t st) {
     const size_t smem = static_cast<size_t>(NE) * dm.d * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(router_small_kernel<XT, NE, RT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     router_small_kernel<XT, NE, RT><<<dm.route_blocks, SmallCfg<NE, RT>::WARPS * 32, smem, st>>>(
-        static_cast<const XT*>(x), W_r, bias, dm.T, dm.d, dm.E, dm.K, idx, gates, logits, psum, status);
+        static_cast<const XT*>(x), W_r, bias, dm.T, dm.d, dm.E, dm.K, idx, gates, logits, psum, status, sel_bias);
     count_launches();
     return cudaGetLastError();
 }
@@ -389,10 +420,10 @@ cudaError_t launch_small_t(const Dims& dm, const void* x, const float* W_r, cons
 template <typename XT>
 cudaError_t launch_small(const Dims& dm, const void* x, const float* W_r, const float* bias,
                          int32_t* idx, float* gates, float* logits, float* psum, int32_t* status,
-                         cudaStream_t st) {
-    if (dm.E <= 8) return launch_small_t<XT, 8, 4>(dm, x, W_r, bias, idx, gates, logits, psum, status, st);
-    if (dm.E <= 16) return launch_small_t<XT, 16, 4>(dm, x, W_r, bias, idx, gates, logits, psum, status, st);
-    return launch_small_t<XT, 32, 2>(dm, x, W_r, bias, idx, gates, logits, psum, status, st);
+                         const float* sel_bias, cudaStream_t st) {
+    if (dm.E <= 8) return launch_small_t<XT, 8, 4>(dm, x, W_r, bias, idx, gates, logits, psum, status, sel_bias, st);
+    if (dm.E <= 16) return launch_small_t<XT, 16, 4>(dm, x, W_r, bias, idx, gates, logits, psum, status, sel_bias, st);
+    return launch_small_t<XT, 32, 2>(dm, x, W_r, bias, idx, gates, logits, psum, status, sel_bias, st);
 }
 
 }  // namespace
@@ -409,14 +440,18 @@ bool router_uses_tc(const Dims& dm) {
 cudaError_t launch_router(const Dims& dm, const void* x, const float* W_r, const float* logit_bias,
                           int32_t* topk_idx, float* gates, float* logits_out, float* psum,
                           const RouterScratch& rs, cudaStream_t st) {
+    // bias_mode 0: the bias enters the logits; 1: only the top-K keys
+    const float* sel_bias = dm.bias_mode == 1 ? logit_bias : nullptr;
+    if (dm.bias_mode == 1) logit_bias = nullptr;
     if (router_uses_small(dm)) {
         if (dm.dtype == MOE_F32)
-            return launch_small<float>(dm, x, W_r, logit_bias, topk_idx, gates, logits_out, psum, rs.status, st);
+            return launch_small<float>(dm, x, W_r, logit_bias, topk_idx, gates, logits_out, psum, rs.status,
+                                       sel_bias, st);
         return launch_small<__nv_bfloat16>(dm, x, W_r, logit_bias, topk_idx, gates, logits_out, psum, rs.status,
-                                           st);
+                                           sel_bias, st);
     }
     if (!router_uses_tc(dm))
-        return launch_generic<float>(dm, x, W_r, logit_bias, topk_idx, gates, logits_out, psum, st);
+        return launch_generic<float>(dm, x, W_r, logit_bias, topk_idx, gates, logits_out, psum, sel_bias, st);
     const RouterTcPlan plan = router_tc_plan(dm);
     cudaError_t e = launch_router_tc(dm, plan, x, W_r, rs.w3, rs.part, rs.status, st);
     if (e != cudaSuccess) return e;
@@ -432,7 +467,7 @@ cudaError_t launch_router(const Dims& dm, const void* x, const float* W_r, const
         logits = rs.logits;
     }
     const dim3 grid(dm.route_blocks), block(NTHREADS);
-#define MOE_SEL(EPT) router_select_kernel<EPT><<<grid, block, 0, st>>>(logits, logit_bias, dm.T, dm.E, dm.K, topk_idx, gates, logits_out, psum)
+#define MOE_SEL(EPT) router_select_kernel<EPT><<<grid, block, 0, st>>>(logits, logit_bias, dm.T, dm.E, dm.K, topk_idx, gates, logits_out, psum, sel_bias)
     if (dm.E <= 32) MOE_SEL(1);
     else if (dm.E <= 64) MOE_SEL(2);
     else if (dm.E <= 128) MOE_SEL(4);

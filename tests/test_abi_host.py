@@ -127,6 +127,14 @@ def test_null_pointers_rejected_without_launch():
     assert M.moe_kernel_launches() == launches_before
 
 
+def test_bias_mode_validated():
+    cfg = M.make_config(T=64, d_model=128, n_routed=8, top_k=2, d_ff=256, bias_mode=2)
+    n = ctypes.c_size_t(0)
+    assert M.lib().moe_workspace_size(ctypes.byref(cfg), ctypes.byref(n)) == M.MOE_ERR_INVALID_ARG
+    cfg.bias_mode = M.MOE_BIAS_SELECTION
+    assert M.lib().moe_workspace_size(ctypes.byref(cfg), ctypes.byref(n)) == M.MOE_OK
+
+
 def test_fp8_requires_scales():
     L = M.lib()
     cfg = M.make_config(T=64, d_model=128, n_routed=8, top_k=2, d_ff=128, dtype=2)

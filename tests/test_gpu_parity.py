@@ -33,6 +33,15 @@ CASES = {
     "fp8-ragged-shared": MoEShape("f1", 300, 512, 16, 4, 256, n_shared=1, d_ff_shared=384, dtype=DTYPE_FP8),
     "fp8-decode-skewed": MoEShape("f2", 37, 1024, 256, 8, 256, n_shared=1, d_ff_shared=256,
                                   dtype=DTYPE_FP8, zipf_logit_bias=True),
+    # selection-only bias on each router path: small (N_r <= 32), tensor-core, fp32 generic
+    "bf16-selbias-small-router": MoEShape("s1", 300, 256, 8, 2, 256, dtype=DTYPE_BF16,
+                                          bias_mode=1, selection_bias=True),
+    "bf16-selbias-tc-router": MoEShape("s2", 600, 256, 128, 4, 128, n_shared=1, d_ff_shared=128,
+                                       capacity_factor=1.0, dtype=DTYPE_BF16, bias_mode=1, selection_bias=True),
+    "f32-selbias-generic-router": MoEShape("s3", 100, 128, 40, 3, 128, dtype=DTYPE_F32,
+                                           bias_mode=1, selection_bias=True),
+    "fp8-selbias": MoEShape("s4", 200, 512, 64, 8, 256, n_shared=1, d_ff_shared=128,
+                            dtype=DTYPE_FP8, bias_mode=1, selection_bias=True),
 }
 
 
