@@ -231,21 +231,25 @@ def capacity_of(T: int, K: int, N_r: int, cf: float) -> Optional[int]:
     return int(math.ceil(Fraction(cf32) * T * K / N_r))
 
 
-def dispatch_plan(idx: np.ndarray, N_r: int, C: Optional[int]) -> Dict[str, np.ndarray]:
+def dispatch_plan(idx: np.ndarray, N_r: int, C: Optional[int], priority: str = "token") -> Dict[str, np.ndarray]:
     """Counts, kept counts, segment offsets and the slot<->row permutation.
 
-    Slots (t, k) of expert j are ranked in ascending token order; slot of rank
-    r is kept iff r < C.  Kept slots of expert j occupy rows
-    offsets[j] .. offsets[j] + kept[j] - 1 in token order.
+    Slots (t, k) of expert j are ranked in ascending token order
+    (priority "token", [TopK] FAQ Q2: the earliest tokens are kept), or
+    slot-major (priority "slot": every token's k-th choice before any
+    (k+1)-th choice, each in token order); slot of rank r is kept iff r < C.
+    Kept slots of expert j occupy rows offsets[j] .. offsets[j] + kept[j] - 1
+    in rank order.
     """
     T, K = idx.shape
     counts = np.zeros(N_r, np.int64)
     rank = np.full((T, K), -1, np.int64)
-    for t in range(T):
-        for k in range(K):
-            j = int(idx[t, k])
-            rank[t, k] = counts[j]
-            counts[j] += 1
+    order = ([(t, k) for t in range(T) for k in range(K)] if priority == "token"
+             else [(t, k) for k in range(K) for t in range(T)])
+    for t, k in order:
+        j = int(idx[t, k])
+        rank[t, k] = counts[j]
+        counts[j] += 1
     kept = counts.copy() if C is None else np.minimum(counts, C)
     offsets = np.zeros(N_r + 1, np.int64)
     offsets[1:] = np.cumsum(kept)
@@ -334,7 +338,8 @@ def route(shape, inputs, logits: Optional[np.ndarray] = None):
     idx = topk_select(keys, shape.top_k)
     g = gates_of(s, idx)
     C = capacity_of(shape.T, shape.top_k, shape.n_routed, shape.capacity_factor)
-    plan = dispatch_plan(idx, shape.n_routed, C)
+    plan = dispatch_plan(idx, shape.n_routed, C,
+                         "slot" if getattr(shape, "capacity_priority", 0) == 1 else "token")
     f, P, L = balance_stats(plan["counts"], s, shape.top_k, shape.alpha)
     return {"logits": l64, "s": s, "idx": idx, "gates": g, "C": C, "plan": plan,
             "f": f, "P": P, "loss": L, "gap": topk_gap(keys64, shape.top_k)}
@@ -401,10 +406,15 @@ def layer_forward(shape, inputs, tokens: Optional[np.ndarray] = None,
         for n, key in enumerate(rows):
             y_slot[key] = y[n]
     out = np.zeros((len(tokens), shape.d_model), np.float64)
+    # [TopK] §解決策2: a slot over the capacity is dropped, or (overflow_mode 1)
+    # the token passes that expert unchanged: its own input times its gate
+    passthrough = getattr(shape, "overflow_mode", 0) == 1
     for i, t in enumerate(tokens):
         for k in range(K):
             if (i, k) in y_slot:
                 out[i] += rt["gates"][t, k] * y_slot[(i, k)]
+            elif passthrough:
+                out[i] += rt["gates"][t, k] * x[i]
     for s_i in range(shape.n_shared):
         W1, b1, W2, b2 = expert_weights(inputs, "Ws", s_i, fp8)
         y = expert_ffn(xin, W1, b1, W2, b2, fp8_hidden=fp8)

@@ -51,6 +51,12 @@ class MoEShape:
     # softmax, gates and P on the unbiased logits)
     bias_mode: int = 0
     selection_bias: bool = False   # draw a N(0, 0.5^2) per-expert bias
+    # capacity variants: which slots an expert keeps first (0 = token order,
+    # 1 = slot-major: every token's first choice before any second choice),
+    # and what a slot dropped by the capacity limit contributes (0 = nothing,
+    # 1 = the token's own input times its gate: the token passes through)
+    capacity_priority: int = 0
+    overflow_mode: int = 0
 
     def replace(self, **kw) -> "MoEShape":
         return dataclasses.replace(self, **kw)

@@ -391,3 +391,38 @@ def test_selection_bias_zero_changes_nothing():
     b = _one_token(None, 0)
     assert a["idx"].tolist() == b["idx"].tolist() == [[0, 1]]
     assert np.array_equal(a["gates"], b["gates"]) and np.array_equal(a["P"], b["P"])
+
+
+# ---------------------------------------------------------------------------
+# Capacity variants ([TopK] §解決策2 and FAQ Q2).
+
+
+def test_slot_major_priority_hand_worked():
+    """idx = [[1, 0], [0, 1], [0, 1]], C = 2.  Token order keeps the first two
+    tokens of each expert; slot-major keeps every first choice before any
+    second choice, so expert 0 drops token 0's second choice instead of
+    token 2's first."""
+    idx = np.array([[1, 0], [0, 1], [0, 1]])
+    tok = O.dispatch_plan(idx, 2, 2, "token")
+    slot = O.dispatch_plan(idx, 2, 2, "slot")
+    assert tok["slot_row"].tolist() == [[2, 0], [1, 3], [-1, -1]]
+    assert slot["slot_row"].tolist() == [[2, -1], [0, 3], [1, -1]]
+    assert tok["counts"].tolist() == slot["counts"].tolist() == [3, 3]
+    assert slot["row_slot"].tolist() == [2, 4, 0, 3]
+
+
+def test_overflow_passthrough_with_zero_experts():
+    """All expert weights and biases zero: every kept slot contributes 0, so
+    with pass-through the output is exactly the sum over dropped slots of
+    g * x (here K = 1, g = 1, C = 1: tokens 1 and 2 come out as their input)."""
+    from synthetic import MoEShape
+    x = np.array([[1.0, -2.0], [0.5, 3.0], [-1.5, 0.25]])
+    inp = {"x": x, "W_r": np.array([[1.0, 0.0]]), "logit_bias": None,
+           "W1": np.zeros((1, 64, 2)), "b1": np.zeros((1, 64)), "W2": np.zeros((1, 2, 64)), "b2": np.zeros((1, 2)),
+           "W1_scales": None, "W2_scales": None}
+    cf = 0.25                                   # 0.25 * 3 = 0.75 -> C = 1
+    for mode, expect in ((0, np.zeros_like(x)), (1, np.array([[0.0, 0.0], [0.5, 3.0], [-1.5, 0.25]]))):
+        sh = MoEShape("p", 3, 2, 1, 1, 64, capacity_factor=cf, dtype=0, overflow_mode=mode)
+        assert O.capacity_of(3, 1, 1, cf) == 1
+        out = O.layer_forward(sh, inp)["out"]
+        assert np.array_equal(out, expect), (mode, out)
