@@ -351,7 +351,7 @@ def run_ours(args):
                          g("b1"), g("W2"), g("W2_scales"), g("b2"), g("Ws1"), g("Ws1_scales"), g("bs1"),
                          g("Ws2"), g("Ws2_scales"), g("bs2"), b["y"], ws)
         ev[3].record(stream)
-        M.moe_combine(cfg, b["y"], b["gates"], b["slot_row"], b["out"])
+        M.moe_combine(cfg, b["y"], b["gates"], b["slot_row"], b["out"], x=inp["x"])
         ev[4].record(stream)
         M.moe_balance_stats(cfg, b["counts"], ws, b["f"], b["P"], b["loss"])
         ev[5].record(stream)

@@ -108,7 +108,25 @@ typedef struct {
     float   alpha;           /* balance weight (the pages recommend 0.01)         */
     int32_t dtype;           /* MOE_F32 | MOE_BF16 | MOE_FP8_E4M3_BLOCK           */
     int32_t bias_mode;       /* how logit_bias is used (see MOE_BIAS_*)           */
+    int32_t capacity_priority; /* which slots an expert keeps (MOE_PRIORITY_*)   */
+    int32_t overflow_mode;   /* what a slot over the capacity gives (MOE_OVERFLOW_*) */
 } moe_config;
+
+/* capacity_priority ("Sparse MoE Top-Kルーティング" §解決策2, FAQ Q2).
+ * MOE_PRIORITY_TOKEN: an expert's slots are ranked in token order and the
+ * first C are kept (the earliest tokens).  MOE_PRIORITY_SLOT: every token's
+ * first choice ranks before any second choice (then token order), so a
+ * token's top expert is dropped last.  Rows of an expert's segment follow the
+ * rank order. */
+#define MOE_PRIORITY_TOKEN  0
+#define MOE_PRIORITY_SLOT   1
+
+/* overflow_mode (same section: tokens over the capacity are dropped or passed
+ * through).  MOE_OVERFLOW_DROP: a dropped slot adds nothing.
+ * MOE_OVERFLOW_PASS: a dropped slot adds gate * x[t], the token's own input
+ * (it passes that expert unchanged); moe_combine then needs x. */
+#define MOE_OVERFLOW_DROP   0
+#define MOE_OVERFLOW_PASS   1
 
 /* bias_mode.  MOE_BIAS_LOGITS: the per-expert bias is added to the router
  * logits, so softmax, top-K, gates and P all see it.  MOE_BIAS_SELECTION:
@@ -177,8 +195,10 @@ MOE_EXPORT int moe_route(const moe_config* cfg, const void* x, const float* W_r,
 /* ---- stage 2: dispatch ----------------------------------------------------
  * counts[j] = #slots selecting expert j (pre-drop); kept[j] = min(counts, C);
  * offsets (N_r+1) = exclusive prefix sum of kept; slot_row[t,k] = row of
- * slot (t,k) in x_disp (ascending t within an expert's segment) or -1 if
- * dropped; row_slot[r] = t*K+k for r < offsets[N_r].
+ * slot (t,k) in x_disp (in capacity-rank order within an expert's segment:
+ * ascending t, or slot-major with MOE_PRIORITY_SLOT), -1 if dropped by the
+ * capacity, -2 if its expert index is invalid; row_slot[r] = t*K+k for
+ * r < offsets[N_r].
  * x_disp receives x[t] for every kept slot: as-is in fp32/bf16 mode; in FP8
  * mode as e4m3 codes with x_disp_scales (rows, d_model/128) fp32, plus (with
  * shared experts) the quantised x of every token at rows R_cap..R_cap+T-1.
@@ -212,10 +232,13 @@ MOE_EXPORT int moe_expert_ffn(const moe_config* cfg, const void* x, const void* 
 
 /* ---- stage 4: combine ------------------------------------------------------
  * out[t] = sum_{k ascending, slot_row[t,k] >= 0} gates[t,k] * y[slot_row[t,k]]
+ *          (+ gates[t,k] * x[t] for slot_row[t,k] == -1 with MOE_OVERFLOW_PASS)
  *          + sum_{s ascending} y[R_cap + s*T + t], accumulated in fp32.
+ * x (T, d_model), as given to moe_dispatch: read only with MOE_OVERFLOW_PASS
+ * (may be NULL otherwise).
  * out (T, d_model) fp32 (MOE_F32) or bf16 (round-to-nearest-even). */
 MOE_EXPORT int moe_combine(const moe_config* cfg, const void* y, const float* gates,
-                const int32_t* slot_row, void* out, void* stream);
+                const int32_t* slot_row, const void* x, void* out, void* stream);
 
 /* ---- stage 5: balance statistics ------------------------------------------
  * f[j] = counts[j] / (T*K); P[j] = (1/T) sum_t s[t,j] from the partial sums

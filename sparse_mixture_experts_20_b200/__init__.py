@@ -30,6 +30,8 @@ MOE_DEV_BAD_ROUTING = 0x1
 MOE_DEV_TIMEOUT = 0x2
 MOE_F32, MOE_BF16, MOE_FP8_E4M3_BLOCK = 0, 1, 2
 MOE_BIAS_LOGITS, MOE_BIAS_SELECTION = 0, 1
+MOE_PRIORITY_TOKEN, MOE_PRIORITY_SLOT = 0, 1
+MOE_OVERFLOW_DROP, MOE_OVERFLOW_PASS = 0, 1
 
 EXPORTED = (
     "moe_workspace_size", "moe_buffer_rows", "moe_workspace_init", "moe_get_device_status",
@@ -45,6 +47,7 @@ class moe_config(ctypes.Structure):
         ("top_k", ctypes.c_int32), ("d_ff", ctypes.c_int32), ("n_shared", ctypes.c_int32),
         ("d_ff_shared", ctypes.c_int32), ("capacity_factor", ctypes.c_float),
         ("alpha", ctypes.c_float), ("dtype", ctypes.c_int32), ("bias_mode", ctypes.c_int32),
+        ("capacity_priority", ctypes.c_int32), ("overflow_mode", ctypes.c_int32),
     ]
 
 
@@ -83,7 +86,7 @@ def lib() -> ctypes.CDLL:
             "moe_route": [cfgp, P, P, P, P, P, P, P, P],
             "moe_dispatch": [cfgp, P, P, P, P, P, P, P, P, P, P, P],
             "moe_expert_ffn": [cfgp] + [P] * 19,
-            "moe_combine": [cfgp, P, P, P, P, P],
+            "moe_combine": [cfgp, P, P, P, P, P, P],
             "moe_balance_stats": [cfgp, P, P, P, P, P, P],
             "moe_layer_forward": [cfgp] + [P] * 24,
             "moe_selftest_wait_timeout": [cfgp, ctypes.c_int64, P, P],
@@ -101,8 +104,8 @@ def lib() -> ctypes.CDLL:
 
 def make_config(shape=None, **kw) -> moe_config:
     """moe_config from any object with the fields T, d_model, n_routed, top_k,
-    d_ff, n_shared, d_ff_shared, capacity_factor, alpha, dtype, bias_mode
-    (keyword arguments override)."""
+    d_ff, n_shared, d_ff_shared, capacity_factor, alpha, dtype, bias_mode,
+    capacity_priority, overflow_mode (keyword arguments override)."""
     fields = [f for f, _ in moe_config._fields_]
     vals = {f: getattr(shape, f) for f in fields if shape is not None and hasattr(shape, f)}
     vals.update(kw)
@@ -112,6 +115,8 @@ def make_config(shape=None, **kw) -> moe_config:
     vals.setdefault("alpha", 0.01)
     vals.setdefault("dtype", MOE_BF16)
     vals.setdefault("bias_mode", MOE_BIAS_LOGITS)
+    vals.setdefault("capacity_priority", MOE_PRIORITY_TOKEN)
+    vals.setdefault("overflow_mode", MOE_OVERFLOW_DROP)
     return moe_config(**{f: vals[f] for f in fields})
 
 
@@ -187,9 +192,10 @@ def moe_expert_ffn(cfg, x, x_disp, x_disp_scales, offsets, W1, W1_scales, b1, W2
                                 _p(y), _p(ws), _stream(stream)), "moe_expert_ffn")
 
 
-def moe_combine(cfg, y, gates, slot_row, out, stream=None):
-    _check(lib().moe_combine(ctypes.byref(cfg), _p(y), _p(gates), _p(slot_row), _p(out), _stream(stream)),
-           "moe_combine")
+def moe_combine(cfg, y, gates, slot_row, out, stream=None, x=None):
+    """x (the layer input) is read only with overflow_mode = MOE_OVERFLOW_PASS."""
+    _check(lib().moe_combine(ctypes.byref(cfg), _p(y), _p(gates), _p(slot_row), _p(x), _p(out),
+                             _stream(stream)), "moe_combine")
 
 
 def moe_balance_stats(cfg, counts, ws, f, P, loss, stream=None):

@@ -30,7 +30,7 @@ template <bool F32, int KT>           // KT >= K: register slots for the token's
 __global__ void __launch_bounds__(32 * CB_WARPS, KT <= 8 ? 4 : 2)
 combine_kernel(const void* __restrict__ y_, const float* __restrict__ gates,
                const int32_t* __restrict__ slot_row, int T, int d, int K, int S, int r_cap,
-               void* __restrict__ out_, int wpt) {
+               const void* __restrict__ x_, void* __restrict__ out_, int wpt) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int t = blockIdx.x * (CB_WARPS / wpt) + warp / wpt;
     const int sub = warp % wpt;
@@ -48,17 +48,21 @@ combine_kernel(const void* __restrict__ y_, const float* __restrict__ gates,
     const uint4* y = static_cast<const uint4*>(y_);          // rows of nchunks 16-byte chunks
     uint4* out = static_cast<uint4*>(out_) + static_cast<size_t>(t) * nchunks;
     for (int c = sub * 32 + lane; c < nchunks; c += 32 * wpt) {
+        // a kept slot reads its expert row; with pass-through (x_ != nullptr)
+        // a slot dropped by the capacity (row -1) reads the token's own input
+        const uint4* xr = static_cast<const uint4*>(x_);
         uint4 raw[KT];
 #pragma unroll
         for (int k = 0; k < KT; ++k)
             raw[k] = (k < K && rows[k] >= 0) ? __ldg(y + static_cast<size_t>(rows[k]) * nchunks + c)
-                                             : make_uint4(0, 0, 0, 0);
+                     : (k < K && rows[k] == -1 && xr != nullptr) ? __ldg(xr + static_cast<size_t>(t) * nchunks + c)
+                                                                 : make_uint4(0, 0, 0, 0);
         float acc[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = 0.f;
 #pragma unroll
         for (int k = 0; k < KT; ++k) {
-            if (k >= K || rows[k] < 0) continue;
+            if (k >= K || rows[k] < -1 || (rows[k] == -1 && xr == nullptr)) continue;
             if (F32) {
                 const float* f = reinterpret_cast<const float*>(&raw[k]);
 #pragma unroll
@@ -133,13 +137,14 @@ balance_kernel(const int32_t* __restrict__ counts, const float* __restrict__ psu
 }  // namespace
 
 cudaError_t launch_combine(const Dims& dm, const void* y, const float* gates,
-                           const int32_t* slot_row, void* out, cudaStream_t st) {
+                           const int32_t* slot_row, const void* x, void* out, cudaStream_t st) {
+    if (!dm.passthrough) x = nullptr;
     const bool f32 = dm.dtype == MOE_F32;
     int wpt = 1;                              // enough warps in flight to fill the GPU at small T
     while (wpt < CB_WARPS && static_cast<long long>(dm.T) * wpt < 148LL * 32) wpt *= 2;
     const int blocks = (dm.T + CB_WARPS / wpt - 1) / (CB_WARPS / wpt);
 #define MOE_COMBINE(F, KT) combine_kernel<F, KT><<<blocks, 32 * CB_WARPS, 0, st>>>(          \
-        y, gates, slot_row, dm.T, dm.d, dm.K, dm.S, dm.r_cap, out, wpt)
+        y, gates, slot_row, dm.T, dm.d, dm.K, dm.S, dm.r_cap, x, out, wpt)
 #define MOE_COMBINE_K(F)                                                                         \
     if (dm.K <= 2) MOE_COMBINE(F, 2);                                                            \
     else if (dm.K <= 4) MOE_COMBINE(F, 4);                                                       \

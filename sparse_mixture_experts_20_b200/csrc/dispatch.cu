@@ -39,7 +39,7 @@ __device__ __forceinline__ bool slot_valid(const int* ids, int k, int E) {
 constexpr int MAXK = 16;
 
 __global__ void __launch_bounds__(256)
-bitmap_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int K, int t_words,
+bitmap_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int K, int t_words, int planes,
               uint32_t* __restrict__ bitmap, int32_t* status) {
     const int lane = threadIdx.x & 31;
     const int w = blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -62,17 +62,26 @@ bitmap_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int K, int t_w
         }
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) set_device_status(status, MOE_DEV_BAD_ROUTING);
-    for (int j0 = 0; j0 < E; j0 += 32) {
-        uint32_t mine = 0;
-        for (int jj = 0; jj < 32 && j0 + jj < E; ++jj) {
-            const int j = j0 + jj;
-            bool hit = false;
+    // planes == 1: one bitmap per word (any slot); planes == K: one per slot
+    // index (slot-major capacity priority), plane p holding the p-th choices
+    for (int pl = 0; pl < planes; ++pl) {
+        for (int j0 = 0; j0 < E; j0 += 32) {
+            uint32_t mine = 0;
+            for (int jj = 0; jj < 32 && j0 + jj < E; ++jj) {
+                const int j = j0 + jj;
+                bool hit = false;
+                if (planes == 1) {
 #pragma unroll
-            for (int k = 0; k < MAXK; ++k) hit |= (valid[k] == j);
-            const uint32_t m = __ballot_sync(0xffffffffu, hit);
-            if (lane == jj) mine = m;
+                    for (int k = 0; k < MAXK; ++k) hit |= (valid[k] == j);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < MAXK; ++k) hit |= (k == pl && valid[k] == j);
+                }
+                const uint32_t m = __ballot_sync(0xffffffffu, hit);
+                if (lane == jj) mine = m;
+            }
+            if (j0 + lane < E) bitmap[(static_cast<size_t>(pl) * t_words + w) * E + j0 + lane] = mine;
         }
-        if (j0 + lane < E) bitmap[static_cast<size_t>(w) * E + j0 + lane] = mine;
     }
 }
 
@@ -147,7 +156,7 @@ scatter_kernel(const void* __restrict__ x_, const int32_t* __restrict__ topk_idx
                const int32_t* __restrict__ offsets, int T, int d, int E, int K, int capacity,
                int r_cap, int shared_copy, int32_t* __restrict__ slot_row,
                int32_t* __restrict__ row_slot, void* __restrict__ x_disp_,
-               float* __restrict__ x_disp_scales, int wpt) {
+               float* __restrict__ x_disp_scales, int wpt, int t_words, int slot_major) {
     constexpr int PF = 4;                                  // 16-byte chunks per lane in flight
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
@@ -167,7 +176,7 @@ scatter_kernel(const void* __restrict__ x_, const int32_t* __restrict__ topk_idx
     }
     // ---- slot resolution (lane k: slot k)
     const int my_id = lane < K ? topk_idx[static_cast<size_t>(t) * K + lane] : -1;
-    int row = -1;
+    int row = -2;                                          // -2: invalid index, -1: over the capacity
     {
         bool valid = lane < K && my_id >= 0 && my_id < E;
         for (int q = 0; q < K; ++q) {                      // repeated by an earlier slot?
@@ -175,10 +184,11 @@ scatter_kernel(const void* __restrict__ x_, const int32_t* __restrict__ topk_idx
             if (q < lane && other == my_id) valid = false;
         }
         if (valid) {
-            const int w = t >> 5;
-            const uint32_t below = bitmap[static_cast<size_t>(w) * E + my_id] & ((1u << (t & 31)) - 1u);
-            const int rank = word_base[static_cast<size_t>(w) * E + my_id] + __popc(below);
-            if (capacity < 0 || rank < capacity) row = offsets[my_id] + rank;
+            // bitmap word: (plane, word); plane = the slot index under slot-major priority
+            const size_t qw = static_cast<size_t>(slot_major ? lane : 0) * t_words + (t >> 5);
+            const uint32_t below = bitmap[qw * E + my_id] & ((1u << (t & 31)) - 1u);
+            const int rank = word_base[qw * E + my_id] + __popc(below);
+            row = (capacity < 0 || rank < capacity) ? offsets[my_id] + rank : -1;
         }
         if (lane < K && sub == 0) {
             slot_row[static_cast<size_t>(t) * K + lane] = row;
@@ -269,8 +279,12 @@ cudaError_t launch_dispatch(const Dims& dm, const void* x, const int32_t* topk_i
                             int32_t* slot_row, int32_t* row_slot, void* x_disp,
                             float* x_disp_scales, uint32_t* bitmap, int32_t* word_base,
                             int32_t* status, cudaStream_t st) {
-    bitmap_kernel<<<(dm.t_words + 7) / 8, 256, 0, st>>>(topk_idx, dm.T, dm.E, dm.K, dm.t_words, bitmap, status);
-    scan_kernel<<<1, 1024, 0, st>>>(bitmap, dm.E, dm.t_words, dm.capacity, word_base, counts, kept, offsets);
+    bitmap_kernel<<<(dm.t_words + 7) / 8, 256, 0, st>>>(topk_idx, dm.T, dm.E, dm.K, dm.t_words, dm.planes,
+                                                        bitmap, status);
+    // the scan runs over the (plane, word) sequence: token order within a
+    // plane, planes in slot order
+    scan_kernel<<<1, 1024, 0, st>>>(bitmap, dm.E, dm.planes * dm.t_words, dm.capacity, word_base, counts, kept,
+                                    offsets);
     const int shared_copy = (dm.dtype == MOE_FP8_E4M3_BLOCK && dm.S > 0) ? 1 : 0;
     // warps per token: enough warps in flight to fill the GPU at small T
     int wpt = 1;
@@ -279,7 +293,7 @@ cudaError_t launch_dispatch(const Dims& dm, const void* x, const int32_t* topk_i
     const int blocks = (dm.T + tpb - 1) / tpb;
 #define MOE_SCATTER(MODE) scatter_kernel<MODE><<<blocks, 32 * SC_WARPS, 0, st>>>(          \
         x, topk_idx, bitmap, word_base, offsets, dm.T, dm.d, dm.E, dm.K, dm.capacity,      \
-        dm.r_cap, shared_copy, slot_row, row_slot, x_disp, x_disp_scales, wpt)
+        dm.r_cap, shared_copy, slot_row, row_slot, x_disp, x_disp_scales, wpt, dm.t_words, dm.slot_major)
     if (dm.dtype == MOE_F32) MOE_SCATTER(0);
     else if (dm.dtype == MOE_BF16) MOE_SCATTER(1);
     else MOE_SCATTER(2);

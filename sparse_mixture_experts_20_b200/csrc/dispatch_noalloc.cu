@@ -56,8 +56,8 @@ extern "C" int moe_dispatch_noalloc(const moe_config* cfg, const void* x, const 
     if ((reinterpret_cast<uintptr_t>(x) & 15u) || (reinterpret_cast<uintptr_t>(x_disp) & 15u))
         return MOE_ERR_INVALID_ARG;
     if (dm.dtype == MOE_FP8_E4M3_BLOCK && !x_disp_scales) return MOE_ERR_INVALID_ARG;
-    // bitmap and word bases, each (T/32, N_r) 32-bit words, 256-byte aligned
-    const size_t part = (static_cast<size_t>(dm.t_words) * dm.E * 4 + 255) & ~static_cast<size_t>(255);
+    // bitmap and word bases, each (planes, T/32, N_r) 32-bit words, 256-byte aligned
+    const size_t part = (static_cast<size_t>(dm.planes) * dm.t_words * dm.E * 4 + 255) & ~static_cast<size_t>(255);
     if (2 * part > kNoAllocScratchBytes) return MOE_ERR_UNSUPPORTED;
     void* base = nullptr;
     cudaError_t e = scratch_on_current_device(&base);

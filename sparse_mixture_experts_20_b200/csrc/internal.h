@@ -39,9 +39,12 @@ struct Dims {
     int y_rows;
     int dtype;
     int bias_mode;  // 0: logit_bias enters the logits; 1: only the top-K keys
+    int slot_major; // capacity ranks: 0 token order, 1 slot-major
+    int passthrough;// a slot over the capacity adds gate * x
     float alpha;
     int route_blocks;
     int t_words;
+    int planes;     // token bitmaps per word: 1, or K (one per slot) when slot_major
 };
 
 constexpr int kRouteTokens = 32;    // tokens per router block
@@ -84,7 +87,7 @@ cudaError_t launch_dispatch(const Dims& dm, const void* x, const int32_t* topk_i
                             int32_t* status, cudaStream_t st);
 
 cudaError_t launch_combine(const Dims& dm, const void* y, const float* gates,
-                           const int32_t* slot_row, void* out, cudaStream_t st);
+                           const int32_t* slot_row, const void* x, void* out, cudaStream_t st);
 
 cudaError_t launch_balance(const Dims& dm, const int32_t* counts, const float* psum,
                            float* f, float* P, float* loss, cudaStream_t st);

@@ -59,6 +59,8 @@ int validate(const moe_config* cfg, Dims* dm) {
         return MOE_ERR_INVALID_ARG;
     if (c.dtype != MOE_F32 && c.dtype != MOE_BF16 && c.dtype != MOE_FP8_E4M3_BLOCK) return MOE_ERR_INVALID_ARG;
     if (c.bias_mode != MOE_BIAS_LOGITS && c.bias_mode != MOE_BIAS_SELECTION) return MOE_ERR_INVALID_ARG;
+    if (c.capacity_priority != MOE_PRIORITY_TOKEN && c.capacity_priority != MOE_PRIORITY_SLOT) return MOE_ERR_INVALID_ARG;
+    if (c.overflow_mode != MOE_OVERFLOW_DROP && c.overflow_mode != MOE_OVERFLOW_PASS) return MOE_ERR_INVALID_ARG;
     if (c.n_routed > 256 || c.top_k > 16 || c.n_shared > 8) return MOE_ERR_UNSUPPORTED;
     const int q = c.dtype == MOE_FP8_E4M3_BLOCK ? 128 : 64;
     if (c.d_model % q || c.d_ff % q || (c.n_shared > 0 && c.d_ff_shared % q)) return MOE_ERR_UNSUPPORTED;
@@ -74,6 +76,8 @@ int validate(const moe_config* cfg, Dims* dm) {
     dm->dffs = c.n_shared > 0 ? c.d_ff_shared : 0;
     dm->dtype = c.dtype;
     dm->bias_mode = c.bias_mode;
+    dm->slot_major = c.capacity_priority == MOE_PRIORITY_SLOT ? 1 : 0;
+    dm->passthrough = c.overflow_mode == MOE_OVERFLOW_PASS ? 1 : 0;
     dm->alpha = c.alpha;
     dm->capacity = capacity_of(c.capacity_factor, c.T, c.top_k, c.n_routed);
     long long rcap = static_cast<long long>(c.T) * c.top_k;
@@ -86,6 +90,7 @@ int validate(const moe_config* cfg, Dims* dm) {
     dm->y_rows = dm->r_cap + c.n_shared * c.T;
     dm->route_blocks = (c.T + kRouteTokens - 1) / kRouteTokens;
     dm->t_words = (c.T + 31) / 32;
+    dm->planes = dm->slot_major ? c.top_k : 1;
     return MOE_OK;
 }
 
@@ -97,8 +102,8 @@ WsLayout ws_layout(const Dims& dm) {
     const size_t hb = dm.dtype == MOE_F32 ? 4 : (dm.dtype == MOE_BF16 ? 2 : 1);
     L.status = take(256);
     L.psum = take(static_cast<size_t>(dm.route_blocks) * dm.E * 4);
-    L.bitmap = take(static_cast<size_t>(dm.t_words) * dm.E * 4);
-    L.word_base = take(static_cast<size_t>(dm.t_words) * dm.E * 4);
+    L.bitmap = take(static_cast<size_t>(dm.planes) * dm.t_words * dm.E * 4);
+    L.word_base = take(static_cast<size_t>(dm.planes) * dm.t_words * dm.E * 4);
     L.h_r = take(static_cast<size_t>(dm.r_cap) * dm.dff * hb);
     L.h_r_scales = take(fp8 ? static_cast<size_t>(dm.r_cap) * (dm.dff / 128) * 4 : 0);
     L.h_s = take(static_cast<size_t>(dm.S) * dm.T * dm.dffs * hb);
@@ -374,12 +379,13 @@ int moe_expert_ffn(const moe_config* cfg, const void* x, const void* x_disp, con
 }
 
 int moe_combine(const moe_config* cfg, const void* y, const float* gates, const int32_t* slot_row,
-                void* out, void* stream) {
+                const void* x, void* out, void* stream) {
     Dims dm;
     const int v = validate(cfg, &dm);
     if (v != MOE_OK) return v;
     if (!y || !gates || !slot_row || !out || !aligned16(y) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
-    return cuda_status(launch_combine(dm, y, gates, slot_row, out, static_cast<cudaStream_t>(stream)));
+    if (dm.passthrough && (!x || !aligned16(x))) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_combine(dm, y, gates, slot_row, x, out, static_cast<cudaStream_t>(stream)));
 }
 
 int moe_balance_stats(const moe_config* cfg, const int32_t* counts, const void* ws, float* f, float* P,
@@ -430,7 +436,7 @@ int moe_layer_forward(const moe_config* cfg, const void* x, const float* W_r, co
     const int r = run_expert_ffn(dm, L, x, x_disp, x_disp_sc, offsets, W1, W1_scales, b1, W2, W2_scales, b2,
                                  Ws1, Ws1_scales, bs1, Ws2, Ws2_scales, bs2, y, ws, st);
     if (r != MOE_OK) return r;
-    e = launch_combine(dm, y, g, slot_row, out, st);
+    e = launch_combine(dm, y, g, slot_row, x, out, st);
     if (e != cudaSuccess) return cuda_status(e);
     return cuda_status(launch_balance(dm, cnt, at<float>(ws, L.psum), f, P, loss, st));
 }

@@ -65,7 +65,7 @@ def run_stages(shape, inp, logits=True):
                      inp["Ws1"], inp["Ws1_scales"], inp["bs1"], inp["Ws2"], inp["Ws2_scales"], inp["bs2"],
                      o["y"], ws)
     o["out"] = torch.empty((T, d), dtype=act_dtype(shape), device=dev)
-    M.moe_combine(cfg, o["y"], o["gates"], o["slot_row"], o["out"])
+    M.moe_combine(cfg, o["y"], o["gates"], o["slot_row"], o["out"], x=inp["x"])
     o["f"] = torch.empty(E, **f32)
     o["P"] = torch.empty(E, **f32)
     o["loss"] = torch.empty(1, **f32)
@@ -183,9 +183,10 @@ def check_expert_ffn(shape, inp, o, rt_prod, rows=None, tokens=None):
         assert rel_frob(got, ref) < tol, (s, rel_frob(got, ref))
 
 
-def check_combine(shape, o, rt_prod):
-    """out[t] = sum_k g y[slot_row] + sum_s y_shared, from the product's own y,
-    gates and slot_row (only rounding of the output may differ)."""
+def check_combine(shape, o, rt_prod, x=None):
+    """out[t] = sum_k g y[slot_row] (+ g x[t] for slots over the capacity with
+    pass-through) + sum_s y_shared, from the product's own y, gates and
+    slot_row (only rounding of the output may differ)."""
     y = cpu(o["y"]).double().numpy()
     g = cpu(o["gates"]).double().numpy()
     sr = cpu(o["slot_row"]).numpy()
@@ -194,6 +195,9 @@ def check_combine(shape, o, rt_prod):
     for k in range(K):
         ok = sr[:, k] >= 0
         ref[ok] += g[ok, k:k + 1] * y[sr[ok, k]]
+        if getattr(shape, "overflow_mode", 0) == 1:
+            dropped = sr[:, k] == -1
+            ref[dropped] += g[dropped, k:k + 1] * O.to_f64(cpu(x))[dropped]
     rc = o["r_cap"]
     for s in range(shape.n_shared):
         ref += y[rc + s * T: rc + (s + 1) * T]
@@ -211,7 +215,8 @@ def check_end_to_end(shape, inp, out, idx_prod, tokens=None, routing=None):
     tokens = np.arange(T) if tokens is None else np.asarray(tokens)
     ok = rt["gap"][tokens] >= NEAR_TIE
     if shape.capacity_factor > 0:
-        prod_plan = O.dispatch_plan(np.asarray(idx_prod), shape.n_routed, rt["C"])
+        prod_plan = O.dispatch_plan(np.asarray(idx_prod), shape.n_routed, rt["C"],
+                                    "slot" if getattr(shape, "capacity_priority", 0) == 1 else "token")
         same = np.all((prod_plan["slot_row"][tokens] >= 0) == (rt["plan"]["slot_row"][tokens] >= 0), axis=1)
         same &= np.all(np.sort(np.asarray(idx_prod)[tokens], 1) == np.sort(rt["idx"][tokens], 1), axis=1)
         ok &= same

@@ -117,7 +117,7 @@ def test_null_pointers_rejected_without_launch():
     assert L.moe_route(c, None, None, None, None, None, None, None, None) == M.MOE_ERR_INVALID_ARG
     assert L.moe_dispatch(c, *([None] * 11)) == M.MOE_ERR_INVALID_ARG
     assert L.moe_expert_ffn(c, *([None] * 19)) == M.MOE_ERR_INVALID_ARG
-    assert L.moe_combine(c, None, None, None, None, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_combine(c, None, None, None, None, None, None) == M.MOE_ERR_INVALID_ARG
     assert L.moe_balance_stats(c, None, None, None, None, None, None) == M.MOE_ERR_INVALID_ARG
     assert L.moe_layer_forward(c, *([None] * 24)) == M.MOE_ERR_INVALID_ARG
     # misaligned workspace / inputs (fake, never dereferenced)

@@ -42,6 +42,17 @@ CASES = {
                                            bias_mode=1, selection_bias=True),
     "fp8-selbias": MoEShape("s4", 200, 512, 64, 8, 256, n_shared=1, d_ff_shared=128,
                             dtype=DTYPE_FP8, bias_mode=1, selection_bias=True),
+    # capacity variants: slot-major priority, overflow pass-through, both
+    "bf16-slotmajor-cap": MoEShape("c1", 300, 256, 8, 2, 256, capacity_factor=0.8, dtype=DTYPE_BF16,
+                                   capacity_priority=1),
+    "bf16-passthrough-cap": MoEShape("c2", 300, 256, 8, 2, 256, capacity_factor=0.8, dtype=DTYPE_BF16,
+                                     overflow_mode=1),
+    "f32-slotmajor-passthrough": MoEShape("c3", 203, 128, 6, 2, 192, n_shared=1, d_ff_shared=128,
+                                          capacity_factor=0.75, dtype=DTYPE_F32, capacity_priority=1,
+                                          overflow_mode=1),
+    "fp8-slotmajor-passthrough": MoEShape("c4", 300, 512, 16, 4, 256, n_shared=1, d_ff_shared=128,
+                                          capacity_factor=0.75, dtype=DTYPE_FP8, capacity_priority=1,
+                                          overflow_mode=1),
 }
 
 
@@ -62,7 +73,7 @@ def test_stage_and_layer_parity(name):
     rt_prod = TL.check_routing(sh, inp, o)
     TL.check_dispatch(sh, inp, o, rt_prod)
     TL.check_expert_ffn(sh, inp, o, rt_prod)
-    TL.check_combine(sh, o, rt_prod)
+    TL.check_combine(sh, o, rt_prod, x=inp["x"])
     n1 = M.moe_kernel_launches()
     lay = TL.run_layer(sh, inp)
     n_layer = M.moe_kernel_launches() - n1
@@ -93,7 +104,7 @@ def test_all_tokens_to_one_expert_with_capacity():
     assert rt["plan"]["counts"][5] == 0
     TL.check_dispatch(sh, inp, o, rt)
     TL.check_expert_ffn(sh, inp, o, rt)
-    TL.check_combine(sh, o, rt)
+    TL.check_combine(sh, o, rt, x=inp["x"])
     err, _ = TL.check_end_to_end(sh, inp, o["out"], TL.cpu(o["topk_idx"]).numpy())
     assert err < TL.TOL_REL_FROB[sh.dtype]
 
@@ -120,7 +131,7 @@ def test_bad_routing_is_flagged_and_dropped():
     status = M.moe_get_device_status(cfg, ws, clear=True)
     assert status & M.MOE_DEV_BAD_ROUTING
     sr = slot_row.cpu().numpy()
-    assert sr[5, 1] == -1 and sr[9, 1] == -1
+    assert sr[5, 1] == -2 and sr[9, 1] == -2        # invalid index (-1 means over the capacity)
     assert int(counts.sum()) == T * K - 2
     assert M.moe_get_device_status(cfg, ws) == 0
 
