@@ -42,6 +42,10 @@ CASES = {
                                            bias_mode=1, selection_bias=True),
     "fp8-selbias": MoEShape("s4", 200, 512, 64, 8, 256, n_shared=1, d_ff_shared=128,
                             dtype=DTYPE_FP8, bias_mode=1, selection_bias=True),
+    # limits of the interface: top-16 of 256 experts, 8 shared experts, one FP8 token
+    "bf16-k16-e256": MoEShape("m1", 200, 256, 256, 16, 128, dtype=DTYPE_BF16),
+    "bf16-8-shared": MoEShape("m2", 96, 128, 8, 2, 128, n_shared=8, d_ff_shared=64, dtype=DTYPE_BF16),
+    "fp8-one-token": MoEShape("m3", 1, 256, 16, 4, 256, n_shared=1, d_ff_shared=128, dtype=DTYPE_FP8),
     # capacity variants: slot-major priority, overflow pass-through, both
     "bf16-slotmajor-cap": MoEShape("c1", 300, 256, 8, 2, 256, capacity_factor=0.8, dtype=DTYPE_BF16,
                                    capacity_priority=1),
