@@ -30,10 +30,23 @@ namespace {
 constexpr int TT = kRouteTokens;   // tokens per block
 constexpr int KC = 32;             // columns per shared-memory chunk (generic kernel)
 constexpr int NTHREADS = 256;
+constexpr int kSelectSplits = 4;  // K splits the select kernel sums itself
 
 template <typename XT> __device__ __forceinline__ float to_f(XT v);
 template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
 template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// Order-preserving map of a float to an unsigned key: a > b as floats iff
+// key(a) > key(b), with -0 folded onto +0 so that the two compare equal; every
+// non-NaN value maps above 0, which stays free to mean "not selectable".
+__device__ __forceinline__ uint32_t order_key(float f) {
+    uint32_t u = __float_as_uint(f);
+    if (u == 0x80000000u) u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float order_key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
 
 // lg: TT rows of EPT*32 (+1 pad) softmax logits (any logit bias already
 // added) and -inf in padded expert columns.  Rows of tokens >= T are ignored.
@@ -65,31 +78,29 @@ __device__ __forceinline__ void select_block(float* lg_raw, int t0, int T, int E
             for (int b = 0; b < EPT; ++b)
                 if (lane + 32 * b < E) logits_out[static_cast<size_t>(t) * E + lane + 32 * b] = v[b];
         }
-        // selection keys: the logits, plus the selection-only bias if any
-        float kv[EPT];
+        // selection keys: the logits, plus the selection-only bias if any,
+        // mapped to unsigned integers in the same order (0 = not selectable)
+        uint32_t key[EPT];
 #pragma unroll
         for (int b = 0; b < EPT; ++b) {
             const int j = lane + 32 * b;
-            kv[b] = (sel_bias != nullptr && j < E) ? v[b] + __ldg(sel_bias + j) : v[b];
+            const float kv = (sel_bias != nullptr && j < E) ? v[b] + __ldg(sel_bias + j) : v[b];
+            key[b] = j < E ? order_key(kv) : 0u;
         }
         uint32_t taken = 0;
         float vmax = 0.f, sel_v = 0.f;
         int sel_j = 0;
         for (int k = 0; k < K; ++k) {
-            float bv = -INFINITY;
+            // this lane's largest free key, the lowest index among equals
+            uint32_t bk = 0u;
             int bj = 0x7fffffff;
 #pragma unroll
-            for (int b = 0; b < EPT; ++b) {
-                const int j = lane + 32 * b;
-                const bool ok = j < E && !((taken >> b) & 1u);
-                if (ok && (kv[b] > bv || (kv[b] == bv && j < bj))) { bv = kv[b]; bj = j; }
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                const int oj = __shfl_xor_sync(0xffffffffu, bj, off);
-                if (ov > bv || (ov == bv && oj < bj)) { bv = ov; bj = oj; }
-            }
+            for (int b = 0; b < EPT; ++b)
+                if (!((taken >> b) & 1u) && key[b] > bk) { bk = key[b]; bj = lane + 32 * b; }
+            // the warp's largest key, then the lowest index holding it
+            const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
+            bj = __reduce_min_sync(0xffffffffu, bk == wk ? bj : 0x7fffffff);
+            float bv = order_key_value(wk);
             if (sel_bias != nullptr) {
                 // the winner's softmax logit (its key includes the bias)
                 float ub = v[0];
@@ -103,13 +114,11 @@ __device__ __forceinline__ void select_block(float* lg_raw, int t0, int T, int E
             if (lane == k) { sel_v = bv; sel_j = bj; }
         }
         if (sel_bias != nullptr) {                    // the softmax maximum over all experts
-            float m = -INFINITY;
+            uint32_t m = 0u;
 #pragma unroll
             for (int b = 0; b < EPT; ++b)
-                if (lane + 32 * b < E) m = fmaxf(m, v[b]);
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-            vmax = m;
+                if (lane + 32 * b < E) m = max(m, order_key(v[b]));
+            vmax = order_key_value(__reduce_max_sync(0xffffffffu, m));
         }
         float e_sum = 0.f;
 #pragma unroll
@@ -356,34 +365,83 @@ router_small_kernel(const XT* __restrict__ x, const float* __restrict__ W_r,
 
 // ---------------------------------------------------------------- from precomputed logits
 
+// One warp per token (32 warps: the block's 32 tokens at once).  The logits
+// are the sum of the ks partial planes part[s][t][j] in split order; the
+// loads of one split are all issued before any of them is used.
+constexpr int SEL_THREADS = 1024;
+static_assert(TT == SEL_THREADS / 32, "one warp per token");
+
 template <int EPT>
-__global__ void __launch_bounds__(NTHREADS)
-router_select_kernel(const float* __restrict__ logits, const float* __restrict__ logit_bias, int T, int E, int K,
-                     int32_t* __restrict__ topk_idx, float* __restrict__ gates,
+__global__ void __launch_bounds__(SEL_THREADS)
+router_select_kernel(const float* __restrict__ part, int ks, const float* __restrict__ logit_bias,
+                     int T, int E, int K, int32_t* __restrict__ topk_idx, float* __restrict__ gates,
                      float* __restrict__ logits_out, float* __restrict__ psum,
                      const float* __restrict__ sel_bias) {
     constexpr int NP = EPT * 32;
+    constexpr int PER = TT * NP / SEL_THREADS;
     __shared__ float lg[TT * (NP + 1)];
     const int t0 = blockIdx.x * TT;
-    for (int i = threadIdx.x; i < TT * NP; i += NTHREADS) {
+    const size_t plane = static_cast<size_t>(T) * E;
+    float acc[PER];
+    bool ok[PER];
+    const float* src[PER];
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+        const int i = threadIdx.x + q * SEL_THREADS;
         const int r = i / NP, j = i % NP;
         const int t = t0 + r;
-        float v = -INFINITY;
-        if (j < E && t < T) v = logits[static_cast<size_t>(t) * E + j] + (logit_bias ? logit_bias[j] : 0.f);
-        lg[r * (NP + 1) + j] = v;
+        ok[q] = j < E && t < T;
+        src[q] = part + (ok[q] ? static_cast<size_t>(t) * E + j : 0);
+        acc[q] = ok[q] ? __ldg(src[q]) : 0.f;
+    }
+    for (int sp = 1; sp < ks; ++sp) {
+        float nx[PER];
+#pragma unroll
+        for (int q = 0; q < PER; ++q) nx[q] = ok[q] ? __ldg(src[q] + sp * plane) : 0.f;
+#pragma unroll
+        for (int q = 0; q < PER; ++q) acc[q] += nx[q];
+    }
+#pragma unroll
+    for (int q = 0; q < PER; ++q) {
+        const int i = threadIdx.x + q * SEL_THREADS;
+        const int r = i / NP, j = i % NP;
+        lg[r * (NP + 1) + j] = ok[q] ? acc[q] + (logit_bias ? __ldg(logit_bias + j) : 0.f) : -INFINITY;
     }
     __syncthreads();
-    select_block<EPT>(lg, t0, T, E, K, topk_idx, gates, logits_out, psum, sel_bias);
+    select_block<EPT, SEL_THREADS / 32>(lg, t0, T, E, K, topk_idx, gates, logits_out, psum, sel_bias);
 }
 
-// out[i] = sum_{s < ks} part[s * n + i], in split order.
-__global__ void __launch_bounds__(256)
+// out[i] = sum_{s < ks} part[s * n + i], in split order; four elements per
+// thread when n allows, with the loads of four splits in flight at once.
+__global__ void __launch_bounds__(128)
 router_reduce_kernel(const float* __restrict__ part, int ks, size_t n, float* __restrict__ out) {
     const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
-    for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride) {
-        float s = part[i];
-        for (int k = 1; k < ks; ++k) s += __ldg(part + static_cast<size_t>(k) * n + i);
-        out[i] = s;
+    const size_t i0 = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if ((n & 3) == 0) {
+        const size_t n4 = n >> 2;
+        const float4* p4 = reinterpret_cast<const float4*>(part);
+        for (size_t i = i0; i < n4; i += stride) {
+            float4 s = __ldg(p4 + i);
+            int k = 1;
+            for (; k + 4 <= ks; k += 4) {
+                float4 v[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) v[u] = __ldg(p4 + static_cast<size_t>(k + u) * n4 + i);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) { s.x += v[u].x; s.y += v[u].y; s.z += v[u].z; s.w += v[u].w; }
+            }
+            for (; k < ks; ++k) {
+                const float4 v = __ldg(p4 + static_cast<size_t>(k) * n4 + i);
+                s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+            }
+            reinterpret_cast<float4*>(out)[i] = s;
+        }
+    } else {
+        for (size_t i = i0; i < n; i += stride) {
+            float s = part[i];
+            for (int k = 1; k < ks; ++k) s += __ldg(part + static_cast<size_t>(k) * n + i);
+            out[i] = s;
+        }
     }
 }
 
@@ -455,19 +513,24 @@ cudaError_t launch_router(const Dims& dm, const void* x, const float* W_r, const
     const RouterTcPlan plan = router_tc_plan(dm);
     cudaError_t e = launch_router_tc(dm, plan, x, W_r, rs.w3, rs.part, rs.status, st);
     if (e != cudaSuccess) return e;
+    // a few splits are summed by the select kernel as it loads them; many
+    // are first reduced by a kernel spread over the whole GPU
     const float* logits = rs.part;
-    if (plan.ksplit > 1) {
+    int ks = plan.ksplit;
+    if (ks > kSelectSplits) {
         const size_t n = static_cast<size_t>(dm.T) * dm.E;
-        int blocks = static_cast<int>((n + 255) / 256);
-        if (blocks > 4 * 148) blocks = 4 * 148;
-        router_reduce_kernel<<<blocks, 256, 0, st>>>(rs.part, plan.ksplit, n, rs.logits);
+        const size_t items = (n & 3) == 0 ? n / 4 : n;
+        int blocks = static_cast<int>((items + 127) / 128);
+        if (blocks > 8 * 148) blocks = 8 * 148;
+        router_reduce_kernel<<<blocks, 128, 0, st>>>(rs.part, ks, n, rs.logits);
         count_launches();
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         logits = rs.logits;
+        ks = 1;
     }
-    const dim3 grid(dm.route_blocks), block(NTHREADS);
-#define MOE_SEL(EPT) router_select_kernel<EPT><<<grid, block, 0, st>>>(logits, logit_bias, dm.T, dm.E, dm.K, topk_idx, gates, logits_out, psum, sel_bias)
+    const dim3 grid(dm.route_blocks), block(SEL_THREADS);
+#define MOE_SEL(EPT) router_select_kernel<EPT><<<grid, block, 0, st>>>(logits, ks, logit_bias, dm.T, dm.E, dm.K, topk_idx, gates, logits_out, psum, sel_bias)
     if (dm.E <= 32) MOE_SEL(1);
     else if (dm.E <= 64) MOE_SEL(2);
     else if (dm.E <= 128) MOE_SEL(4);

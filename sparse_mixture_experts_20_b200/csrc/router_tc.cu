@@ -9,10 +9,12 @@
 //
 // router_split_kernel writes the planes side by side, W3 = [hi | mid | lo]
 // (E rows of 3 d).  router_tc_kernel is a single-tile tcgen05 GEMM per CTA:
-// grid (m-tiles of 128 tokens, n-tiles of BN experts, K splits), TMA into a
-// ring of 128-byte-swizzled stages, one thread issuing tcgen05.mma into
-// tensor memory, four epilogue warps writing fp32 partial logits
-// part[split][t][e].  The splits are summed in a fixed order afterwards.
+// grid (m-tiles of 128 tokens, n-tiles of BN experts, K splits over the
+// 64-column blocks of d), TMA into a ring of 128-byte-swizzled stages that
+// each hold one x block and the three plane blocks it multiplies (x is read
+// once, not once per plane), one thread issuing tcgen05.mma into tensor
+// memory, four epilogue warps writing fp32 partial logits part[split][t][e].
+// The splits are summed in a fixed order afterwards.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cstring>
@@ -30,18 +32,20 @@ constexpr uint64_t kRouterDrainNs = 200000000ull;
 struct __align__(64) RouterTcParams {
     CUtensorMap a_map;   // x (T, d) bf16
     CUtensorMap b_map;   // W3 (E, 3 d) bf16
-    int T, E, d_blocks, kb_total, ksplit;
+    int T, E, d, d_blocks, ksplit;
     float* part;         // (ksplit, T, E)
     int32_t* status;
     uint64_t timeout_ns;
 };
 
+// A stage: one 64-column block of x (RBM rows) and the same block of each of
+// the three planes (BN rows each), 128 bytes per row.
 template <int BN> struct RCfg {
-    static constexpr int STAGES = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+    static constexpr int STAGES = BN == 256 ? 2 : (BN == 128 ? 3 : (BN == 64 ? 5 : 7));
     static constexpr int A_BYTES = RBM * 128;
-    static constexpr int B_BYTES = BN * 128;
+    static constexpr int B_BYTES = BN * 128;                // one plane
     static constexpr int OFF_B = STAGES * A_BYTES;
-    static constexpr int OFF_BAR = OFF_B + STAGES * B_BYTES;
+    static constexpr int OFF_BAR = OFF_B + STAGES * 3 * B_BYTES;
     static constexpr int N_BARS = 2 * STAGES + 2;          // full, empty, accf, drain
     static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
     static constexpr int TOTAL = OFF_MISC + 16;
@@ -49,22 +53,31 @@ template <int BN> struct RCfg {
     static constexpr uint32_t TMEM_COLS = BN;               // 32..256, a power of two
 };
 
+// Row blockIdx.y of W_r, four columns per thread (d is a multiple of 64 and
+// W_r 16-byte aligned): one 16-byte load, one 8-byte store per plane.
 __global__ void __launch_bounds__(256)
-router_split_kernel(const float* __restrict__ W_r, int E, int d, __nv_bfloat16* __restrict__ w3) {
-    const size_t n = static_cast<size_t>(E) * d;
-    for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-        const size_t j = i / d, k = i % d;
-        const float w = W_r[i];
-        const __nv_bfloat16 hi = __float2bfloat16_rn(w);
-        const float r1 = w - __bfloat162float(hi);
-        const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-        const float r2 = r1 - __bfloat162float(mid);
-        const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
-        __nv_bfloat16* row = w3 + j * 3 * d;
-        row[k] = hi;
-        row[d + k] = mid;
-        row[2 * d + k] = lo;
+router_split_kernel(const float* __restrict__ W_r, int d, __nv_bfloat16* __restrict__ w3) {
+    const int j = blockIdx.y;
+    const float4* src = reinterpret_cast<const float4*>(W_r + static_cast<size_t>(j) * d);
+    __nv_bfloat16* row = w3 + static_cast<size_t>(j) * 3 * d;
+    for (int c = blockIdx.x * blockDim.x + threadIdx.x; c < d / 4; c += gridDim.x * blockDim.x) {
+        const float4 w4 = __ldg(src + c);
+        const float w[4] = {w4.x, w4.y, w4.z, w4.w};
+        __nv_bfloat16 pl[3][4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const __nv_bfloat16 hi = __float2bfloat16_rn(w[q]);
+            const float r1 = w[q] - __bfloat162float(hi);
+            const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+            const float r2 = r1 - __bfloat162float(mid);
+            pl[0][q] = hi;
+            pl[1][q] = mid;
+            pl[2][q] = __float2bfloat16_rn(r2);
+        }
+#pragma unroll
+        for (int p = 0; p < 3; ++p)
+            *reinterpret_cast<uint2*>(row + static_cast<size_t>(p) * d + 4 * c) =
+                *reinterpret_cast<const uint2*>(pl[p]);
     }
 }
 
@@ -93,8 +106,8 @@ router_tc_kernel(const __grid_constant__ RouterTcParams p) {
     const int m0 = blockIdx.x * RBM;
     const int n0 = blockIdx.y * BN;
     const int ks = blockIdx.z;
-    const int kb_lo = static_cast<int>(static_cast<long long>(ks) * p.kb_total / p.ksplit);
-    const int kb_hi = static_cast<int>(static_cast<long long>(ks + 1) * p.kb_total / p.ksplit);
+    const int kb_lo = static_cast<int>(static_cast<long long>(ks) * p.d_blocks / p.ksplit);
+    const int kb_hi = static_cast<int>(static_cast<long long>(ks + 1) * p.d_blocks / p.ksplit);
 
     if (warp == 0) tmem_alloc<C::TMEM_COLS>(tmem_slot);
     if (warp == 1 && lane == 0) {
@@ -117,9 +130,12 @@ router_tc_kernel(const __grid_constant__ RouterTcParams p) {
             bool ok = true;
             for (int kb = kb_lo; kb < kb_hi; ++kb) {
                 if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
-                mbar_arrive_expect_tx(&full[stage], C::A_BYTES + C::B_BYTES);
-                tma_load_2d(smem + stage * C::A_BYTES, &p.a_map, &full[stage], (kb % p.d_blocks) * 64, m0);
-                tma_load_2d(smem + C::OFF_B + stage * C::B_BYTES, &p.b_map, &full[stage], kb * 64, n0);
+                mbar_arrive_expect_tx(&full[stage], C::A_BYTES + 3 * C::B_BYTES);
+                tma_load_2d(smem + stage * C::A_BYTES, &p.a_map, &full[stage], kb * 64, m0);
+#pragma unroll
+                for (int pl = 0; pl < 3; ++pl)
+                    tma_load_2d(smem + C::OFF_B + (stage * 3 + pl) * C::B_BYTES, &p.b_map, &full[stage],
+                                pl * p.d + kb * 64, n0);
                 ++issued;
                 if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
@@ -145,10 +161,14 @@ router_tc_kernel(const __grid_constant__ RouterTcParams p) {
                 if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
                 tc_fence_after();
                 const uint64_t adesc = smem_desc_k_sw128(smem + stage * C::A_BYTES);
-                const uint64_t bdesc = smem_desc_k_sw128(smem + C::OFF_B + stage * C::B_BYTES);
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    umma_f16(tmem_base, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > kb_lo || k > 0) ? 1u : 0u);
+                for (int pl = 0; pl < 3; ++pl) {
+                    const uint64_t bdesc = smem_desc_k_sw128(smem + C::OFF_B + (stage * 3 + pl) * C::B_BYTES);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        umma_f16(tmem_base, adesc + 2 * k, bdesc + 2 * k, idesc,
+                                 (kb > kb_lo || pl > 0 || k > 0) ? 1u : 0u);
+                }
                 issued_any = true;
                 umma_commit(&empty[stage]);
                 if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -217,7 +237,7 @@ cudaError_t launch_bn(const Dims& dm, const RouterTcPlan& plan, const RouterTcPa
 RouterTcPlan router_tc_plan(const Dims& dm) {
     RouterTcPlan pl{};
     pl.mt = (dm.T + RBM - 1) / RBM;
-    const int kb_total = 3 * dm.d / 64;
+    const int kb_total = dm.d / 64;          // 64-column blocks of d
     const int target = 148;                  // CTAs for one wave on a B200
     int ep = 32;
     while (ep < dm.E && ep < 256) ep *= 2;
@@ -236,10 +256,8 @@ RouterTcPlan router_tc_plan(const Dims& dm) {
 
 cudaError_t launch_router_tc(const Dims& dm, const RouterTcPlan& plan, const void* x, const float* W_r,
                              void* w3, float* part, int32_t* status, cudaStream_t st) {
-    const size_t n = static_cast<size_t>(dm.E) * dm.d;
-    int blocks = static_cast<int>((n + 255) / 256);
-    if (blocks > 4 * 148) blocks = 4 * 148;
-    router_split_kernel<<<blocks, 256, 0, st>>>(W_r, dm.E, dm.d, static_cast<__nv_bfloat16*>(w3));
+    const int col_blocks = (dm.d / 4 + 255) / 256;
+    router_split_kernel<<<dim3(col_blocks, dm.E), 256, 0, st>>>(W_r, dm.d, static_cast<__nv_bfloat16*>(w3));
     count_launches();
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -249,8 +267,8 @@ cudaError_t launch_router_tc(const Dims& dm, const RouterTcPlan& plan, const voi
     if (!encode_tma_2d(&p.b_map, w3, dm.E, 3 * dm.d, 2, plan.bn)) return cudaErrorInvalidValue;
     p.T = dm.T;
     p.E = dm.E;
+    p.d = dm.d;
     p.d_blocks = dm.d / 64;
-    p.kb_total = 3 * dm.d / 64;
     p.ksplit = plan.ksplit;
     p.part = part;
     p.status = status;
