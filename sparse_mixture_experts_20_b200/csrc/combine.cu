@@ -20,8 +20,10 @@ namespace {
 
 
 constexpr int CB_WARPS = 8;       // warps per combine block
+constexpr int kMaxWarpsPerToken = 32;
 
-// W warps per token (W = 1 for large batches, up to 8 for small ones).  Lanes
+// W warps per token (W = 1 for large batches, up to 32 -- four blocks -- for
+// small ones); global warp g serves token g / W, share g % W.  Lanes
 // 0..K-1 read the token's slot rows and gates and broadcast them; each lane
 // then owns 16-byte chunks of the output row: it issues the loads of all the
 // token's kept rows for a chunk before accumulating them in ascending k
@@ -31,9 +33,10 @@ __global__ void __launch_bounds__(32 * CB_WARPS, KT <= 8 ? 4 : 2)
 combine_kernel(const void* __restrict__ y_, const float* __restrict__ gates,
                const int32_t* __restrict__ slot_row, int T, int d, int K, int S, int r_cap,
                const void* __restrict__ x_, void* __restrict__ out_, int wpt) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int t = blockIdx.x * (CB_WARPS / wpt) + warp / wpt;
-    const int sub = warp % wpt;
+    const int lane = threadIdx.x & 31;
+    const int gw = blockIdx.x * CB_WARPS + (threadIdx.x >> 5);
+    const int t = gw / wpt;
+    const int sub = gw % wpt;
     if (t >= T) return;
     const int my_row = lane < K ? slot_row[static_cast<size_t>(t) * K + lane] : -1;
     const float my_g = lane < K ? gates[static_cast<size_t>(t) * K + lane] : 0.f;
@@ -141,8 +144,8 @@ cudaError_t launch_combine(const Dims& dm, const void* y, const float* gates,
     if (!dm.passthrough) x = nullptr;
     const bool f32 = dm.dtype == MOE_F32;
     int wpt = 1;                              // enough warps in flight to fill the GPU at small T
-    while (wpt < CB_WARPS && static_cast<long long>(dm.T) * wpt < 148LL * 32) wpt *= 2;
-    const int blocks = (dm.T + CB_WARPS / wpt - 1) / (CB_WARPS / wpt);
+    while (wpt < kMaxWarpsPerToken && static_cast<long long>(dm.T) * wpt < 148LL * 32) wpt *= 2;
+    const int blocks = static_cast<int>((static_cast<long long>(dm.T) * wpt + CB_WARPS - 1) / CB_WARPS);
 #define MOE_COMBINE(F, KT) combine_kernel<F, KT><<<blocks, 32 * CB_WARPS, 0, st>>>(          \
         y, gates, slot_row, dm.T, dm.d, dm.K, dm.S, dm.r_cap, x, out, wpt)
 #define MOE_COMBINE_K(F)                                                                         \

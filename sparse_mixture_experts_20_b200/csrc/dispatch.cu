@@ -8,14 +8,16 @@
 // item 5: tokens are dispatched in FP8.
 //
 // Three kernels, no atomics, deterministic:
-//   1. bitmap_kernel : warp per 32 tokens; for each expert j a ballot gives
-//      the 32-bit mask of those tokens that selected j -> bitmap[word][j].
+//   1. bitmap_kernel : warp per 32 tokens; lane i ORs bit i into the mask of
+//      each expert its token selected (shared memory), giving the 32-bit mask
+//      of the word's tokens that selected j -> bitmap[word][j].
 //      Out-of-range or repeated indices set MOE_DEV_BAD_ROUTING and are
 //      ignored.
 //   2. scan_kernel   : one block; per expert, prefix sums of popcounts over
 //      words -> word_base[word][j] (slots of j in earlier words), counts,
-//      kept = min(counts, C), offsets = exclusive scan of kept.
-//   3. scatter_kernel: warp per token; lane k < K finds the slot's rank
+//      kept = min(counts, C), offsets = exclusive scan of kept (parallel
+//      scans over word slices and over experts).
+//   3. scatter_kernel: warp(s) per token; lane k < K finds the slot's rank
 //      (word_base + popcount of the lower lanes' bits), keeps it if rank < C,
 //      writes slot_row / row_slot; then the warp copies (bf16/fp32) or
 //      quantises to e4m3 (FP8) the token's row into each kept destination
@@ -38,112 +40,133 @@ __device__ __forceinline__ bool slot_valid(const int* ids, int k, int E) {
 
 constexpr int MAXK = 16;
 
+// Warp per 32-token word.  The word's masks (planes * E of them) are built in
+// this warp's slice of shared memory by atomicOr -- K operations per lane
+// instead of a ballot per expert; OR does not depend on the order, so the
+// result is deterministic -- and then written out coalesced.
 __global__ void __launch_bounds__(256)
 bitmap_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int K, int t_words, int planes,
               uint32_t* __restrict__ bitmap, int32_t* status) {
+    extern __shared__ uint32_t bm_s[];                    // (warps of the block, planes * E)
     const int lane = threadIdx.x & 31;
-    const int w = blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (w >= t_words) return;
+    const int wib = threadIdx.x >> 5;
+    const int w = blockIdx.x * (blockDim.x >> 5) + wib;
+    if (w >= t_words) return;                             // whole warps only; no block barrier below
+    const int words = planes * E;
+    uint32_t* sm = bm_s + static_cast<size_t>(wib) * words;
+    for (int i = lane; i < words; i += 32) sm[i] = 0u;
     const int t = w * 32 + lane;
     int ids[MAXK];
-    bool bad = false;
 #pragma unroll
     for (int k = 0; k < MAXK; ++k) {
         ids[k] = -1;
         if (k < K && t < T) ids[k] = topk_idx[static_cast<size_t>(t) * K + k];
     }
-    int valid[MAXK];
+    bool bad = false;
+    __syncwarp();
 #pragma unroll
     for (int k = 0; k < MAXK; ++k) {
-        valid[k] = -1;
         if (k < K && t < T) {
-            if (slot_valid(ids, k, E)) valid[k] = ids[k];
-            else bad = true;
+            if (slot_valid(ids, k, E)) {
+                // planes == 1: one mask per expert; planes == K: one per slot
+                // index (slot-major capacity priority), plane k holding the
+                // k-th choices
+                atomicOr(&sm[(planes == 1 ? 0 : k) * E + ids[k]], 1u << lane);
+            } else {
+                bad = true;
+            }
         }
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) set_device_status(status, MOE_DEV_BAD_ROUTING);
-    // planes == 1: one bitmap per word (any slot); planes == K: one per slot
-    // index (slot-major capacity priority), plane p holding the p-th choices
-    for (int pl = 0; pl < planes; ++pl) {
-        for (int j0 = 0; j0 < E; j0 += 32) {
-            uint32_t mine = 0;
-            for (int jj = 0; jj < 32 && j0 + jj < E; ++jj) {
-                const int j = j0 + jj;
-                bool hit = false;
-                if (planes == 1) {
-#pragma unroll
-                    for (int k = 0; k < MAXK; ++k) hit |= (valid[k] == j);
-                } else {
-#pragma unroll
-                    for (int k = 0; k < MAXK; ++k) hit |= (k == pl && valid[k] == j);
-                }
-                const uint32_t m = __ballot_sync(0xffffffffu, hit);
-                if (lane == jj) mine = m;
-            }
-            if (j0 + lane < E) bitmap[(static_cast<size_t>(pl) * t_words + w) * E + j0 + lane] = mine;
-        }
+    __syncwarp();
+    for (int i = lane; i < words; i += 32) {
+        const int pl = i / E, j = i - pl * E;
+        bitmap[(static_cast<size_t>(pl) * t_words + w) * E + j] = sm[i];
     }
 }
 
-// One block of 1024 threads.  Thread (j, p): expert j, word slice p of P.
+// One block of 1024 threads.  Thread (p, j) = (tid / E, tid % E): expert j,
+// word slice p of P = 1024 / E (consecutive threads read consecutive experts
+// of one word: coalesced).  Per thread: the popcounts of its slice, loaded
+// eight words at a time; a scan over the slices of each expert; the
+// per-word prefixes written on a second pass over the (now cached) words;
+// and an exclusive scan of kept over the experts for the offsets.
 __global__ void __launch_bounds__(1024)
-scan_kernel(const uint32_t* __restrict__ bitmap, int E, int t_words, int capacity,
+scan_kernel(const uint32_t* __restrict__ bitmap, int E, int n_words, int capacity,
             int32_t* __restrict__ word_base, int32_t* __restrict__ counts,
             int32_t* __restrict__ kept, int32_t* __restrict__ offsets) {
     __shared__ int part[1024];
     __shared__ int kept_s[256];
-    int P = 1;
-    while (P * 2 * E <= 1024 && P < 128) P *= 2;
     const int tid = threadIdx.x;
-    const int j = tid / P, p = tid % P;
-    const int wpp = (t_words + P - 1) / P;
-    const int w0 = p * wpp, w1 = min(t_words, w0 + wpp);
+    const int P = 1024 / E;                                // >= 4: E <= 256
+    const int p = tid / E, j = tid - p * E;
+    const bool act = p < P;
+    const int wpp = (n_words + P - 1) / P;
+    const int w0 = act ? min(n_words, p * wpp) : 0;
+    const int w1 = act ? min(n_words, w0 + wpp) : 0;
     int sum = 0;
-    if (j < E)
-        for (int w = w0; w < w1; ++w) sum += __popc(bitmap[static_cast<size_t>(w) * E + j]);
+    {
+        int w = w0;
+        for (; w + 8 <= w1; w += 8) {
+            uint32_t v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = __ldg(bitmap + static_cast<size_t>(w + u) * E + j);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) sum += __popc(v[u]);
+        }
+        for (; w < w1; ++w) sum += __popc(__ldg(bitmap + static_cast<size_t>(w) * E + j));
+    }
     part[tid] = sum;
     __syncthreads();
-    if (j < E && p == 0) {                  // exclusive scan over the P slices of expert j
-        int run = 0;
-        for (int q = 0; q < P; ++q) {
-            const int v = part[tid + q];
-            part[tid + q] = run;
-            run += v;
+    for (int off = 1; off < P; off <<= 1) {                // inclusive scan over the slices of j
+        const int add = (act && p >= off) ? part[tid - off * E] : 0;
+        __syncthreads();
+        part[tid] += add;
+        __syncthreads();
+    }
+    if (act && p == P - 1) {
+        counts[j] = part[tid];
+        kept_s[j] = capacity >= 0 ? min(part[tid], capacity) : part[tid];
+    }
+    {
+        int run = part[tid] - sum;                         // words of j before this slice
+        int w = w0;
+        for (; w + 8 <= w1; w += 8) {
+            uint32_t v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = __ldg(bitmap + static_cast<size_t>(w + u) * E + j);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                word_base[static_cast<size_t>(w + u) * E + j] = run;
+                run += __popc(v[u]);
+            }
         }
-        counts[j] = run;
-        kept_s[j] = (capacity >= 0) ? min(run, capacity) : run;
+        for (; w < w1; ++w) {
+            word_base[static_cast<size_t>(w) * E + j] = run;
+            run += __popc(__ldg(bitmap + static_cast<size_t>(w) * E + j));
+        }
     }
     __syncthreads();
-    if (j < E) {
-        int run = part[tid];
-        for (int w = w0; w < w1; ++w) {
-            word_base[static_cast<size_t>(w) * E + j] = run;
-            run += __popc(bitmap[static_cast<size_t>(w) * E + j]);
-        }
+    const int kv = tid < E ? kept_s[tid] : 0;
+    int incl = kv;
+    for (int off = 1; off < E; off <<= 1) {                // inclusive scan of kept over experts
+        const int add = (tid < E && tid >= off) ? kept_s[tid - off] : 0;
+        __syncthreads();
+        if (tid < E) kept_s[tid] = (incl += add);
+        __syncthreads();
     }
-    if (tid < 32) {                         // offsets = exclusive scan of kept (warp 0)
-        int carry = 0;
-        for (int base = 0; base < E; base += 32) {
-            const int i = base + tid;
-            int v = (i < E) ? kept_s[i] : 0;
-            if (i < E) kept[i] = v;
-            int incl = v;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int o = __shfl_up_sync(0xffffffffu, incl, off);
-                if (tid >= off) incl += o;
-            }
-            if (i < E) offsets[i] = carry + incl - v;
-            carry += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        if (tid == 0) offsets[E] = carry;
+    if (tid < E) {
+        kept[tid] = kv;
+        offsets[tid] = incl - kv;
+        if (tid == E - 1) offsets[E] = incl;
     }
 }
 
 constexpr int SC_WARPS = 8;       // warps per scatter block
 
-// W warps per token (W = 1 for large batches; up to 8 when there are too few
-// tokens to fill the GPU).  Lanes 0..K-1 resolve the token's K slots to destination
+// W warps per token (W = 1 for large batches; up to 32 -- four blocks -- when
+// there are too few tokens to fill the GPU); global warp g serves token g / W,
+// share g % W.  Lanes 0..K-1 resolve the token's K slots to destination
 // rows (rank = word_base + popcount of the earlier tokens' bits of the word);
 // the rows are broadcast with shuffles and the warp copies (bf16 / fp32) or
 // quantises to e4m3 (FP8) the token's row into every kept destination with
@@ -159,9 +182,9 @@ scatter_kernel(const void* __restrict__ x_, const int32_t* __restrict__ topk_idx
                float* __restrict__ x_disp_scales, int wpt, int t_words, int slot_major) {
     constexpr int PF = 4;                                  // 16-byte chunks per lane in flight
     const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int t = blockIdx.x * (SC_WARPS / wpt) + warp / wpt;
-    const int sub = warp % wpt;                            // this warp's share of the row
+    const int gw = blockIdx.x * SC_WARPS + (threadIdx.x >> 5);
+    const int t = gw / wpt;
+    const int sub = gw % wpt;                              // this warp's share of the row
     if (t >= T) return;
     const int lane0 = sub * 32 + lane;                     // chunk of the first round
     const int stride = 32 * wpt;                           // chunks between rounds
@@ -279,8 +302,12 @@ cudaError_t launch_dispatch(const Dims& dm, const void* x, const int32_t* topk_i
                             int32_t* slot_row, int32_t* row_slot, void* x_disp,
                             float* x_disp_scales, uint32_t* bitmap, int32_t* word_base,
                             int32_t* status, cudaStream_t st) {
-    bitmap_kernel<<<(dm.t_words + 7) / 8, 256, 0, st>>>(topk_idx, dm.T, dm.E, dm.K, dm.t_words, dm.planes,
-                                                        bitmap, status);
+    // warps per block: up to 8, with at most 32 KB of masks in shared memory
+    const int words = dm.planes * dm.E;
+    int wpb = 8;
+    while (wpb > 1 && wpb * words * 4 > 32 * 1024) wpb >>= 1;
+    bitmap_kernel<<<(dm.t_words + wpb - 1) / wpb, 32 * wpb, static_cast<size_t>(wpb) * words * 4, st>>>(
+        topk_idx, dm.T, dm.E, dm.K, dm.t_words, dm.planes, bitmap, status);
     // the scan runs over the (plane, word) sequence: token order within a
     // plane, planes in slot order
     scan_kernel<<<1, 1024, 0, st>>>(bitmap, dm.E, dm.planes * dm.t_words, dm.capacity, word_base, counts, kept,
@@ -288,9 +315,8 @@ cudaError_t launch_dispatch(const Dims& dm, const void* x, const int32_t* topk_i
     const int shared_copy = (dm.dtype == MOE_FP8_E4M3_BLOCK && dm.S > 0) ? 1 : 0;
     // warps per token: enough warps in flight to fill the GPU at small T
     int wpt = 1;
-    while (wpt < SC_WARPS && static_cast<long long>(dm.T) * wpt < 148LL * 32) wpt *= 2;
-    const int tpb = SC_WARPS / wpt;
-    const int blocks = (dm.T + tpb - 1) / tpb;
+    while (wpt < 32 && static_cast<long long>(dm.T) * wpt < 148LL * 32) wpt *= 2;
+    const int blocks = static_cast<int>((static_cast<long long>(dm.T) * wpt + SC_WARPS - 1) / SC_WARPS);
 #define MOE_SCATTER(MODE) scatter_kernel<MODE><<<blocks, 32 * SC_WARPS, 0, st>>>(          \
         x, topk_idx, bitmap, word_base, offsets, dm.T, dm.d, dm.E, dm.K, dm.capacity,      \
         dm.r_cap, shared_copy, slot_row, row_slot, x_disp, x_disp_scales, wpt, dm.t_words, dm.slot_major)
