@@ -1,4 +1,5 @@
-"""fp64 CPU oracle of the sparse MoE FFN layer forward.
+"""fp64 CPU oracle of the sparse MoE FFN layer: the forward, and its backward
+for the fp32 and bf16 workloads.
 
 TEST INFRASTRUCTURE.  Only tests, the smoke check and the benchmark's
 CPU-baseline leg may import this module.  It shares no code with the CUDA
@@ -48,6 +49,16 @@ collapsed router gives alpha * N_r); the first C tokens kept under capacity;
 hand-computed capacities (including fp32 values of the capacity factor);
 the e4m3 and bf16 rounding against torch's conversions.  The expert FFN
 arithmetic beyond these is pinned only through the dense limit.
+
+The backward (layer_backward) is the derivative of this forward; the pages
+give no backward.  Its readings: the top-K choice, the capacity decisions and
+f_j are piecewise constant (no gradient through them); P_j carries the
+balance-loss gradient to s; a selection-only bias gets none.  Pins
+(tests/test_oracle_backward_pins.py): central differences of the forward's
+objective <dout, out> + lam * L_balance over every input and weight of tiny
+layers (capacity drops, pass-through, shared experts, both bias modes,
+K = 1, K = N_r); closed forms for K = 1, for the balance loss alone and for
+K = N_r (gates equal to the softmax).
 """
 from __future__ import annotations
 
@@ -63,6 +74,7 @@ __all__ = [
     "router_logits", "softmax", "topk_select", "gates_of", "capacity_of",
     "dispatch_plan", "silu", "expert_ffn", "balance_stats", "topk_gap",
     "route", "layer_forward", "to_f64", "expert_weights",
+    "silu_grad", "expert_ffn_backward", "layer_backward",
 ]
 
 E4M3_MAX = 448.0
@@ -424,3 +436,124 @@ def layer_forward(shape, inputs, tokens: Optional[np.ndarray] = None,
     if fp8:
         out = bf16_round(out)
     return {"out": out, "tokens": tokens, "routing": rt}
+
+
+# ----------------------------------------------------------------------------
+# Backward of the layer (the derivative of what the forward above computes;
+# the pages state the forward only: [DSMoE] §共有エキスパート機構 for the
+# output, §ルーティングとバランス損失 for the gates and the balance loss,
+# §アルゴリズム for the expert module; [TopK] §解決策2 for the capacity and the
+# overflow pass-through)
+# ----------------------------------------------------------------------------
+
+def silu_grad(z: np.ndarray) -> np.ndarray:
+    """d SiLU / dz = sigma(z) (1 + z (1 - sigma(z)))."""
+    sg = 1.0 / (1.0 + np.exp(-z))
+    return sg * (1.0 + z * (1.0 - sg))
+
+
+def expert_ffn_backward(xr: np.ndarray, dy: np.ndarray, W1: np.ndarray, b1: np.ndarray,
+                        W2: np.ndarray) -> dict:
+    """Gradients of y = W2 SiLU(W1 x + b1) + b2 over the rows of xr, given
+    dy = dJ/dy per row: dx (rows, d), dW1, db1, dW2, db2 summed over rows."""
+    z = xr @ W1.T + b1[None, :]
+    h = silu(z)
+    dh = dy @ W2
+    dz = dh * silu_grad(z)
+    return {"dx": dz @ W1, "dW1": dz.T @ xr, "db1": dz.sum(axis=0),
+            "dW2": dy.T @ h, "db2": dy.sum(axis=0)}
+
+
+def layer_backward(shape, inputs, dout: np.ndarray, lam: float = 1.0,
+                   routing: Optional[dict] = None) -> dict:
+    """Gradients of J = sum_t <dout_t, out_t> + lam * L_balance with respect
+    to x, the router weight, the per-expert bias and every expert's weights,
+    for the fp32 and bf16 workloads (fp64 throughout, nothing rounded).
+
+    Readings (the pages give no backward; this is the derivative of the
+    forward as the oracle computes it):
+      * the top-K choice, the capacity decisions and f_j (a fraction of
+        counts) are piecewise constant: no gradient flows through them;
+      * with S = sum_{k in TopK} s_k and g_k = s_{idx_k} / S, a slot's gate
+        gradient a_k = <dout_t, y_k> (kept), <dout_t, x_t> (dropped with
+        pass-through) or 0 (dropped), and ds_{idx_m} = (a_m - sum_k a_k g_k) / S;
+      * P_j = mean_t s_tj adds lam * alpha * N_r * f_j / T to every ds_tj;
+      * softmax: dl_i = s_i (ds_i - sum_j s_j ds_j); the router is linear, so
+        dW_r = dl^T x, dx += dl W_r, and the bias gets sum_t dl when it is
+        added to the logits (bias_mode 0); a selection-only bias (bias_mode 1)
+        enters only the top-K keys and gets none;
+      * a kept slot's expert sees dy = g_k dout_t; a dropped slot with
+        pass-through adds g_k dout_t to dx; shared experts see dy = dout_t.
+
+    Returns a dict with "x" (T, d), "W_r" (N_r, d), "logit_bias" (N_r,) or
+    None, "W1", "b1", "W2", "b2" (stacked over routed experts), "Ws1", "bs1",
+    "Ws2", "bs2" (shared, or None) and the intermediates "dgates" (T, K),
+    "ds" (T, N_r) and "dlogits" (T, N_r).
+    """
+    if shape.dtype == 2:
+        raise ValueError("layer_backward covers the fp32 and bf16 workloads")
+    rt = routing if routing is not None else route(shape, inputs)
+    T, K, N_r = shape.T, shape.top_k, shape.n_routed
+    x = to_f64(inputs["x"])
+    dout = np.asarray(dout, np.float64)
+    W_r = to_f64(inputs["W_r"])
+    s, idx, g = rt["s"], rt["idx"].astype(np.int64), rt["gates"]
+    slot_row = rt["plan"]["slot_row"]
+    passthrough = getattr(shape, "overflow_mode", 0) == 1
+    dx = np.zeros_like(x)
+    d_exp = {k: [] for k in ("W1", "b1", "W2", "b2")}
+    a = np.zeros((T, K), np.float64)                 # dJ/dg per slot
+    for e in range(N_r):
+        W1, b1, W2, b2 = expert_weights(inputs, "W", e, False)
+        slots = [(t, k) for t in range(T) for k in range(K) if idx[t, k] == e and slot_row[t, k] >= 0]
+        if slots:
+            tt = np.array([t for t, _ in slots])
+            kk = np.array([k for _, k in slots])
+            xr = x[tt]
+            y = expert_ffn(xr, W1, b1, W2, b2)
+            a[tt, kk] = np.einsum("rd,rd->r", dout[tt], y)
+            gb = expert_ffn_backward(xr, g[tt, kk][:, None] * dout[tt], W1, b1, W2)
+            np.add.at(dx, tt, gb["dx"])
+        else:
+            gb = {"dW1": np.zeros_like(W1), "db1": np.zeros_like(b1),
+                  "dW2": np.zeros_like(W2), "db2": np.zeros_like(b2)}
+        for k in d_exp:
+            d_exp[k].append(gb["d" + k])
+    for t in range(T):
+        for k in range(K):
+            if slot_row[t, k] < 0 and passthrough:
+                a[t, k] = float(dout[t] @ x[t])
+                dx[t] += g[t, k] * dout[t]
+    # gates -> s over the selected experts of each token
+    S = np.take_along_axis(s, idx, axis=1).sum(axis=1)
+    ds = np.zeros_like(s)
+    common = (a * g).sum(axis=1)
+    for t in range(T):
+        for k in range(K):
+            ds[t, idx[t, k]] += (a[t, k] - common[t]) / S[t]
+    # balance loss through P (f held constant)
+    f = rt["f"]
+    ds += lam * shape.alpha * N_r * f[None, :] / T
+    # softmax and the linear router
+    dl = s * (ds - (s * ds).sum(axis=1, keepdims=True))
+    dx += dl @ W_r
+    lb = inputs.get("logit_bias")
+    d_bias = None
+    if lb is not None:
+        d_bias = dl.sum(axis=0) if getattr(shape, "bias_mode", 0) == 0 else np.zeros(N_r)
+    shared = {k: None for k in ("Ws1", "bs1", "Ws2", "bs2")}
+    if shape.n_shared > 0:
+        parts = {k: [] for k in shared}
+        for si in range(shape.n_shared):
+            W1, b1, W2, b2 = expert_weights(inputs, "Ws", si, False)
+            gb = expert_ffn_backward(x, dout, W1, b1, W2)
+            dx += gb["dx"]
+            for k in ("W1", "b1", "W2", "b2"):
+                parts[("Ws" if k[0] == "W" else "bs") + k[1]].append(gb["d" + k])
+        shared = {k: np.stack(v) for k, v in parts.items()}
+    res = {"x": dx, "W_r": dl.T @ x, "logit_bias": d_bias,
+           "dgates": a, "ds": ds, "dlogits": dl}
+    for k in d_exp:
+        res[k] = np.stack(d_exp[k])
+    res.update(shared)
+    return res
