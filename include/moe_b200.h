@@ -297,6 +297,77 @@ MOE_EXPORT int moe_dispatch_noalloc(const moe_config* cfg, const void* x, const 
                                     int32_t* slot_row, int32_t* row_slot, void* x_disp,
                                     float* x_disp_scales, void* stream);
 
+/* ---- backward of the layer (fp32 and bf16 layers) ------------------------
+ * Gradients of J = sum_t <dout_t, out_t> + lam * L_balance with respect to x,
+ * W_r, the per-expert logit bias and every routed and shared expert's
+ * weights and biases.  The pages ("論文解説: DeepSeekMoE" §共有エキスパート機構,
+ * §ルーティングとバランス損失, §アルゴリズム; "Sparse MoE Top-Kルーティング"
+ * §解決策2) define the forward only; this is its derivative, read as:
+ *   - the top-K choice, the capacity decisions and f_j (a fraction of counts)
+ *     pass no gradient;
+ *   - slot (t, k) gets a = <dout_t, y of the slot> if kept, <dout_t, x_t> if
+ *     dropped with MOE_OVERFLOW_PASS, else 0; with S = sum over the selected
+ *     s, ds of the slot's expert += (a_k - sum_k' a_k' g_k') / S; P_j adds
+ *     lam * alpha * N_r * f_j / T to every ds_tj; dl = s * (ds - <s, ds>);
+ *   - dW_r = dl^T x; dx gets dl W_r; with MOE_BIAS_LOGITS the bias gets
+ *     sum_t dl, with MOE_BIAS_SELECTION (selection only) zero;
+ *   - a kept slot's expert sees dy = g * dout_t, a shared expert dout_t;
+ *     z = W1 x + b1 is recomputed; dz = (W2^T dy) * SiLU'(z); dW2 = dy SiLU(z)^T,
+ *     dW1 = dz x^T, db1 / db2 the sums of dz / dy; dx gets W1^T dz of each
+ *     kept slot, and g * dout_t of each slot dropped with pass-through.
+ * MOE_FP8_E4M3_BLOCK returns MOE_ERR_UNSUPPORTED.  Every reduction runs in a
+ * fixed order (bit-reproducible).  Inputs are the forward's inputs and the
+ * results of its stages on the same batch; outputs are fp32 and written in
+ * full (experts no slot reached get zero gradients).  All pointers are device
+ * memory, 16-byte aligned; NULL only where marked. */
+typedef struct moe_backward_io {
+    /* forward inputs */
+    const void* x;              /* (T, d_model) activation dtype */
+    const float* W_r;           /* (N_r, d_model) */
+    const void* W1;             /* (N_r, d_ff, d_model) activation dtype */
+    const float* b1;            /* (N_r, d_ff) */
+    const void* W2;             /* (N_r, d_model, d_ff) */
+    const float* b2;            /* (N_r, d_model) */
+    const void* Ws1;            /* (n_shared, d_ff_shared, d_model); NULL if n_shared == 0 */
+    const float* bs1;           /* (n_shared, d_ff_shared) */
+    const void* Ws2;            /* (n_shared, d_model, d_ff_shared) */
+    const float* bs2;           /* (n_shared, d_model) */
+    /* results of the forward stages */
+    const float* logits;        /* (T, N_r): moe_route's logits_out (the logits the softmax saw) */
+    const int32_t* topk_idx;    /* (T, K) moe_route */
+    const float* gates;         /* (T, K) moe_route */
+    const int32_t* counts;      /* (N_r) moe_dispatch: pre-capacity counts */
+    const int32_t* offsets;     /* (N_r + 1) moe_dispatch */
+    const int32_t* slot_row;    /* (T, K) moe_dispatch */
+    const int32_t* row_slot;    /* (R_cap) moe_dispatch */
+    const void* x_disp;         /* (x_disp rows, d_model) moe_dispatch */
+    const void* y;              /* (y rows, d_model) moe_expert_ffn */
+    /* upstream gradient */
+    const void* dout;           /* (T, d_model) activation dtype */
+    /* gradients, fp32 */
+    float* dx;                  /* (T, d_model) */
+    float* dW_r;                /* (N_r, d_model) */
+    float* d_logit_bias;        /* (N_r) or NULL */
+    float* dW1;                 /* (N_r, d_ff, d_model) */
+    float* db1;                 /* (N_r, d_ff) */
+    float* dW2;                 /* (N_r, d_model, d_ff) */
+    float* db2;                 /* (N_r, d_model) */
+    float* dWs1;                /* (n_shared, d_ff_shared, d_model); NULL if n_shared == 0 */
+    float* dbs1;                /* (n_shared, d_ff_shared) */
+    float* dWs2;                /* (n_shared, d_model, d_ff_shared) */
+    float* dbs2;                /* (n_shared, d_model) */
+} moe_backward_io;
+
+/* Bytes of the scratch moe_layer_backward needs (fp32 per-slot, per-token
+ * and per-row intermediates).  FP8 layers: MOE_ERR_UNSUPPORTED. */
+MOE_EXPORT int moe_backward_workspace_size(const moe_config* cfg, size_t* bytes);
+
+/* Enqueues the backward on `stream`.  lam: weight of the balance loss in J
+ * (finite).  bws: caller scratch of moe_backward_workspace_size() bytes,
+ * 256-byte aligned, any contents (fully rewritten before it is read). */
+MOE_EXPORT int moe_layer_backward(const moe_config* cfg, float lam, const moe_backward_io* io,
+                                  void* bws, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

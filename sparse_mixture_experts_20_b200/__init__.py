@@ -37,7 +37,7 @@ EXPORTED = (
     "moe_workspace_size", "moe_buffer_rows", "moe_workspace_init", "moe_get_device_status",
     "moe_last_cuda_error", "moe_status_string", "moe_route", "moe_dispatch", "moe_expert_ffn",
     "moe_combine", "moe_balance_stats", "moe_layer_forward", "moe_selftest_wait_timeout",
-    "moe_dispatch_noalloc", "moe_kernel_launches",
+    "moe_dispatch_noalloc", "moe_kernel_launches", "moe_backward_workspace_size", "moe_layer_backward",
 )
 
 
@@ -49,6 +49,18 @@ class moe_config(ctypes.Structure):
         ("alpha", ctypes.c_float), ("dtype", ctypes.c_int32), ("bias_mode", ctypes.c_int32),
         ("capacity_priority", ctypes.c_int32), ("overflow_mode", ctypes.c_int32),
     ]
+
+
+class moe_backward_io(ctypes.Structure):
+    """Pointers of moe_layer_backward, in the header's order."""
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "x", "W_r", "W1", "b1", "W2", "b2", "Ws1", "bs1", "Ws2", "bs2",
+        "logits", "topk_idx", "gates", "counts", "offsets", "slot_row", "row_slot", "x_disp", "y",
+        "dout",
+        "dx", "dW_r", "d_logit_bias", "dW1", "db1", "dW2", "db2", "dWs1", "dbs1", "dWs2", "dbs2")]
+
+
+BACKWARD_IO_FIELDS = tuple(n for n, _ in moe_backward_io._fields_)
 
 
 class MoEError(RuntimeError):
@@ -92,6 +104,8 @@ def lib() -> ctypes.CDLL:
             "moe_selftest_wait_timeout": [cfgp, ctypes.c_int64, P, P],
             "moe_dispatch_noalloc": [cfgp, P, P, P, P, P, P, P, P, P, P],
             "moe_kernel_launches": [],
+            "moe_backward_workspace_size": [cfgp, ctypes.POINTER(ctypes.c_size_t)],
+            "moe_layer_backward": [cfgp, ctypes.c_float, ctypes.POINTER(moe_backward_io), P, P],
         }
         restype = {"moe_status_string": ctypes.c_char_p, "moe_kernel_launches": ctypes.c_uint64}
         for name, args in sig.items():
@@ -216,6 +230,29 @@ def moe_layer_forward(cfg, x, W_r, logit_bias, W1, W1_scales, b1, W2, W2_scales,
 def moe_selftest_wait_timeout(cfg, timeout_ns: int, ws, stream=None):
     _check(lib().moe_selftest_wait_timeout(ctypes.byref(cfg), int(timeout_ns), _p(ws), _stream(stream)),
            "moe_selftest_wait_timeout")
+
+
+def moe_backward_workspace_size(cfg: moe_config) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().moe_backward_workspace_size(ctypes.byref(cfg), ctypes.byref(n)), "moe_backward_workspace_size")
+    return n.value
+
+
+def backward_io(tensors: dict) -> moe_backward_io:
+    """moe_backward_io from a dict of tensors keyed by the header's field
+    names (missing or None fields are NULL)."""
+    unknown = set(tensors) - set(BACKWARD_IO_FIELDS)
+    if unknown:
+        raise KeyError(f"not moe_backward_io fields: {sorted(unknown)}")
+    return moe_backward_io(**{n: _p(tensors.get(n)) for n in BACKWARD_IO_FIELDS})
+
+
+def moe_layer_backward(cfg, lam: float, tensors: dict, bws, stream=None):
+    """Gradients of <dout, out> + lam * L_balance (fp32, written into the dx,
+    dW_r, ... tensors of `tensors`); bws: moe_backward_workspace_size() bytes."""
+    io = backward_io(tensors)
+    _check(lib().moe_layer_backward(ctypes.byref(cfg), ctypes.c_float(lam), ctypes.byref(io), _p(bws),
+                                    _stream(stream)), "moe_layer_backward")
 
 
 def moe_dispatch_noalloc(cfg, x, topk_idx, counts, kept, offsets, slot_row, row_slot, x_disp,

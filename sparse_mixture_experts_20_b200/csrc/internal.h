@@ -141,4 +141,9 @@ void note_cuda_error(int err);
 // Adds n to the process-wide kernel launch counter (moe_kernel_launches).
 void count_launches(int n = 1);
 
+// Layer backward (backward.cu): scratch bytes and the launch sequence.
+size_t backward_ws_bytes(const Dims& dm);
+cudaError_t launch_backward(const Dims& dm, float lam, const moe_backward_io& io, void* bws,
+                            cudaStream_t st);
+
 }  // namespace moe

@@ -441,6 +441,34 @@ int moe_layer_forward(const moe_config* cfg, const void* x, const float* W_r, co
     return cuda_status(launch_balance(dm, cnt, at<float>(ws, L.psum), f, P, loss, st));
 }
 
+int moe_backward_workspace_size(const moe_config* cfg, size_t* bytes) {
+    Dims dm;
+    const int v = validate(cfg, &dm);
+    if (v != MOE_OK) return v;
+    if (!bytes) return MOE_ERR_INVALID_ARG;
+    if (dm.dtype == MOE_FP8_E4M3_BLOCK) return MOE_ERR_UNSUPPORTED;
+    *bytes = backward_ws_bytes(dm);
+    return MOE_OK;
+}
+
+int moe_layer_backward(const moe_config* cfg, float lam, const moe_backward_io* io, void* bws, void* stream) {
+    Dims dm;
+    const int v = validate(cfg, &dm);
+    if (v != MOE_OK) return v;
+    if (dm.dtype == MOE_FP8_E4M3_BLOCK) return MOE_ERR_UNSUPPORTED;
+    if (!io || !bws || (reinterpret_cast<uintptr_t>(bws) & 255u) || !std::isfinite(lam)) return MOE_ERR_INVALID_ARG;
+    const void* need[] = {io->x, io->W_r, io->W1, io->b1, io->W2, io->b2, io->logits, io->topk_idx, io->gates,
+                          io->counts, io->offsets, io->slot_row, io->row_slot, io->x_disp, io->y, io->dout,
+                          io->dx, io->dW_r, io->dW1, io->db1, io->dW2, io->db2};
+    for (const void* p : need) if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+    if (io->d_logit_bias && !aligned16(io->d_logit_bias)) return MOE_ERR_INVALID_ARG;
+    if (dm.S > 0) {
+        const void* sh[] = {io->Ws1, io->bs1, io->Ws2, io->bs2, io->dWs1, io->dbs1, io->dWs2, io->dbs2};
+        for (const void* p : sh) if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+    }
+    return cuda_status(launch_backward(dm, lam, *io, bws, static_cast<cudaStream_t>(stream)));
+}
+
 int moe_selftest_wait_timeout(const moe_config* cfg, int64_t timeout_ns, void* ws, void* stream) {
     Dims dm;
     const int v = validate(cfg, &dm);

@@ -141,3 +141,55 @@ def test_fp8_requires_scales():
     p = 0x10000
     args = [p] * 8 + [None, p, None]     # x .. x_disp valid, x_disp_scales NULL, ws, stream
     assert L.moe_dispatch(ctypes.byref(cfg), *args) == M.MOE_ERR_INVALID_ARG
+
+
+def _bwd_layout_bytes(T, d, E, K, dff, S, dffs, r_cap):
+    """Closed form of the backward scratch: fp32 regions, each rounded up to
+    256 bytes, in the order a, dl, dy, z, dz, dx rows, shared dy, z, dz, dx."""
+    regions = [T * K, T * E, r_cap * d, r_cap * dff, r_cap * dff, r_cap * d,
+               T * d if S else 0, T * dffs if S else 0, T * dffs if S else 0, T * d]
+    return sum((n * 4 + 255) // 256 * 256 for n in regions)
+
+
+@pytest.mark.parametrize("cid", [1, 2, 3])
+def test_backward_workspace_closed_form(cid):
+    sh = CONFIGS[cid]
+    cfg = M.make_config(sh)
+    _, r_cap, _, _ = M.moe_buffer_rows(cfg)
+    assert M.moe_backward_workspace_size(cfg) == _bwd_layout_bytes(
+        sh.T, sh.d_model, sh.n_routed, sh.top_k, sh.d_ff, sh.n_shared, sh.d_ff_shared, r_cap)
+
+
+def test_backward_rejects_fp8_and_bad_arguments_without_launch():
+    L = M.lib()
+    before = M.moe_kernel_launches()
+    n = ctypes.c_size_t(0)
+    fp8 = M.make_config(CONFIGS[4])
+    assert L.moe_backward_workspace_size(ctypes.byref(fp8), ctypes.byref(n)) == M.MOE_ERR_UNSUPPORTED
+    io = M.moe_backward_io()
+    assert L.moe_layer_backward(ctypes.byref(fp8), 1.0, ctypes.byref(io), 0x1000, None) == M.MOE_ERR_UNSUPPORTED
+    cfg = M.make_config(T=64, d_model=128, n_routed=8, top_k=2, d_ff=128, n_shared=1, d_ff_shared=64)
+    c = ctypes.byref(cfg)
+    assert L.moe_layer_backward(c, 1.0, None, 0x1000, None) == M.MOE_ERR_INVALID_ARG
+    # every field set to an aligned fake address except one required pointer:
+    # rejected on the host (the fakes are never dereferenced)
+    fake = {f: 0x10000 for f in M.BACKWARD_IO_FIELDS}
+    for missing in ("x", "logits", "row_slot", "dout", "dx", "dW1", "dWs2"):
+        io = M.moe_backward_io(**{k: (None if k == missing else v) for k, v in fake.items()})
+        assert L.moe_layer_backward(c, 1.0, ctypes.byref(io), 0x1000, None) == M.MOE_ERR_INVALID_ARG, missing
+    io = M.moe_backward_io(**{k: (0x10008 if k == "y" else v) for k, v in fake.items()})
+    assert L.moe_layer_backward(c, 1.0, ctypes.byref(io), 0x1000, None) == M.MOE_ERR_INVALID_ARG
+    io = M.moe_backward_io(**{k: (None if k == "dx" else v) for k, v in fake.items()})
+    assert L.moe_layer_backward(c, float("nan"), ctypes.byref(io), 0x1000, None) == M.MOE_ERR_INVALID_ARG
+    assert M.moe_kernel_launches() == before
+
+
+def test_backward_io_binding_names_every_field():
+    assert M.BACKWARD_IO_FIELDS[0] == "x" and M.BACKWARD_IO_FIELDS[-1] == "dbs2"
+    assert len(M.BACKWARD_IO_FIELDS) == 31
+    hdr = open(os.path.join(ROOT, "include", "moe_b200.h")).read()
+    body = hdr[hdr.index("typedef struct moe_backward_io"):hdr.index("} moe_backward_io;")]
+    declared = re.findall(r"\*\s*(\w+);", body)
+    assert tuple(declared) == M.BACKWARD_IO_FIELDS
+    with pytest.raises(KeyError):
+        M.backward_io({"not_a_field": None})
