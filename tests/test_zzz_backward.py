@@ -26,10 +26,10 @@ CASES = {
                                     dtype=DTYPE_F32, zipf_logit_bias=True),
     "bf16-pass-slot": MoEShape("k2", 150, 128, 8, 2, 128, capacity_factor=0.8, dtype=DTYPE_BF16,
                                capacity_priority=1, overflow_mode=1),
-    "bf16-selbias-shared": MoEShape("k3", 96, 64, 16, 4, 64, n_shared=2, d_ff_shared=64, dtype=DTYPE_BF16,
+    "bf16-selbias-shared": MoEShape("k3", 96, 128, 16, 4, 128, n_shared=2, d_ff_shared=64, dtype=DTYPE_BF16,
                                     bias_mode=1, selection_bias=True),
-    "f32-k-equals-n": MoEShape("k4", 40, 64, 4, 4, 64, dtype=DTYPE_F32),
-    "bf16-e64-k8": MoEShape("k5", 64, 64, 64, 8, 64, dtype=DTYPE_BF16),
+    "f32-k-equals-n": MoEShape("k4", 40, 128, 4, 4, 128, dtype=DTYPE_F32),
+    "bf16-e64-k8": MoEShape("k5", 64, 128, 64, 8, 128, dtype=DTYPE_BF16),
 }
 
 
