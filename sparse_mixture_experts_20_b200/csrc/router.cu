@@ -14,7 +14,8 @@
 //     once.
 //   * the tensor-core router (router_tc.cu, bf16 x, larger N_r): W_r split into
 //     three bf16 planes, one tcgen05 GEMM with K = 3 d, partial logits per K
-//     split summed here by router_reduce_kernel;
+//     split summed in split order by router_select_kernel as it loads them
+//     (up to 4 splits) or first by router_reduce_kernel;
 //   * router_generic_kernel (fp32 x with a large W_r): a shared-memory tiled
 //     fp32 GEMM.
 // All three end in select_block: per token a warp-wide softmax, a K-round

@@ -4,8 +4,9 @@
 // W_r x with an fp32 router weight.  The activations x are exactly bf16, so
 // the logits are computed as x (W_hi + W_mid + W_lo)^T where the three bf16
 // planes are the successive roundings of W_r (8 + 8 + 8 significant bits, so
-// their sum is W_r exactly): one bf16 GEMM with K = 3 d whose A operand
-// re-reads x for each plane and whose fp32 accumulator sums all three.
+// their sum is W_r exactly): one bf16 GEMM with K = 3 d, each block of x
+// multiplied by the same block of all three planes, into one fp32
+// accumulator.
 //
 // router_split_kernel writes the planes side by side, W3 = [hi | mid | lo]
 // (E rows of 3 d).  router_tc_kernel is a single-tile tcgen05 GEMM per CTA:
