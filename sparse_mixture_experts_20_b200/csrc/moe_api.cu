@@ -4,6 +4,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstring>
+#include <nvtx3/nvToolsExt.h>
 #include "common.cuh"
 #include "internal.h"
 
@@ -17,6 +18,15 @@ int cuda_status(cudaError_t e) {
     g_last_cuda_error = static_cast<int>(e);
     return MOE_ERR_CUDA;
 }
+
+// Named NVTX range over one entry point (the enqueue of its kernels), for
+// profiler timelines; without an attached tool the calls do nothing.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
@@ -335,6 +345,7 @@ const char* moe_status_string(int status) {
 
 int moe_route(const moe_config* cfg, const void* x, const float* W_r, const float* logit_bias,
               int32_t* topk_idx, float* gates, float* logits_out, void* ws, void* stream) {
+    NvtxRange nvtx("moe_route");
     Dims dm;
     const int v = validate(cfg, &dm);
     if (v != MOE_OK) return v;
@@ -348,6 +359,7 @@ int moe_route(const moe_config* cfg, const void* x, const float* W_r, const floa
 int moe_dispatch(const moe_config* cfg, const void* x, const int32_t* topk_idx, int32_t* counts,
                  int32_t* kept, int32_t* offsets, int32_t* slot_row, int32_t* row_slot, void* x_disp,
                  float* x_disp_scales, void* ws, void* stream) {
+    NvtxRange nvtx("moe_dispatch");
     Dims dm;
     const int v = validate(cfg, &dm);
     if (v != MOE_OK) return v;
@@ -366,6 +378,7 @@ int moe_expert_ffn(const moe_config* cfg, const void* x, const void* x_disp, con
                    const void* W2, const float* W2_scales, const float* b2, const void* Ws1,
                    const float* Ws1_scales, const float* bs1, const void* Ws2, const float* Ws2_scales,
                    const float* bs2, void* y, void* ws, void* stream) {
+    NvtxRange nvtx("moe_expert_ffn");
     Dims dm;
     const int v = validate(cfg, &dm);
     if (v != MOE_OK) return v;
@@ -380,6 +393,7 @@ int moe_expert_ffn(const moe_config* cfg, const void* x, const void* x_disp, con
 
 int moe_combine(const moe_config* cfg, const void* y, const float* gates, const int32_t* slot_row,
                 const void* x, void* out, void* stream) {
+    NvtxRange nvtx("moe_combine");
     Dims dm;
     const int v = validate(cfg, &dm);
     if (v != MOE_OK) return v;
@@ -390,6 +404,7 @@ int moe_combine(const moe_config* cfg, const void* y, const float* gates, const 
 
 int moe_balance_stats(const moe_config* cfg, const int32_t* counts, const void* ws, float* f, float* P,
                       float* loss, void* stream) {
+    NvtxRange nvtx("moe_balance_stats");
     Dims dm;
     const int v = validate(cfg, &dm);
     if (v != MOE_OK) return v;
@@ -406,6 +421,7 @@ int moe_layer_forward(const moe_config* cfg, const void* x, const float* W_r, co
                       const void* Ws2, const float* Ws2_scales, const float* bs2,
                       void* out, float* f, float* P, float* loss,
                       int32_t* topk_idx, float* gates, int32_t* counts, void* ws, void* stream) {
+    NvtxRange nvtx("moe_layer_forward");
     Dims dm;
     const int v = validate(cfg, &dm);
     if (v != MOE_OK) return v;
@@ -452,6 +468,7 @@ int moe_backward_workspace_size(const moe_config* cfg, size_t* bytes) {
 }
 
 int moe_layer_backward(const moe_config* cfg, float lam, const moe_backward_io* io, void* bws, void* stream) {
+    NvtxRange nvtx("moe_layer_backward");
     Dims dm;
     const int v = validate(cfg, &dm);
     if (v != MOE_OK) return v;
