@@ -278,7 +278,8 @@ MOE_EXPORT int moe_selftest_wait_timeout(const moe_config* cfg, int64_t timeout_
  * caller that cannot afford the device-wide synchronisation of cudaMalloc.
  * Same outputs as moe_dispatch (same kernels, bit for bit) but no `ws`
  * argument: the dispatch scratch (token bitmaps and prefix counts,
- * 2 * ceil(T/32) * N_r 32-bit words, each half rounded up to 256 bytes) comes
+ * 2 * P * ceil(T/32) * N_r 32-bit words with P = top_k under
+ * MOE_PRIORITY_SLOT and 1 otherwise, each half rounded up to 256 bytes) comes
  * from a 2 MiB array in device memory that belongs to the library, so every
  * GPU that loads the library holds those 2 MiB until the process exits.
  * Shapes whose scratch exceeds 2 MiB return MOE_ERR_UNSUPPORTED (e.g. T up to
