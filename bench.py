@@ -62,8 +62,8 @@ def parse():
 
 
 def workload(args):
-    from synthetic import CONFIGS
-    sh = CONFIGS[args.config]
+    from synthetic import WORKLOADS
+    sh = WORKLOADS[args.config]
     if args.set:
         kw = {}
         for item in args.set:
@@ -302,7 +302,7 @@ def run_ours(args):
     import torch.distributed as dist
 
     import sparse_mixture_experts_20_b200 as M
-    from synthetic import CONFIGS, make_inputs
+    from synthetic import WORKLOADS, make_inputs
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -7,7 +7,7 @@ CPU oracle and the CUDA library are fed from it.
 """
 from .inputs import (  # noqa: F401
     MoEShape,
-    CONFIGS,
+    WORKLOADS,
     DTYPE_F32,
     DTYPE_BF16,
     DTYPE_FP8,

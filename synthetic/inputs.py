@@ -62,7 +62,7 @@ class MoEShape:
         return dataclasses.replace(self, **kw)
 
 
-CONFIGS: Dict[int, MoEShape] = {
+WORKLOADS: Dict[int, MoEShape] = {
     1: MoEShape("tiny-fp32 T64 d128 E8 k2 ff256", 64, 128, 8, 2, 256,
                 dtype=DTYPE_F32),
     2: MoEShape("mixtral-8x7b-shaped T4096 d4096 E8 k2 ff14336 bf16",

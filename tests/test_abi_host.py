@@ -9,7 +9,7 @@ import pytest
 
 import oracle as O
 import sparse_mixture_experts_20_b200 as M
-from synthetic import CONFIGS
+from synthetic import WORKLOADS
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -59,9 +59,9 @@ def test_status_strings():
     assert L.moe_status_string(5) == b"MOE_ERR_DEVICE_TIMEOUT"
 
 
-@pytest.mark.parametrize("cid", sorted(CONFIGS))
+@pytest.mark.parametrize("cid", sorted(WORKLOADS))
 def test_workspace_and_rows_for_every_config(cid):
-    sh = CONFIGS[cid]
+    sh = WORKLOADS[cid]
     cfg = M.make_config(sh)
     assert M.moe_workspace_size(cfg) > 0
     cap, r_cap, xr, yr = M.moe_buffer_rows(cfg)
@@ -153,7 +153,7 @@ def _bwd_layout_bytes(T, d, E, K, dff, S, dffs, r_cap):
 
 @pytest.mark.parametrize("cid", [1, 2, 3])
 def test_backward_workspace_closed_form(cid):
-    sh = CONFIGS[cid]
+    sh = WORKLOADS[cid]
     cfg = M.make_config(sh)
     _, r_cap, _, _ = M.moe_buffer_rows(cfg)
     assert M.moe_backward_workspace_size(cfg) == _bwd_layout_bytes(
@@ -164,7 +164,7 @@ def test_backward_rejects_fp8_and_bad_arguments_without_launch():
     L = M.lib()
     before = M.moe_kernel_launches()
     n = ctypes.c_size_t(0)
-    fp8 = M.make_config(CONFIGS[4])
+    fp8 = M.make_config(WORKLOADS[4])
     assert L.moe_backward_workspace_size(ctypes.byref(fp8), ctypes.byref(n)) == M.MOE_ERR_UNSUPPORTED
     io = M.moe_backward_io()
     assert L.moe_layer_backward(ctypes.byref(fp8), 1.0, ctypes.byref(io), 0x1000, None) == M.MOE_ERR_UNSUPPORTED

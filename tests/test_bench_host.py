@@ -15,7 +15,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 
 import bench  # noqa: E402
-from synthetic import CONFIGS  # noqa: E402
+from synthetic import WORKLOADS  # noqa: E402
 
 
 def _free_port():
@@ -66,12 +66,12 @@ def test_set_overrides_build_a_reduced_case():
     sh = bench.workload(args)
     assert (sh.n_routed, sh.T, sh.d_model, sh.top_k) == (64, 1024, 7168, 8)
     assert sh.name.endswith("[n_routed=64,T=1024]")
-    assert bench.workload(bench.argparse.Namespace(config=2, set=[])) == CONFIGS[2]
+    assert bench.workload(bench.argparse.Namespace(config=2, set=[])) == WORKLOADS[2]
 
 
 def test_roofline_work_per_step_closed_forms():
     import numpy as np
-    sh = CONFIGS[2]
+    sh = WORKLOADS[2]
     kept = np.full(sh.n_routed, sh.T * sh.top_k // sh.n_routed)
     R = int(kept.sum())
     assert bench.algorithmic_ffn(sh, R) == 4.0 * sh.d_model * sh.d_ff * R
@@ -81,7 +81,7 @@ def test_roofline_work_per_step_closed_forms():
     act = R * d * 2 + 2 * R * f * 2 + R * d * 2
     assert touched == sh.n_routed and b == weights + act
     # FP8: one byte per weight plus the fp32 block scales
-    sh4 = CONFIGS[4]
+    sh4 = WORKLOADS[4]
     kept4 = np.zeros(sh4.n_routed, dtype=np.int64)
     kept4[:3] = 10
     b4, t4 = bench.ffn_bytes(sh4, kept4)
@@ -105,19 +105,19 @@ def test_traffic_lookup_requires_the_captured_sources():
 
 def test_ffn_kernel_follows_dtype_and_pair_switch(monkeypatch):
     monkeypatch.delenv("MOE_GEMM_PAIR", raising=False)
-    assert bench.ffn_kernel(CONFIGS[1])[0] == "ffn_f32_kernel"
-    assert bench.ffn_kernel(CONFIGS[2])[0] == "grouped_ffn_bf16_pair_kernel"
-    assert bench.ffn_kernel(CONFIGS[4])[0] == "grouped_ffn_fp8_kernel"
+    assert bench.ffn_kernel(WORKLOADS[1])[0] == "ffn_f32_kernel"
+    assert bench.ffn_kernel(WORKLOADS[2])[0] == "grouped_ffn_bf16_pair_kernel"
+    assert bench.ffn_kernel(WORKLOADS[4])[0] == "grouped_ffn_fp8_kernel"
     monkeypatch.setenv("MOE_GEMM_PAIR", "0")
-    assert bench.ffn_kernel(CONFIGS[2])[0] == "grouped_ffn_bf16_kernel"
+    assert bench.ffn_kernel(WORKLOADS[2])[0] == "grouped_ffn_bf16_kernel"
     for cid in (1, 2, 4):
-        for f in bench.ffn_kernel(CONFIGS[cid])[1]:
+        for f in bench.ffn_kernel(WORKLOADS[cid])[1]:
             assert os.path.exists(os.path.join(bench.CSRC, f))
 
 
 def test_stage_bytes_closed_forms():
     import numpy as np
-    sh = CONFIGS[2]
+    sh = WORKLOADS[2]
     T, d, E, K = sh.T, sh.d_model, sh.n_routed, sh.top_k
     kept = np.full(E, T * K // E)
     R = T * K

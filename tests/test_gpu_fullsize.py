@@ -8,7 +8,7 @@ import pytest
 import torch
 
 import oracle as O
-from synthetic import CONFIGS
+from synthetic import WORKLOADS
 
 import moe_testlib as TL
 
@@ -19,7 +19,7 @@ pytestmark = pytest.mark.gpu
 def test_fullsize_config(cid):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
-    sh = CONFIGS[cid]
+    sh = WORKLOADS[cid]
     inp = TL.gpu_inputs(sh, seed=0, on_device_gen=True)
     o = TL.run_stages(sh, inp)
     assert o["status"] == 0

@@ -8,14 +8,14 @@ import torch
 
 import oracle as O
 import sparse_mixture_experts_20_b200 as M
-from synthetic import CONFIGS, DTYPE_BF16, DTYPE_F32, DTYPE_FP8, MoEShape
+from synthetic import WORKLOADS, DTYPE_BF16, DTYPE_F32, DTYPE_FP8, MoEShape
 
 import moe_testlib as TL
 
 pytestmark = pytest.mark.gpu
 
 CASES = {
-    "cfg1-tiny-f32": CONFIGS[1],
+    "cfg1-tiny-f32": WORKLOADS[1],
     "f32-ragged-shared-cap": MoEShape("f32r", 203, 128, 6, 2, 192, n_shared=1, d_ff_shared=128,
                                       capacity_factor=1.0, dtype=DTYPE_F32),
     "bf16-ragged-shared-cap": MoEShape("b1", 777, 256, 8, 2, 384, n_shared=1, d_ff_shared=192,

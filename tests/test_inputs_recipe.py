@@ -16,7 +16,7 @@ import torch
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 
-from synthetic import CONFIGS, DTYPE_BF16, DTYPE_F32, DTYPE_FP8, MoEShape, encode_fp8_blocks, make_inputs  # noqa: E402
+from synthetic import WORKLOADS, DTYPE_BF16, DTYPE_F32, DTYPE_FP8, MoEShape, encode_fp8_blocks, make_inputs  # noqa: E402
 
 SH = MoEShape("recipe", 512, 256, 8, 2, 512, n_shared=1, d_ff_shared=256, dtype=DTYPE_BF16)
 
@@ -54,7 +54,7 @@ def test_seed_fixes_every_draw():
 
 
 def test_zipf_logit_bias_of_the_decode_workload():
-    sh = CONFIGS[5]
+    sh = WORKLOADS[5]
     b = make_inputs(sh.replace(T=4), seed=0, route_only=True)["logit_bias"].double().numpy()
     ranks = np.exp(-b / 1.5)                       # b = 1.5 ln(1/rank)
     assert np.allclose(ranks, np.round(ranks), rtol=0, atol=1e-3)
