@@ -129,7 +129,13 @@ def e4m3_round(v: np.ndarray) -> np.ndarray:
 
 
 def pow2_scale(amax: np.ndarray) -> np.ndarray:
-    """Smallest power of two 2^k with amax / 2^k <= 448; 1 where amax == 0."""
+    """Smallest power of two 2^k with amax / 2^k <= 448; 1 where amax == 0.
+
+    Scales are stored as fp32, so k is kept in the normal fp32 exponent range
+    [-126, 127] (a reading: the pages give no scale rule at all).  Only a
+    block whose amax is below 448 * 2^-126 (about 5.3e-36) meets the lower
+    bound; its scale is 2^-126 and its codes are then smaller than 448.  The
+    upper bound is out of reach of fp32 inputs."""
     amax = np.asarray(amax, dtype=np.float64)
     out = np.ones_like(amax)
     nz = amax > 0
@@ -138,7 +144,7 @@ def pow2_scale(amax: np.ndarray) -> np.ndarray:
     # guard the float log2 against an off-by-one at exact powers of two
     s = np.where(amax[nz] / s > E4M3_MAX, s * 2.0, s)
     s = np.where(amax[nz] / (s / 2.0) <= E4M3_MAX, s / 2.0, s)
-    out[nz] = s
+    out[nz] = np.clip(s, 2.0 ** -126, 2.0 ** 127)
     return out
 
 

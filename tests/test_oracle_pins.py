@@ -89,6 +89,57 @@ def test_selection_on_logits_equals_selection_on_softmax():
     assert np.array_equal(np.sort(by_s[ok], 1), np.sort(rt["idx"][ok], 1))
 
 
+# ---------------------------------------------------------------- near-tie gap
+#
+# topk_gap decides which tokens the end-to-end comparison leaves out (a K-th
+# and (K+1)-th logit closer than 1e-5 may swap between fp32 and fp64).  It is
+# the margin of the top-K choice: the K-th largest key minus the (K+1)-th,
+# infinite when every expert is chosen.
+
+@pytest.mark.parametrize("row,expect", [
+    # descending 3, 1, 1, 0
+    ([3.0, 1.0, 1.0, 0.0], {1: 2.0, 2: 0.0, 3: 1.0, 4: math.inf}),
+    # descending 2, 2, 0.5, 0.25, -1 (unsorted, with a tie at the top)
+    ([0.5, 2.0, -1.0, 2.0, 0.25], {1: 0.0, 2: 1.5, 3: 0.25, 4: 1.25, 5: math.inf}),
+])
+def test_topk_gap_hand_computed(row, expect):
+    l = np.array([row])
+    for K, g in expect.items():
+        assert O.topk_gap(l, K)[0] == g, (row, K)
+
+
+def test_topk_gap_is_the_margin_of_the_brute_force_choice():
+    # independent of any sort: the smallest chosen key minus the largest key
+    # left out, with the chosen set from the brute-force search above
+    rng = np.random.default_rng(9)
+    for n, K in [(5, 1), (6, 2), (7, 3), (8, 7)]:
+        l = rng.normal(size=(60, n)).round(2)          # some exact ties
+        got = O.topk_gap(l, K)
+        for t in range(l.shape[0]):
+            sel = _brute_topk(list(l[t]), K)
+            rest = [i for i in range(n) if i not in sel]
+            assert got[t] == min(l[t][sel]) - max(l[t][rest]), (n, K, t)
+
+
+def test_route_gap_uses_the_selection_keys():
+    # one token, d = 1: x = 1 and W_r = (3, 1, 1, 0) give logits 3, 1, 1, 0
+    x = np.array([[1.0]])
+    W_r = np.array([[3.0], [1.0], [1.0], [0.0]])
+    b = np.array([-2.5, 0.0, 0.25, 0.0])
+    inp = {"x": x, "W_r": W_r, "logit_bias": None}
+    sh = MoEShape("gap", 1, 1, 4, 1, 8, dtype=DTYPE_F32)
+    assert O.route(sh, inp)["gap"][0] == 2.0
+    assert O.route(sh.replace(top_k=2), inp)["gap"][0] == 0.0
+    # a bias changes the keys to 0.5, 1, 1.25, 0 in both modes: added to the
+    # logits (mode 0) or to the selection keys only (mode 1)
+    for mode in (0, 1):
+        inp_b = dict(inp, logit_bias=b)
+        r1 = O.route(sh.replace(bias_mode=mode), inp_b)
+        r2 = O.route(sh.replace(bias_mode=mode, top_k=2), inp_b)
+        assert list(r1["idx"][0]) == [2] and list(r2["idx"][0]) == [2, 1]
+        assert r1["gap"][0] == 0.25 and r2["gap"][0] == 0.5, mode
+
+
 # ---------------------------------------------------------------- dispatch plan
 
 @pytest.mark.parametrize("cf", [0.0, 0.5, 1.0, 1.25])
@@ -293,6 +344,23 @@ def test_pow2_scale_is_smallest_power_of_two():
     assert np.all(k == np.round(k))
     assert np.all(a / s <= 448.0) and np.all(a / (s / 2) > 448.0)
     assert O.pow2_scale(np.array([0.0]))[0] == 1.0
+
+
+def test_pow2_scale_stays_a_normal_fp32_value():
+    # amax = 448 * 2^-126 is the smallest block maximum whose own scale, 2^-126,
+    # is still a normal fp32 number; below it the scale stays at 2^-126
+    edge = 448.0 * 2.0 ** -126
+    tiny = np.array([edge, edge / 2, 1e-37, 2.0 ** -149, np.nextafter(edge, np.inf)])
+    s = O.pow2_scale(tiny)
+    assert list(s[:4]) == [2.0 ** -126] * 4
+    assert s[4] == 2.0 ** -125
+    # the stored scale survives a round trip through fp32 unchanged
+    assert np.array_equal(s.astype(np.float32).astype(np.float64), s)
+    # codes of a tiny block are the values over 2^-126, rounded to e4m3
+    v = np.full((1, 128), 1e-37)
+    codes, sc = O.quantize_rows_1x128(v)
+    assert sc[0, 0] == 2.0 ** -126
+    assert np.all(O.e4m3_decode(codes) == O.e4m3_decode(O.e4m3_round(np.array([1e-37 * 2.0 ** 126])))[0])
 
 
 def test_fp8_quantised_row_error_bound():
