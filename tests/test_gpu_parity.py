@@ -182,3 +182,28 @@ def test_host_batches_pipeline_matches_forward():
         torch.cuda.synchronize()
         assert torch.equal(outs[k], out.cpu()), k
         assert torch.equal(losses[k], loss.cpu()), k
+
+
+def test_fp8_tiny_block_scale_stays_normal():
+    """A 128-column block whose largest magnitude is below 448 * 2^-126 gets
+    the scale 2^-126, on the GPU as in the oracle, so codes and scales of the
+    dispatched rows still match bit for bit and the layer output stays within
+    tolerance."""
+    require_gpu()
+    sh = MoEShape("tiny-amax", 200, 512, 16, 4, 256, n_shared=1, d_ff_shared=128, dtype=DTYPE_FP8)
+    inp = TL.gpu_inputs(sh, seed=21)
+    x = inp["x"].clone()
+    x[3, 128:256] = (x[3, 128:256].float() * 1e-37).to(torch.bfloat16)     # amax ~ 3e-37
+    x[50, 0:128] = 1e-38                                                   # below 2^-126
+    x[77, 384:512] = (x[77, 384:512].float() * 2.0 ** -130).to(torch.bfloat16)
+    inp["x"] = x
+    o = TL.run_stages(sh, inp)
+    assert o["status"] == 0
+    rt_prod = TL.check_routing(sh, inp, o)
+    TL.check_dispatch(sh, inp, o, rt_prod)
+    sc = TL.cpu(o["x_disp_scales"]).double().numpy()
+    rc = o["r_cap"]
+    assert sc[rc + 3, 1] == 2.0 ** -126 and sc[rc + 50, 0] == 2.0 ** -126 and sc[rc + 77, 3] == 2.0 ** -126
+    TL.check_expert_ffn(sh, inp, o, rt_prod)
+    err, _ = TL.check_end_to_end(sh, inp, o["out"], TL.cpu(o["topk_idx"]).numpy())
+    assert err < TL.TOL_REL_FROB[sh.dtype], err
