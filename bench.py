@@ -1,21 +1,27 @@
 #!/usr/bin/env python
 """Benchmark of the sparse MoE FFN layer forward on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 4] [--workloads all|none|2,3]
+                    [--impl ours|reference]
 
 A step is one pass of the whole layer (router, dispatch, expert FFN grouped
 GEMMs, combine, balance statistics) over one batch of seeded synthetic input
-that is already resident in HBM.  The default workload is the
-Mixtral-8x7B-shaped bf16 layer (T=4096, d=4096, 8 experts, top-2,
-d_ff=14336).  Each timed step is bracketed by CUDA events on the launching
-stream, with a 256 MiB write between steps to flush L2.  Under torchrun each
-rank runs an independent replica (the layer forward has no cross-GPU
-exchange); the time is the max over ranks and the value counts the tokens of
-all ranks.
+that is already resident in HBM.  The headline workload is the largest one
+that fits one GPU: the DeepSeek-V3-shaped prefill layer (T=4096, d=7168, 256
+experts, top-8, d_ff=2048, one shared expert, FP8 e4m3 dispatch and weights
+with block scales, bf16 combine).  The other four workloads (tiny fp32,
+Mixtral-8x7B-shaped bf16, DeepSeekMoE-style bf16 with a capacity limit, V3
+decode with skewed routing) are measured the same way in the same run and
+nested under "workloads".  Each timed step is bracketed by CUDA events on the
+launching stream, with a 256 MiB write between steps (outside the events) to
+flush L2.  Under torchrun each rank runs an independent replica (the layer
+forward has no cross-GPU exchange); the time is the max over ranks and the
+value counts the tokens of all ranks.
 
-One JSON line on rank 0: tokens/s plus the grouped-GEMM roofline, the CPU
-oracle baseline (rank 0, N=1), an end-to-end figure through the public API
-with host buffers, and the SM clocks sampled during the timed region.
+One JSON line on rank 0: tokens/s plus the grouped-GEMM roofline, the
+per-stage HBM fractions, the CPU oracle baseline (rank 0, N=1), an end-to-end
+figure through the public API with host buffers, and the SM clocks sampled
+during the timed region; the same fields per nested workload.
 
 --impl reference times the CPU oracle (the reference implementation of this
 repository: a plain fp64 restatement of the pages) on bounded token samples
@@ -44,6 +50,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 CPU_SAMPLE = {1: 64, 2: 4096, 3: 8192, 4: 16, 5: 64}
 REF_SAMPLE = {1: 64, 2: 32, 3: 64, 4: 1, 5: 4}
 L2_FLUSH_BYTES = 256 << 20
+STAGES = ["route", "dispatch", "expert_ffn", "combine", "balance"]
 
 
 def parse():
@@ -51,7 +58,10 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--config", type=int, default=4, help="headline workload (1-5)")
+    ap.add_argument("--workloads", default="all",
+                    help="other workloads measured in the same run and nested in the line: "
+                         "'all' (the four others), 'none', or a comma list such as '2,3'")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -73,6 +83,17 @@ def workload(args):
         sh = sh.replace(**kw)
         sh = sh.replace(name=sh.name + " [" + ",".join(args.set) + "]")
     return sh
+
+
+def other_workloads(args):
+    """The workloads measured after the headline one, in ascending order."""
+    if args.set or args.workloads == "none":
+        return []
+    if args.workloads == "all":
+        ids = [1, 2, 3, 4, 5]
+    else:
+        ids = sorted({int(v) for v in args.workloads.split(",") if v.strip()})
+    return [c for c in ids if c != args.config]
 
 
 def load_peaks():
@@ -107,7 +128,16 @@ def workload_config(sh, seed, parallelism):
             "top_k": sh.top_k, "d_ff": sh.d_ff, "n_shared": sh.n_shared, "d_ff_shared": sh.d_ff_shared,
             "capacity_factor": sh.capacity_factor, "seed": seed, "parallelism": parallelism,
             "l2": ("n/a (host oracle)" if parallelism == "cpu"
-                   else "flushed between timed steps (256 MiB write)")}
+                   else "value: flushed between timed steps (256 MiB write, outside the timed events); "
+                        "e2e: not flushed, the expert weights read every step "
+                        f"({weight_bytes(sh) / 1e9:.2f} GB) exceed the 126 MB L2" +
+                        (" (this tiny workload fits in L2)" if weight_bytes(sh) < 126e6 else ""))}
+
+
+def weight_bytes(sh):
+    """Bytes of all routed and shared expert weights of the layer."""
+    wb = {0: 4, 1: 2, 2: 1}[sh.dtype]
+    return 2 * sh.d_model * (sh.n_routed * sh.d_ff + sh.n_shared * sh.d_ff_shared) * wb
 
 
 def dtype_name(sh):
@@ -280,6 +310,23 @@ def src_hash(files):
     return h.hexdigest()
 
 
+def stage_traffic(workload_name, stage):
+    """DRAM bytes (read + write) per step of a memory-bound stage's kernels,
+    from the committed ncu summary profiles/stage_traffic.json; None unless
+    it was captured on this workload with that stage's sources unchanged."""
+    p = os.path.join(ROOT, "profiles", "stage_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        for e in json.load(open(p)).get("entries", []):
+            if e.get("workload") == workload_name and e.get("stage") == stage and \
+                    e.get("src_sha1") == src_hash(e.get("sources", [])):
+                return e.get("dram_bytes_per_step")
+    except Exception:
+        return None
+    return None
+
+
 def traffic_from_profile(workload_name, kernel, sha):
     """DRAM bytes (read + write) of the grouped FFN launches of one step, from
     the committed ncu summary; None unless it was captured on this workload
@@ -296,26 +343,17 @@ def traffic_from_profile(workload_name, kernel, sha):
     return None
 
 
-def run_ours(args):
+def measure_workload(args, cid, sh, dev, world, rank, local, peaks, peak_src, cpu_baseline):
+    """Times K steps of one workload on this rank (max over ranks) and returns
+    its fields: tokens/s, per-stage times, the grouped-GEMM roofline, the
+    stage HBM fractions, the end-to-end figure, routing statistics, clocks,
+    and (rank 0 at N=1, if asked) the CPU oracle baseline."""
     import numpy as np
     import torch
-    import torch.distributed as dist
 
     import sparse_mixture_experts_20_b200 as M
-    from synthetic import WORKLOADS, make_inputs
+    from synthetic import make_inputs
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    sh = workload(args)
-    M.lib()
     inp = make_inputs(sh, seed=args.seed + rank, device=dev)
     cfg = M.make_config(sh)
     T, K, E, d = sh.T, sh.top_k, sh.n_routed, sh.d_model
@@ -338,7 +376,7 @@ def run_ours(args):
     g = inp.get
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    n_stage = 5
+    n_stage = len(STAGES)
 
     def step(ev):
         ev[0].record(stream)
@@ -356,10 +394,6 @@ def run_ours(args):
         M.moe_balance_stats(cfg, b["counts"], ws, b["f"], b["P"], b["loss"])
         ev[5].record(stream)
 
-    def barrier():
-        if world > 1:
-            dist.barrier(device_ids=[local])
-
     sampler = ClockSampler(local)
     sampler.start()
     for _ in range(args.warmup):
@@ -368,8 +402,10 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     assert M.moe_get_device_status(cfg, ws) == 0, "device status after warm-up"
 
+    # ---- device-timed steps: inputs resident in HBM, L2 flushed before each
+    # step (outside the events that bracket the step's stages)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_stage + 1)] for _ in range(args.steps)]
-    barrier()
+    barrier(world, local)
     torch.cuda.synchronize(dev)
     sampler.mark()
     launches0 = M.moe_kernel_launches()
@@ -379,7 +415,7 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     launches = M.moe_kernel_launches() - launches0
     sampler.mark()
-    barrier()
+    barrier(world, local)
     stage_ms = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(n_stage)]
                          for k in range(args.steps)])
     step_ms = stage_ms.sum(axis=1)
@@ -387,6 +423,7 @@ def run_ours(args):
     kept = b["kept"].cpu().numpy()
     counts = b["counts"].cpu().numpy()
     status = M.moe_get_device_status(cfg, ws)
+    del b
 
     # ---- end to end through the public API: pinned host x in, out + loss back
     layer = M.MoELayer(cfg, inp, device=dev)
@@ -397,11 +434,11 @@ def run_ours(args):
     for _ in range(max(1, min(args.warmup, 3))):
         x_dev.copy_(x_h, non_blocking=True)
         layer.forward(x_dev)
+    # serial: copy in, compute, copy back, one after another on one stream
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    barrier()
+    barrier(world, local)
     torch.cuda.synchronize(dev)
     for k in range(args.steps):
-        flush.zero_()
         e2e_ev[k][0].record(stream)
         x_dev.copy_(x_h, non_blocking=True)
         out, f, P, loss = layer.forward(x_dev)
@@ -409,25 +446,85 @@ def run_ours(args):
         loss_h.copy_(loss, non_blocking=True)
         e2e_ev[k][1].record(stream)
     torch.cuda.synchronize(dev)
-    barrier()
+    barrier(world, local)
     e2e_serial_ms = max_over_ranks(float(sum(a.elapsed_time(c) for a, c in e2e_ev)), world, dev)
     # pipelined: MoELayer.forward_host_batches overlaps batch k's compute with
     # batch k+1's host->device and batch k-1's device->host copies; every
     # batch's copies are inside the timed region (first copy in .. last copy out)
     layer.forward_host_batches([x_h] * 3, [out_h] * 3, [loss_h] * 3)
-    barrier()
+    barrier(world, local)
     torch.cuda.synchronize(dev)
-    ev0, ev1 = layer.forward_host_batches([x_h] * args.steps, [out_h] * args.steps, [loss_h] * args.steps,
-                                          between=flush.zero_)
+    ev0, ev1 = layer.forward_host_batches([x_h] * args.steps, [out_h] * args.steps, [loss_h] * args.steps)
     torch.cuda.synchronize(dev)
-    barrier()
+    barrier(world, local)
     e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     clocks = sampler.stop()
+    del layer, flush
 
-    peaks, peak_src = load_peaks()
-    ffn_ms = float(stage_ms[:, 2].mean())
+    ffn_ms = float(stage_ms[:, STAGES.index("expert_ffn")].mean())
     flops = algorithmic_ffn(sh, int(kept.sum()))
     fbytes, touched = ffn_bytes(sh, kept)
+    roof = ffn_roofline(sh, flops, fbytes, touched, ffn_ms, peaks, peak_src)
+
+    sb = stage_bytes(sh, kept)
+    stages_hbm = {}
+    for i, name in enumerate(STAGES):
+        if name in sb:
+            ms_i = float(stage_ms[:, i].mean())
+            gbs = sb[name] / (ms_i * 1e-3) / 1e9
+            stages_hbm[name] = {"bytes": sb[name], "gbs": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4),
+                                "traffic": stage_traffic(sh.name, name)}
+    res = {
+        "value": round(job_throughput(T, world, args.steps, total_ms), 1), "unit": "tokens/s",
+        "ms_per_step": round(total_ms / args.steps, 4),
+        "dtype": dtype_name(sh),
+        "config": workload_config(sh, args.seed, "replicas" if world > 1 else "single"),
+        "stages_ms": {n: round(float(stage_ms[:, i].mean()), 4) for i, n in enumerate(STAGES)},
+        "grouped_gemm_tflops": round(flops / (ffn_ms * 1e-3) / 1e12, 1),
+        "stages_hbm": stages_hbm,
+        "roofline": roof,
+        "e2e": {"value": round(job_throughput(T, world, args.steps, e2e_ms), 1), "unit": "tokens/s",
+                "copies": "pinned host x in and out + loss back every step, on their own streams, "
+                          "overlapping the neighbouring steps' compute (MoELayer.forward_host_batches)",
+                "serial_value": round(job_throughput(T, world, args.steps, e2e_serial_ms), 1),
+                "h2d_bytes_per_step": int(inp["x"].numel() * inp["x"].element_size()),
+                "d2h_bytes_per_step": int(T * d * (4 if sh.dtype == 0 else 2) + 4)},
+        "gpu_launches": launches,
+        "routing": {"max_load": int(counts.max()), "mean_load": float(counts.mean()),
+                    "experts_touched": int((counts > 0).sum()), "dropped": int(counts.sum() - kept.sum())},
+        "device_status": status,
+        "clocks": clocks,
+    }
+    if cpu_baseline and rank == 0 and world == 1:
+        host = oracle_inputs_on_host(inp)
+        # passes over the sample until about 10 s of host work (at least one)
+        n_tot, dt_tot, passes = 0, 0.0, 0
+        while passes == 0 or (dt_tot < 10.0 and passes < 16):
+            n, dt = time_oracle(sh, host, CPU_SAMPLE.get(cid, 64), args.seed + passes)
+            n_tot, dt_tot, passes = n_tot + n, dt_tot + dt, passes + 1
+        res["cpu_baseline"] = {"value": round(n_tot / dt_tot, 3), "unit": "tokens/s", "cores": oracle_threads(),
+                               "kind": "oracle",
+                               "sample": f"{passes} pass(es) of {n} of {T} tokens (routing of all {T} each pass), "
+                                         f"fp64 numpy, {dt_tot:.1f} s; fp32/bf16 inputs widened to fp64 once "
+                                         "before timing"}
+        del host
+    del inp
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    return res
+
+
+def barrier(world, local):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[local])
+
+
+def ffn_roofline(sh, flops, fbytes, touched, ffn_ms, peaks, peak_src):
+    """Roofline of the grouped expert FFN (both launches of a step): the
+    slower of the flops at the tensor peak and the bytes at the HBM peak
+    binds; achieved is the algorithmic work over the CUDA-event time."""
+    fp8 = sh.dtype == 2
     tens_peak = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
     t_tensor = flops / (tens_peak * 1e12)
     t_hbm = fbytes / (peaks["hbm_gbs"] * 1e9)
@@ -456,54 +553,49 @@ def run_ours(args):
             sus = sus * (2.0 if fp8 else 1.0)
             roof["frac_of_sustained_peak"] = round(roof["achieved"] / sus, 4)
     roof["algorithmic"] = {"flops": flops, "bytes": fbytes, "experts_touched": touched}
+    return roof
 
-    sb = stage_bytes(sh, kept)
-    stages_hbm = {}
-    for i, name in enumerate(["route", "dispatch", "expert_ffn", "combine", "balance"]):
-        if name in sb:
-            ms_i = float(stage_ms[:, i].mean())
-            gbs = sb[name] / (ms_i * 1e-3) / 1e9
-            stages_hbm[name] = {"bytes": sb[name], "gbs": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 4)}
-    value = job_throughput(T, world, args.steps, total_ms)
-    line = {
-        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": dtype_name(sh),
-        "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights, N(0,0.01) biases)",
-        "config": workload_config(sh, args.seed, "replicas" if world > 1 else "single"),
-        "impl": "ours",
-        "stages_ms": {n: round(float(stage_ms[:, i].mean()), 4) for i, n in
-                      enumerate(["route", "dispatch", "expert_ffn", "combine", "balance"])},
-        "grouped_gemm_tflops": round(flops / (ffn_ms * 1e-3) / 1e12, 1),
-        "stages_hbm": stages_hbm,
-        "roofline": roof,
-        "e2e": {"value": round(job_throughput(T, world, args.steps, e2e_ms), 1), "unit": "tokens/s",
-                "copies": "pinned host x in and out + loss back every step, on their own streams, "
-                          "overlapping the neighbouring steps' compute (MoELayer.forward_host_batches)",
-                "serial_value": round(job_throughput(T, world, args.steps, e2e_serial_ms), 1),
-                "h2d_bytes_per_step": int(inp["x"].numel() * inp["x"].element_size()),
-                "d2h_bytes_per_step": int(T * d * (4 if sh.dtype == 0 else 2) + 4)},
-        "gpu_launches": launches,
-        "routing": {"max_load": int(counts.max()), "mean_load": float(counts.mean()),
-                    "experts_touched": int((counts > 0).sum()), "dropped": int(counts.sum() - kept.sum())},
-        "device_status": status,
-        "clocks": clocks,
-    }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        host = oracle_inputs_on_host(inp)
-        # passes over the sample until about 10 s of host work (at least one)
-        n_tot, dt_tot, passes = 0, 0.0, 0
-        while passes == 0 or (dt_tot < 10.0 and passes < 16):
-            n, dt = time_oracle(sh, host, CPU_SAMPLE.get(args.config, 64), args.seed + passes)
-            n_tot, dt_tot, passes = n_tot + n, dt_tot + dt, passes + 1
-        line["cpu_baseline"] = {"value": round(n_tot / dt_tot, 3), "unit": "tokens/s", "cores": oracle_threads(),
-                                "kind": "oracle",
-                                "sample": f"{passes} pass(es) of {n} of {T} tokens (routing of all {T} each pass), "
-                                          f"fp64 numpy, {dt_tot:.1f} s; fp32/bf16 inputs widened to fp64 once "
-                                          "before timing"}
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import sparse_mixture_experts_20_b200 as M
+    from synthetic import WORKLOADS
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    M.lib()
+    peaks, peak_src = load_peaks()
+    head = measure_workload(args, args.config, workload(args), dev, world, rank, local, peaks, peak_src,
+                            cpu_baseline=not args.no_cpu_baseline)
+    nested = {}
+    for cid in other_workloads(args):
+        nested[str(cid)] = measure_workload(args, cid, WORKLOADS[cid], dev, world, rank, local, peaks, peak_src,
+                                            cpu_baseline=False)
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
+        line = {"metric": METRIC, "value": head["value"], "unit": head["unit"], "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": head["dtype"],
+                "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights, N(0,0.01) biases)",
+                "config": head["config"], "impl": "ours"}
+        for k in ("stages_ms", "grouped_gemm_tflops", "stages_hbm", "roofline", "e2e", "gpu_launches",
+                  "routing", "device_status", "clocks", "cpu_baseline"):
+            if k in head:
+                line[k] = head[k]
+        line["peaks"] = {"source": peak_src, "hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"]}
+        if nested:
+            line["workloads"] = nested
         print(json.dumps(line), flush=True)
 
 

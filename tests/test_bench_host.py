@@ -125,3 +125,33 @@ def test_stage_bytes_closed_forms():
     assert b["route"] == T * d * 2 + E * d * 4 + T * K * 8 + (T // 32) * E * 4
     assert b["dispatch"] == T * K * 4 + T * d * 2 + R * d * 2 + T * K * 4 + R * 4 + (2 * E + 1) * 4
     assert b["combine"] == R * d * 2 + T * K * 8 + T * d * 2
+
+
+def test_headline_is_the_v3_prefill_with_the_others_nested():
+    import bench
+    ns = bench.argparse.Namespace
+    # the default headline is the largest single-GPU workload: V3 prefill, FP8
+    import sys
+    old = sys.argv
+    try:
+        sys.argv = ["bench.py"]
+        args = bench.parse()
+    finally:
+        sys.argv = old
+    assert args.config == 4 and args.workloads == "all"
+    assert "v3-prefill" in bench.workload(args).name
+    assert bench.other_workloads(args) == [1, 2, 3, 5]
+    assert bench.other_workloads(ns(config=2, workloads="none", set=[])) == []
+    assert bench.other_workloads(ns(config=4, workloads="2,3,4", set=[])) == [2, 3]
+    # a reduced profiling case (--set) never carries nested workloads
+    assert bench.other_workloads(ns(config=4, workloads="all", set=["T=1024"])) == []
+
+
+def test_weight_bytes_of_the_workloads():
+    import bench
+    from synthetic import WORKLOADS
+    # 2 x 7168 x (256 + 1) x 2048 e4m3 bytes
+    assert bench.weight_bytes(WORKLOADS[4]) == 2 * 7168 * 257 * 2048
+    # Mixtral shape: 2 x 4096 x 8 x 14336 bf16 values
+    assert bench.weight_bytes(WORKLOADS[2]) == 2 * 4096 * 8 * 14336 * 2
+    assert bench.weight_bytes(WORKLOADS[1]) < 126e6 < bench.weight_bytes(WORKLOADS[3])
