@@ -282,15 +282,20 @@ MOE_EXPORT int moe_selftest_wait_timeout(const moe_config* cfg, int64_t timeout_
  * MOE_PRIORITY_SLOT and 1 otherwise, each half rounded up to 256 bytes) comes
  * from a 2 MiB array in device memory that belongs to the library, so every
  * GPU that loads the library holds those 2 MiB until the process exits.
- * Shapes whose scratch exceeds 2 MiB return MOE_ERR_UNSUPPORTED (e.g. T up to
- * 32768 tokens at N_r = 256).  The call allocates nothing.  The first call on
- * each device looks up the array's device address (cudaGetSymbolAddress, with
- * that device current); make that first call before any stream capture.
- * Every call on a device shares the one array and leaves its contents behind;
- * the kernels rewrite all of it before reading, so nothing needs clearing,
- * but calls that overlap on the GPU (other streams, other threads) race on it
- * and must be serialised by the caller.  Bad routing indices are dropped as
- * in moe_dispatch but not reported (there is no status word).
+ * Shapes whose scratch exceeds 2 MiB return MOE_ERR_UNSUPPORTED before any
+ * launch (e.g. T up to 32768 tokens at N_r = 256 with token priority; under
+ * slot-major priority with top_k = 8 and N_r = 64, T up to 16384).  The call
+ * allocates nothing.  The array used is the one of the calling thread's
+ * current CUDA context (the current device's primary context unless the
+ * caller made another context current), so `stream` must belong to that
+ * context.  The first call in each context looks up the array's device
+ * address there (cudaGetSymbolAddress) and keeps it for later calls; make
+ * that first call before any stream capture.  Every call in a context shares
+ * the one array and leaves its contents behind; the kernels rewrite all of it
+ * before reading, so nothing needs clearing, but calls that overlap on the
+ * GPU (other streams, other threads) race on it and must be serialised by
+ * the caller.  Bad routing indices are dropped as in moe_dispatch; there is
+ * no status word to report them, but their slot_row entries are -2.
  *   x, topk_idx, counts, kept, offsets, slot_row, row_slot, x_disp,
  *   x_disp_scales: as moe_dispatch. */
 MOE_EXPORT int moe_dispatch_noalloc(const moe_config* cfg, const void* x, const int32_t* topk_idx,

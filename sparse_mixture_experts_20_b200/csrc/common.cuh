@@ -33,6 +33,26 @@ __device__ __forceinline__ void set_device_status(int32_t* status, int32_t bits)
     if (status) atomicOr(status, bits);
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+//
+// The library launches its kernels with programmatic stream serialization
+// (launch_pdl in internal.h): a kernel may be scheduled while the previous
+// kernel of the stream is still finishing, so its launch and set-up overlap
+// that kernel's tail.  Every such kernel calls pdl_wait() before its first
+// access to global memory, read or write: it returns once the previous kernel
+// has completed and its writes are visible (at once when there was no such
+// launch).  pdl_allow_next(), called after the wait, lets the next kernel of
+// the stream be scheduled early in turn; because it comes after the wait,
+// a kernel two launches back has always completed by then.
+
+__device__ __forceinline__ void pdl_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_allow_next() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {

@@ -48,6 +48,8 @@ __global__ void __launch_bounds__(256)
 bitmap_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int K, int t_words, int planes,
               uint32_t* __restrict__ bitmap, int32_t* status) {
     extern __shared__ uint32_t bm_s[];                    // (warps of the block, planes * E)
+    pdl_wait();
+    pdl_allow_next();
     const int lane = threadIdx.x & 31;
     const int wib = threadIdx.x >> 5;
     const int w = blockIdx.x * (blockDim.x >> 5) + wib;
@@ -87,16 +89,21 @@ bitmap_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int K, int t_w
 
 // One block of 1024 threads.  Thread (p, j) = (tid / E, tid % E): expert j,
 // word slice p of P = 1024 / E (consecutive threads read consecutive experts
-// of one word: coalesced).  Per thread: the popcounts of its slice, loaded
-// eight words at a time; a scan over the slices of each expert; the
-// per-word prefixes written on a second pass over the (now cached) words;
-// and an exclusive scan of kept over the experts for the offsets.
+// of one word: coalesced).  Per thread: the popcounts of its slice (up to
+// SCAN_CACHE words loaded all at once and kept in registers for the second
+// pass; longer slices -- many slot planes -- are read in batches of eight,
+// twice); a scan over the slices of each expert; the per-word prefixes
+// written; and an exclusive scan of kept over the experts for the offsets.
+constexpr int SCAN_CACHE = 32;
+
 __global__ void __launch_bounds__(1024)
 scan_kernel(const uint32_t* __restrict__ bitmap, int E, int n_words, int capacity,
             int32_t* __restrict__ word_base, int32_t* __restrict__ counts,
             int32_t* __restrict__ kept, int32_t* __restrict__ offsets) {
     __shared__ int part[1024];
     __shared__ int kept_s[256];
+    pdl_wait();
+    pdl_allow_next();
     const int tid = threadIdx.x;
     const int P = 1024 / E;                                // >= 4: E <= 256
     const int p = tid / E, j = tid - p * E;
@@ -104,8 +111,16 @@ scan_kernel(const uint32_t* __restrict__ bitmap, int E, int n_words, int capacit
     const int wpp = (n_words + P - 1) / P;
     const int w0 = act ? min(n_words, p * wpp) : 0;
     const int w1 = act ? min(n_words, w0 + wpp) : 0;
+    const bool cached = wpp <= SCAN_CACHE;
+    int pc[SCAN_CACHE];
     int sum = 0;
-    {
+    if (cached) {
+#pragma unroll
+        for (int u = 0; u < SCAN_CACHE; ++u)
+            pc[u] = (w0 + u < w1) ? __popc(__ldg(bitmap + static_cast<size_t>(w0 + u) * E + j)) : 0;
+#pragma unroll
+        for (int u = 0; u < SCAN_CACHE; ++u) sum += pc[u];
+    } else {
         int w = w0;
         for (; w + 8 <= w1; w += 8) {
             uint32_t v[8];
@@ -130,20 +145,28 @@ scan_kernel(const uint32_t* __restrict__ bitmap, int E, int n_words, int capacit
     }
     {
         int run = part[tid] - sum;                         // words of j before this slice
-        int w = w0;
-        for (; w + 8 <= w1; w += 8) {
-            uint32_t v[8];
+        if (cached) {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = __ldg(bitmap + static_cast<size_t>(w + u) * E + j);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                word_base[static_cast<size_t>(w + u) * E + j] = run;
-                run += __popc(v[u]);
+            for (int u = 0; u < SCAN_CACHE; ++u) {
+                if (w0 + u < w1) word_base[static_cast<size_t>(w0 + u) * E + j] = run;
+                run += pc[u];
             }
-        }
-        for (; w < w1; ++w) {
-            word_base[static_cast<size_t>(w) * E + j] = run;
-            run += __popc(__ldg(bitmap + static_cast<size_t>(w) * E + j));
+        } else {
+            int w = w0;
+            for (; w + 8 <= w1; w += 8) {
+                uint32_t v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) v[u] = __ldg(bitmap + static_cast<size_t>(w + u) * E + j);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    word_base[static_cast<size_t>(w + u) * E + j] = run;
+                    run += __popc(v[u]);
+                }
+            }
+            for (; w < w1; ++w) {
+                word_base[static_cast<size_t>(w) * E + j] = run;
+                run += __popc(__ldg(bitmap + static_cast<size_t>(w) * E + j));
+            }
         }
     }
     __syncthreads();
@@ -181,6 +204,8 @@ scatter_kernel(const void* __restrict__ x_, const int32_t* __restrict__ topk_idx
                int32_t* __restrict__ row_slot, void* __restrict__ x_disp_,
                float* __restrict__ x_disp_scales, int wpt, int t_words, int slot_major) {
     constexpr int PF = 4;                                  // 16-byte chunks per lane in flight
+    pdl_wait();
+    pdl_allow_next();
     const int lane = threadIdx.x & 31;
     const int gw = blockIdx.x * SC_WARPS + (threadIdx.x >> 5);
     const int t = gw / wpt;
@@ -306,26 +331,28 @@ cudaError_t launch_dispatch(const Dims& dm, const void* x, const int32_t* topk_i
     const int words = dm.planes * dm.E;
     int wpb = 8;
     while (wpb > 1 && wpb * words * 4 > 32 * 1024) wpb >>= 1;
-    bitmap_kernel<<<(dm.t_words + wpb - 1) / wpb, 32 * wpb, static_cast<size_t>(wpb) * words * 4, st>>>(
-        topk_idx, dm.T, dm.E, dm.K, dm.t_words, dm.planes, bitmap, status);
+    cudaError_t e = launch_pdl(bitmap_kernel, dim3((dm.t_words + wpb - 1) / wpb), dim3(32 * wpb),
+                               static_cast<size_t>(wpb) * words * 4, st, 1,
+                               topk_idx, dm.T, dm.E, dm.K, dm.t_words, dm.planes, bitmap, status);
+    if (e != cudaSuccess) return e;
     // the scan runs over the (plane, word) sequence: token order within a
     // plane, planes in slot order
-    scan_kernel<<<1, 1024, 0, st>>>(bitmap, dm.E, dm.planes * dm.t_words, dm.capacity, word_base, counts, kept,
-                                    offsets);
+    e = launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, st, 1, bitmap, dm.E, dm.planes * dm.t_words, dm.capacity,
+                   word_base, counts, kept, offsets);
+    if (e != cudaSuccess) return e;
     const int shared_copy = (dm.dtype == MOE_FP8_E4M3_BLOCK && dm.S > 0) ? 1 : 0;
     // warps per token: enough warps in flight to fill the GPU at small T
     int wpt = 1;
     while (wpt < 32 && static_cast<long long>(dm.T) * wpt < 148LL * 32) wpt *= 2;
     const int blocks = static_cast<int>((static_cast<long long>(dm.T) * wpt + SC_WARPS - 1) / SC_WARPS);
-#define MOE_SCATTER(MODE) scatter_kernel<MODE><<<blocks, 32 * SC_WARPS, 0, st>>>(          \
-        x, topk_idx, bitmap, word_base, offsets, dm.T, dm.d, dm.E, dm.K, dm.capacity,      \
+#define MOE_SCATTER(MODE) e = launch_pdl(scatter_kernel<MODE>, dim3(blocks), dim3(32 * SC_WARPS), 0, st, 1,        \
+        x, topk_idx, bitmap, word_base, offsets, dm.T, dm.d, dm.E, dm.K, dm.capacity,                       \
         dm.r_cap, shared_copy, slot_row, row_slot, x_disp, x_disp_scales, wpt, dm.t_words, dm.slot_major)
     if (dm.dtype == MOE_F32) MOE_SCATTER(0);
     else if (dm.dtype == MOE_BF16) MOE_SCATTER(1);
     else MOE_SCATTER(2);
 #undef MOE_SCATTER
-    count_launches(3);
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace moe

@@ -41,6 +41,8 @@ ffn_f32_kernel(const __grid_constant__ F32Params p) {
     __shared__ int seg_rows[MAX_SEGS];
     __shared__ float As[FBK][FBM + 4];
     __shared__ float Bs[FBK][FBN + 4];
+    pdl_wait();
+    pdl_allow_next();
     const int tid = threadIdx.x;
     const int n0segs = p.g[0].n_mats, nseg = n0segs + p.g[1].n_mats;
     for (int s = tid; s < nseg; s += 256) {
@@ -137,9 +139,7 @@ cudaError_t launch_grouped_ffn_f32(const Dims& dm, const GemmArgs& a, cudaStream
     }
     p.silu = a.silu;
     const int mt_bound = (dm.r_cap + FBM - 1) / FBM + dm.E + dm.S * ((dm.T + FBM - 1) / FBM);
-    ffn_f32_kernel<<<dim3(mt_bound, ntiles), 256, 0, st>>>(p);
-    count_launches();
-    return cudaGetLastError();
+    return launch_pdl(ffn_f32_kernel, dim3(mt_bound, ntiles), dim3(256), 0, st, 1, p);
 }
 
 }  // namespace moe

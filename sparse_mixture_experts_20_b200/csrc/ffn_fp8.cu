@@ -31,7 +31,9 @@
 //               scale per row per 128 columns, so the amax is thread-local),
 //               or bias and bf16 output;
 //   warps 6..9  scale-factor writers: per stage, the 128 row scales of A and
-//               the two block scales of B (prefetched 4 stages ahead) as
+//               the two block scales of B (prefetched 4 stages ahead, in a
+//               register ring that the loop, unrolled over one turn, reloads
+//               slot by slot in place) as
 //               UE8M0, written with tcgen05.st into the stage's slot of
 //               tensor memory; they arrive on the stage's full barrier next to
 //               the TMA bytes, and wait on its empty barrier like the
@@ -49,18 +51,25 @@ namespace {
 using namespace ffn;
 
 constexpr int NUM_THREADS = 320;
-constexpr int BN = 256, BK = 128, STAGES = 4, LOOKAHEAD = 4;
+constexpr int BK = 128, STAGES = 4, LOOKAHEAD = 4;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t ACC1_COL = 192;                   // buffer 1; columns 192..255 shared with buffer 0
-constexpr uint32_t SF_COL0 = ACC1_COL + BN;          // scale-factor slots after the accumulators
 constexpr uint32_t SF_STRIDE = 16;                   // columns per stage slot (4 A + 8 B, padded)
 constexpr uint32_t FULL_ARRIVALS = 1 + 4;            // TMA expect_tx + one lane per scale-factor warp
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
 constexpr uint64_t kDrainTimeoutNs = 200000000ull;
-static_assert(SF_COL0 + STAGES * SF_STRIDE <= TMEM_COLS, "tensor memory budget");
-static_assert(BN - ACC1_COL == 64, "the epilogue drains two 32-column chunks first");
 
-struct Smem {
+// Tile geometry by the width BN of the weight tile: 256 (two accumulators
+// overlapping by 64 tensor-memory columns, see above) or 128 (two disjoint
+// accumulators, for batches with few rows per expert, where the number of
+// tiles -- not the work per tile -- decides how evenly the SMs are loaded).
+template <int BN_> struct FCfg {
+    static constexpr int BN = BN_;
+    static constexpr bool OVERLAP = BN == 256;
+    static constexpr uint32_t ACC1_COL = OVERLAP ? 192u : static_cast<uint32_t>(BN);   // buffer 1
+    static constexpr uint32_t SF_COL0 = ACC1_COL + BN;   // scale-factor slots after the accumulators
+    static_assert(BN == 128 || BN == 256, "weight tile width");
+    static_assert(SF_COL0 + STAGES * SF_STRIDE <= TMEM_COLS, "tensor memory budget");
+    static_assert(!OVERLAP || BN - ACC1_COL == 64, "the epilogue drains two 32-column chunks first");
     static constexpr int A_BYTES = BM * 128;
     static constexpr int B_BYTES = BN * 128;
     static constexpr int OFF_A = 0;
@@ -85,9 +94,10 @@ struct ItemIt {
     TileInfo ti;
 };
 
+template <int BN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
-    using L = Smem;
+    using L = FCfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -116,6 +126,8 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
         for (int gi = 0; gi < 2; ++gi)
             if (p.g[gi].n_mats > 0) { tma_prefetch_desc(&p.a_map[gi]); tma_prefetch_desc(&p.b_map[gi]); }
     }
+    pdl_wait();          // the segment table reads the dispatch offsets
+    pdl_allow_next();
     const int nseg = build_seg_table<BN>(p, seg, NUM_THREADS);
     tc_fence_before();
     __syncthreads();
@@ -164,20 +176,22 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
             for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
                 const TileInfo ti = decode_tile<BN, BK>(tile, p, seg, nseg);
                 // the previous tile's overlapping columns drained ...
-                if (!first && !mbar_wait_bounded(ovl, ovl_ph, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
-                if (!first) ovl_ph ^= 1u;
+                if (L::OVERLAP && !first) {
+                    if (!mbar_wait_bounded(ovl, ovl_ph, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
+                    ovl_ph ^= 1u;
+                }
                 first = false;
                 // ... and this buffer's tile from two tiles back fully drained
                 uint32_t& aph = abuf ? aph1 : aph0;
                 if (!mbar_wait_bounded(&acce[abuf], aph ^ 1u, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (abuf ? ACC1_COL : 0u);
+                const uint32_t d_tmem = tmem_base + (abuf ? L::ACC1_COL : 0u);
                 for (int kb = 0; kb < ti.kblocks; ++kb) {
                     if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t adesc = smem_desc_k_sw128(smem + L::OFF_A + stage * L::A_BYTES);
                     const uint64_t bdesc = smem_desc_k_sw128(smem + L::OFF_B + stage * L::B_BYTES);
-                    const uint32_t sfa = tmem_base + SF_COL0 + static_cast<uint32_t>(stage) * SF_STRIDE;
+                    const uint32_t sfa = tmem_base + L::SF_COL0 + static_cast<uint32_t>(stage) * SF_STRIDE;
 #pragma unroll
                     for (int k = 0; k < 4; ++k)            // 4 x 32 e4m3 of K per stage
                         umma_mxf8_bs(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, sfa, sfa + 4,
@@ -215,14 +229,14 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
             tc_fence_after();
             // this tile's accumulator; its overlapping columns are 192..255 of
             // buffer 0 (the second half) or 0..63 of buffer 1 (the first half)
-            const uint32_t acc = lane_base + (abuf ? ACC1_COL : 0u);
+            const uint32_t acc = lane_base + (abuf ? L::ACC1_COL : 0u);
             const float* bias = g.bias + static_cast<size_t>(ti.mat) * g.N + ti.n0;
             if (p.out_fp8) {
                 // first layer: bias + SiLU, then one e4m3 block per 128 columns
                 // per row; the half holding the overlap goes first
 #pragma unroll 1
                 for (int hi = 0; hi < BN / 128; ++hi) {
-                    const int h = abuf ? hi : (BN / 128 - 1 - hi);
+                    const int h = (abuf || !L::OVERLAP) ? hi : (BN / 128 - 1 - hi);
                     float v[128];
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
@@ -233,8 +247,8 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
                         for (int j = 0; j < 32; ++j) v[c * 32 + j] = __uint_as_float(r[j]);
                     }
                     tc_fence_before();
-                    if (hi == 0) mbar_arrive(ovl);               // overlap read: the next tile may start
-                    else mbar_arrive(&acce[abuf]);               // accumulator fully read: release it
+                    if (L::OVERLAP && hi == 0) mbar_arrive(ovl);  // overlap read: the next tile may start
+                    else if (hi == BN / 128 - 1) mbar_arrive(&acce[abuf]);   // fully read: release it
                     const int n_blk = ti.n0 + h * 128;
                     if (!row_ok || n_blk >= g.N) continue;
                     float amax = 0.f;
@@ -273,11 +287,11 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
                 const int n_valid = min(BN, g.N - ti.n0);
 #pragma unroll 1
                 for (int ci = 0; ci < BN / 32; ++ci) {
-                    const int c = abuf ? ci : (ci + 6) & 7;
+                    const int c = (abuf || !L::OVERLAP) ? ci : (ci + 6) & 7;
                     uint32_t r[32];
                     tmem_ld_32x32b_x32(acc + static_cast<uint32_t>(c * 32), r);
                     tmem_ld_wait();
-                    if (ci == 1) {                               // overlap read: the next tile may start
+                    if (L::OVERLAP && ci == 1) {                 // overlap read: the next tile may start
                         tc_fence_before();
                         mbar_arrive(ovl);
                     } else if (ci == BN / 32 - 1) {              // accumulator fully read: release it
@@ -309,7 +323,7 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
     } else {
         // ================= scale-factor writers (warps 6..9)
         const int quad = warp & 3;
-        const uint32_t sf_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + SF_COL0;
+        const uint32_t sf_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + L::SF_COL0;
         auto valid = [&](const ItemIt& it) { return it.tile < total_tiles; };
         auto start = [&](ItemIt& it) {
             it.tile = blockIdx.x;
@@ -335,7 +349,7 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
             }
             const int nb = g.N / 128;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
+            for (int h = 0; h < BN / 128; ++h) {
                 const int blk = it.ti.n0 / 128 + h;
                 b[h] = (blk < nb) ? __ldg(g.b_scales + (static_cast<size_t>(it.ti.mat) * nb + blk) * kq + it.kb) : 1.0f;
             }
@@ -343,40 +357,44 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
         ItemIt cur, ahead;
         start(cur);
         start(ahead);
-        float ra[LOOKAHEAD][4], rb[LOOKAHEAD][2];
+        float ra[LOOKAHEAD][4], rb[LOOKAHEAD][2] = {};
 #pragma unroll
         for (int j = 0; j < LOOKAHEAD; ++j) {
             if (valid(ahead)) { load(ahead, ra[j], rb[j]); advance(ahead); }
         }
-        int stage = 0;
+        // Item i of the stream uses stage i % STAGES and ring slot i % LOOKAHEAD,
+        // the same index: the loop is unrolled over one turn of the ring, so a
+        // slot's scales (loaded LOOKAHEAD items earlier) are converted and the
+        // slot reloaded in place, with no register moves that would wait on a
+        // load still in flight.
+        static_assert(STAGES == LOOKAHEAD, "one ring slot per stage");
         uint32_t phase = 0;
+        bool aborted = false;
 #pragma unroll 1
-        while (valid(cur)) {
-            // the oldest prefetched scales; the ring shifts by one (register
-            // moves only, so the loop body exists once)
-            const uint32_t wa0 = ue8m0_x4(ra[0][0]), wa1 = ue8m0_x4(ra[0][1]);
-            const uint32_t wa2 = ue8m0_x4(ra[0][2]), wa3 = ue8m0_x4(ra[0][3]);
-            const uint32_t wb0 = ue8m0_x4(rb[0][0]), wb1 = ue8m0_x4(rb[0][1]);
+        while (valid(cur) && !aborted) {
 #pragma unroll
-            for (int j = 0; j + 1 < LOOKAHEAD; ++j) {
-#pragma unroll
-                for (int c = 0; c < 4; ++c) ra[j][c] = ra[j + 1][c];
-                rb[j][0] = rb[j + 1][0];
-                rb[j][1] = rb[j + 1][1];
+            for (int j = 0; j < LOOKAHEAD; ++j) {
+                if (!valid(cur)) break;
+                const uint32_t wa0 = ue8m0_x4(ra[j][0]), wa1 = ue8m0_x4(ra[j][1]);
+                const uint32_t wa2 = ue8m0_x4(ra[j][2]), wa3 = ue8m0_x4(ra[j][3]);
+                const uint32_t wb0 = ue8m0_x4(rb[j][0]), wb1 = ue8m0_x4(rb[j][1]);
+                if (valid(ahead)) { load(ahead, ra[j], rb[j]); advance(ahead); }
+                if (!warp_wait(&empty[j], phase ^ 1u, abort_flag, p.status, p.timeout_ns, lane)) {
+                    aborted = true;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t slot = sf_base + static_cast<uint32_t>(j) * SF_STRIDE;
+                tmem_st_32x32b_x4(slot, wa0, wa1, wa2, wa3);
+                tmem_st_32x32b_x4(slot + 4, wb0, wb0, wb0, wb0);
+                if (BN == 256) tmem_st_32x32b_x4(slot + 8, wb1, wb1, wb1, wb1);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full[j]);
+                advance(cur);
             }
-            if (valid(ahead)) { load(ahead, ra[LOOKAHEAD - 1], rb[LOOKAHEAD - 1]); advance(ahead); }
-            if (!warp_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, p.timeout_ns, lane)) break;
-            tc_fence_after();
-            const uint32_t slot = sf_base + static_cast<uint32_t>(stage) * SF_STRIDE;
-            tmem_st_32x32b_x4(slot, wa0, wa1, wa2, wa3);
-            tmem_st_32x32b_x4(slot + 4, wb0, wb0, wb0, wb0);
-            tmem_st_32x32b_x4(slot + 8, wb1, wb1, wb1, wb1);
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&full[stage]);
-            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
-            advance(cur);
+            phase ^= 1u;
         }
     }
 
@@ -388,18 +406,28 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
     }
 }
 
-}  // namespace
-
-cudaError_t launch_grouped_ffn_fp8(const Dims&, const GemmArgs& a, cudaStream_t st) {
+template <int BN>
+cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
     TcParams p;
     if (!fill_params(p, a, 1, BN, kWaitTimeoutNs)) return cudaErrorInvalidValue;
-    constexpr int smem = Smem::ALLOC;
+    constexpr int smem = FCfg<BN>::ALLOC;
     static_assert(smem <= 227 * 1024, "shared memory budget");
-    cudaError_t e = cudaFuncSetAttribute(grouped_ffn_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(grouped_ffn_fp8_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    grouped_ffn_fp8_kernel<<<device_sm_count(), NUM_THREADS, smem, st>>>(p);
-    count_launches();
-    return cudaGetLastError();
+    return launch_pdl(grouped_ffn_fp8_kernel<BN>, dim3(device_sm_count()), dim3(NUM_THREADS), smem, st, 1, p);
+}
+
+}  // namespace
+
+// Weight tiles 128 wide when the batch averages fewer than 64 rows per
+// routed expert (decode-like: every tile streams its weights once and the
+// tile count sets the balance over the SMs), else 256 wide.
+int fp8_weight_tile(const Dims& dm) {
+    return static_cast<long long>(dm.T) * dm.K < 64LL * dm.E ? 128 : 256;
+}
+
+cudaError_t launch_grouped_ffn_fp8(const Dims& dm, const GemmArgs& a, cudaStream_t st) {
+    return fp8_weight_tile(dm) == 128 ? launch_bn<128>(a, st) : launch_bn<256>(a, st);
 }
 
 }  // namespace moe

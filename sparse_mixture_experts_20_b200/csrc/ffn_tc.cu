@@ -84,6 +84,8 @@ grouped_ffn_bf16_kernel(const __grid_constant__ TcParams p) {
             if (p.g[gi].n_mats > 0) { tma_prefetch_desc(&p.a_map[gi]); tma_prefetch_desc(&p.b_map[gi]); }
         }
     }
+    pdl_wait();          // the segment table reads the dispatch offsets
+    pdl_allow_next();
     const int nseg = build_seg_table<BN>(p, seg, NUM_THREADS);
     tc_fence_before();
     __syncthreads();
@@ -234,9 +236,7 @@ cudaError_t launch_grouped_ffn_bf16(const Dims&, const GemmArgs& a, cudaStream_t
     static_assert(smem <= 227 * 1024, "shared memory budget");
     cudaError_t e = cudaFuncSetAttribute(grouped_ffn_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    grouped_ffn_bf16_kernel<<<device_sm_count(), NUM_THREADS, smem, st>>>(p);
-    count_launches();
-    return cudaGetLastError();
+    return launch_pdl(grouped_ffn_bf16_kernel, dim3(device_sm_count()), dim3(NUM_THREADS), smem, st, 1, p);
 }
 
 }  // namespace moe

@@ -131,6 +131,8 @@ grouped_ffn_bf16_pair_kernel(const __grid_constant__ TcParams p) {
         for (int gi = 0; gi < 2; ++gi)
             if (p.g[gi].n_mats > 0) { tma_prefetch_desc(&p.a_map[gi]); tma_prefetch_desc(&p.b_map[gi]); }
     }
+    pdl_wait();          // the segment table reads the dispatch offsets
+    pdl_allow_next();
     const int nseg = build_seg_table<BN, 2>(p, seg, NUM_THREADS);
     tc_fence_before();
     __syncthreads();
@@ -333,11 +335,7 @@ cudaError_t launch_grouped_ffn_bf16_pair(const Dims&, const GemmArgs& a, cudaStr
     e = cudaOccupancyMaxActiveClusters(&clusters, grouped_ffn_bf16_pair_kernel, &cfg);
     if (e != cudaSuccess) return e;
     if (clusters < 1) return cudaErrorLaunchOutOfResources;
-    cfg.gridDim = dim3(2 * clusters);
-    e = cudaLaunchKernelEx(&cfg, grouped_ffn_bf16_pair_kernel, p);
-    count_launches();
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
+    return launch_pdl(grouped_ffn_bf16_pair_kernel, dim3(2 * clusters), dim3(NUM_THREADS), smem, st, 2, p);
 }
 
 }  // namespace moe

@@ -5,10 +5,21 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include "../../include/moe_b200.h"
 
 namespace moe {
+
+// Named NVTX range over one entry point (the enqueue of its kernels), for
+// profiler timelines; without an attached tool the calls do nothing.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Workspace layout: byte offsets of every region, all 256-byte aligned.
 struct WsLayout {
@@ -48,6 +59,11 @@ struct Dims {
 };
 
 constexpr int kRouteTokens = 32;    // tokens per router block
+
+// Programmatic dependent launch is on unless the environment variable
+// MOE_PDL is "0" (read once).
+bool pdl_enabled();
+
 
 int validate(const moe_config* cfg, Dims* dm);
 WsLayout ws_layout(const Dims& dm);
@@ -127,6 +143,8 @@ cudaError_t launch_grouped_ffn_bf16_pair(const Dims& dm, const GemmArgs& a, cuda
 // CTA-pair kernels are used unless the environment variable MOE_GEMM_PAIR is "0".
 bool gemm_pairs_enabled();
 cudaError_t launch_grouped_ffn_fp8(const Dims& dm, const GemmArgs& a, cudaStream_t st);
+// Weight-tile width (128 or 256) the FP8 grouped GEMM uses for this shape.
+int fp8_weight_tile(const Dims& dm);
 
 cudaError_t launch_wait_selftest(int64_t timeout_ns, int32_t* status, cudaStream_t st);
 
@@ -145,5 +163,36 @@ void count_launches(int n = 1);
 size_t backward_ws_bytes(const Dims& dm);
 cudaError_t launch_backward(const Dims& dm, float lam, const moe_backward_io& io, void* bws,
                             cudaStream_t st);
+
+// Launches `kernel` on `st` with programmatic stream serialization (the
+// kernel must call pdl_wait() before it touches global memory) and, with
+// cluster_x > 1, in clusters of cluster_x CTAs along x.  Returns the launch
+// error; counts the launch.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       int cluster_x, Args&&... args) {
+    cudaLaunchAttribute attr[2];
+    unsigned n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
+    ++n;
+    if (cluster_x > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = static_cast<unsigned>(cluster_x);
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    count_launches(1);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
 
 }  // namespace moe

@@ -3,8 +3,8 @@
 // anything, and returns a MOE_* status; no C++ exception crosses the ABI.
 #include <atomic>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
-#include <nvtx3/nvToolsExt.h>
 #include "common.cuh"
 #include "internal.h"
 
@@ -18,15 +18,6 @@ int cuda_status(cudaError_t e) {
     g_last_cuda_error = static_cast<int>(e);
     return MOE_ERR_CUDA;
 }
-
-// Named NVTX range over one entry point (the enqueue of its kernels), for
-// profiler timelines; without an attached tool the calls do nothing.
-struct NvtxRange {
-    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
-    ~NvtxRange() { nvtxRangePop(); }
-    NvtxRange(const NvtxRange&) = delete;
-    NvtxRange& operator=(const NvtxRange&) = delete;
-};
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
@@ -266,6 +257,14 @@ __global__ void wait_selftest_kernel(int64_t timeout_ns, int32_t* status) {
 }  // namespace
 
 void note_cuda_error(int err) { g_last_cuda_error = err; }
+
+bool pdl_enabled() {
+    static const bool on = [] {
+        const char* v = std::getenv("MOE_PDL");
+        return !(v && v[0] == '0');
+    }();
+    return on;
+}
 
 static std::atomic<uint64_t> g_kernel_launches{0};
 void count_launches(int n) { g_kernel_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }

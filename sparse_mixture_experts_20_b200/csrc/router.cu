@@ -164,6 +164,8 @@ router_generic_kernel(const XT* __restrict__ x, const float* __restrict__ W_r,
     __shared__ float wsh[(NP * (KC + 1) > TT * (NP + 1)) ? NP * (KC + 1) : TT * (NP + 1)];
     float (*wtile)[KC + 1] = reinterpret_cast<float (*)[KC + 1]>(wsh);
     float (*lg)[NP + 1] = reinterpret_cast<float (*)[NP + 1]>(wsh);
+    pdl_wait();
+    pdl_allow_next();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int t0 = blockIdx.x * TT;
     float acc[4][EPT];
@@ -274,6 +276,8 @@ router_small_kernel(const XT* __restrict__ x, const float* __restrict__ W_r,
     static_assert(NV == 32 || NV == 64, "register tile");
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int t0 = blockIdx.x * TT;
+    pdl_wait();
+    pdl_allow_next();
 
     if (tid == 0) {
         abort_s = 0;
@@ -381,6 +385,8 @@ router_select_kernel(const float* __restrict__ part, int ks, const float* __rest
     constexpr int NP = EPT * 32;
     constexpr int PER = TT * NP / SEL_THREADS;
     __shared__ float lg[TT * (NP + 1)];
+    pdl_wait();
+    pdl_allow_next();
     const int t0 = blockIdx.x * TT;
     const size_t plane = static_cast<size_t>(T) * E;
     float acc[PER];
@@ -416,6 +422,8 @@ router_select_kernel(const float* __restrict__ part, int ks, const float* __rest
 // thread when n allows, with the loads of four splits in flight at once.
 __global__ void __launch_bounds__(128)
 router_reduce_kernel(const float* __restrict__ part, int ks, size_t n, float* __restrict__ out) {
+    pdl_wait();
+    pdl_allow_next();
     const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
     const size_t i0 = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if ((n & 3) == 0) {
@@ -452,14 +460,15 @@ cudaError_t launch_generic(const Dims& dm, const void* x, const float* W_r, cons
                            cudaStream_t st) {
     const dim3 grid(dm.route_blocks), block(NTHREADS);
     const XT* xp = static_cast<const XT*>(x);
-#define MOE_GEN(EPT) router_generic_kernel<XT, EPT><<<grid, block, 0, st>>>(xp, W_r, bias, dm.T, dm.d, dm.E, dm.K, idx, gates, logits, psum, sel_bias)
+    cudaError_t e;
+#define MOE_GEN(EPT) e = launch_pdl(router_generic_kernel<XT, EPT>, grid, block, 0, st, 1, xp, W_r, bias, dm.T, dm.d, \
+                                    dm.E, dm.K, idx, gates, logits, psum, sel_bias)
     if (dm.E <= 32) MOE_GEN(1);
     else if (dm.E <= 64) MOE_GEN(2);
     else if (dm.E <= 128) MOE_GEN(4);
     else MOE_GEN(8);
 #undef MOE_GEN
-    count_launches();
-    return cudaGetLastError();
+    return e;
 }
 
 template <typename XT, int NE, int RT>
@@ -470,10 +479,9 @@ cudaError_t launch_small_t(const Dims& dm, const void* x, const float* W_r, cons
     cudaError_t e = cudaFuncSetAttribute(router_small_kernel<XT, NE, RT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    router_small_kernel<XT, NE, RT><<<dm.route_blocks, SmallCfg<NE, RT>::WARPS * 32, smem, st>>>(
-        static_cast<const XT*>(x), W_r, bias, dm.T, dm.d, dm.E, dm.K, idx, gates, logits, psum, status, sel_bias);
-    count_launches();
-    return cudaGetLastError();
+    return launch_pdl(router_small_kernel<XT, NE, RT>, dim3(dm.route_blocks), dim3(SmallCfg<NE, RT>::WARPS * 32), smem,
+                      st, 1, static_cast<const XT*>(x), W_r, bias, dm.T, dm.d, dm.E, dm.K, idx, gates, logits, psum,
+                      status, sel_bias);
 }
 
 template <typename XT>
@@ -523,22 +531,21 @@ cudaError_t launch_router(const Dims& dm, const void* x, const float* W_r, const
         const size_t items = (n & 3) == 0 ? n / 4 : n;
         int blocks = static_cast<int>((items + 127) / 128);
         if (blocks > 8 * 148) blocks = 8 * 148;
-        router_reduce_kernel<<<blocks, 128, 0, st>>>(rs.part, ks, n, rs.logits);
-        count_launches();
-        e = cudaGetLastError();
+        e = launch_pdl(router_reduce_kernel, dim3(blocks), dim3(128), 0, st, 1, static_cast<const float*>(rs.part), ks,
+                       n, rs.logits);
         if (e != cudaSuccess) return e;
         logits = rs.logits;
         ks = 1;
     }
     const dim3 grid(dm.route_blocks), block(SEL_THREADS);
-#define MOE_SEL(EPT) router_select_kernel<EPT><<<grid, block, 0, st>>>(logits, ks, logit_bias, dm.T, dm.E, dm.K, topk_idx, gates, logits_out, psum, sel_bias)
+#define MOE_SEL(EPT) e = launch_pdl(router_select_kernel<EPT>, grid, block, 0, st, 1, logits, ks, logit_bias, dm.T, \
+                                    dm.E, dm.K, topk_idx, gates, logits_out, psum, sel_bias)
     if (dm.E <= 32) MOE_SEL(1);
     else if (dm.E <= 64) MOE_SEL(2);
     else if (dm.E <= 128) MOE_SEL(4);
     else MOE_SEL(8);
 #undef MOE_SEL
-    count_launches();
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace moe

@@ -58,6 +58,8 @@ template <int BN> struct RCfg {
 // W_r 16-byte aligned): one 16-byte load, one 8-byte store per plane.
 __global__ void __launch_bounds__(256)
 router_split_kernel(const float* __restrict__ W_r, int d, __nv_bfloat16* __restrict__ w3) {
+    pdl_wait();
+    pdl_allow_next();
     const int j = blockIdx.y;
     const float4* src = reinterpret_cast<const float4*>(W_r + static_cast<size_t>(j) * d);
     __nv_bfloat16* row = w3 + static_cast<size_t>(j) * 3 * d;
@@ -123,6 +125,8 @@ router_tc_kernel(const __grid_constant__ RouterTcParams p) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();
+    pdl_allow_next();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -228,9 +232,7 @@ cudaError_t launch_bn(const Dims& dm, const RouterTcPlan& plan, const RouterTcPa
     static_assert(smem <= 227 * 1024, "shared memory budget");
     cudaError_t e = cudaFuncSetAttribute(router_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    router_tc_kernel<BN><<<dim3(plan.mt, plan.nt, plan.ksplit), RTHREADS, smem, st>>>(p);
-    count_launches();
-    return cudaGetLastError();
+    return launch_pdl(router_tc_kernel<BN>, dim3(plan.mt, plan.nt, plan.ksplit), dim3(RTHREADS), smem, st, 1, p);
 }
 
 }  // namespace
@@ -258,9 +260,8 @@ RouterTcPlan router_tc_plan(const Dims& dm) {
 cudaError_t launch_router_tc(const Dims& dm, const RouterTcPlan& plan, const void* x, const float* W_r,
                              void* w3, float* part, int32_t* status, cudaStream_t st) {
     const int col_blocks = (dm.d / 4 + 255) / 256;
-    router_split_kernel<<<dim3(col_blocks, dm.E), 256, 0, st>>>(W_r, dm.d, static_cast<__nv_bfloat16*>(w3));
-    count_launches();
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(router_split_kernel, dim3(col_blocks, dm.E), dim3(256), 0, st, 1, W_r, dm.d,
+                               static_cast<__nv_bfloat16*>(w3));
     if (e != cudaSuccess) return e;
     RouterTcParams p;
     std::memset(&p, 0, sizeof(p));
