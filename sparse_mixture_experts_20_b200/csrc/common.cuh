@@ -230,6 +230,16 @@ __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// tcgen05.wait::ld, then marks the registers of r as written here, so that no
+// use of a value loaded by tcgen05.ld can be scheduled before the wait (the
+// wait itself has no data dependence on them).
+template <int N>
+__device__ __forceinline__ void tmem_ld_wait_regs(uint32_t (&r)[N]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
 // Shared-memory matrix descriptor for a K-major operand tile stored in the
 // 128-byte-swizzled layout that TMA writes with CU_TENSOR_MAP_SWIZZLE_128B:
 // rows of 128 bytes, 8-row swizzle atoms 1024 bytes apart.  Fields: start

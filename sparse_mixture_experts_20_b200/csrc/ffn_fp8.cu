@@ -79,8 +79,15 @@ template <int BN_> struct FCfg {
     static constexpr int N_BARS = 2 * STAGES + 4 + 2;
     static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
     static constexpr int OFF_SEG = OFF_MISC + 16;
-    static constexpr int TOTAL = OFF_SEG + SegTable::SEG_INTS * 4;
+    // per epilogue warp, 2 x BN fp32: the biases of its two tiles in flight
+    // (read and written as float4: 16-byte aligned)
+    static constexpr int OFF_BIAS = (OFF_SEG + SegTable::SEG_INTS * 4 + 15) & ~15;
+    static constexpr int TOTAL = OFF_BIAS + 4 * 2 * BN * 4;
     static constexpr int ALLOC = TOTAL + 1024;
+    static_assert(OFF_BIAS % 16 == 0 && (BN * 4) % 16 == 0, "float4 access to the bias buffers");
+    static_assert(OFF_A % 1024 == 0 && OFF_B % 1024 == 0 && A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0,
+                  "128-byte-swizzled TMA tiles start on 1024-byte boundaries");
+    static_assert(OFF_BAR % 8 == 0, "mbarriers are 8-byte aligned");
 };
 
 // A positive power-of-two fp32 scale as a UE8M0 byte (its biased exponent),
@@ -223,6 +230,19 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
             const TileInfo ti = decode_tile<BN, BK>(tile, p, seg, nseg);
             const GroupDev& g = p.g[ti.grp];
             const bool row_ok = r_local < ti.rows_left;
+            // the tile's BN biases into this warp's shared-memory buffer while the
+            // tile's MMAs run (each warp keeps its own copy, so only the warp
+            // itself synchronises); the buffer of tile i is rewritten for tile
+            // i + 2, after this warp is done with tile i
+            float* bias_s = reinterpret_cast<float*>(smem + L::OFF_BIAS) + (quad * 2 + abuf) * BN;
+#pragma unroll
+            for (int i = 4 * lane; i < BN; i += 128) {
+                const float4 v = (ti.n0 + i < g.N)
+                    ? __ldg(reinterpret_cast<const float4*>(g.bias + static_cast<size_t>(ti.mat) * g.N + ti.n0 + i))
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                *reinterpret_cast<float4*>(bias_s + i) = v;
+            }
+            __syncwarp();
             uint32_t& fph = abuf ? fph1 : fph0;
             if (!warp_wait(&accf[abuf], fph, abort_flag, p.status, p.timeout_ns, lane)) break;
             fph ^= 1u;
@@ -230,7 +250,6 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
             // this tile's accumulator; its overlapping columns are 192..255 of
             // buffer 0 (the second half) or 0..63 of buffer 1 (the first half)
             const uint32_t acc = lane_base + (abuf ? L::ACC1_COL : 0u);
-            const float* bias = g.bias + static_cast<size_t>(ti.mat) * g.N + ti.n0;
             if (p.out_fp8) {
                 // first layer: bias + SiLU, then one e4m3 block per 128 columns
                 // per row; the half holding the overlap goes first
@@ -252,10 +271,10 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
                     const int n_blk = ti.n0 + h * 128;
                     if (!row_ok || n_blk >= g.N) continue;
                     float amax = 0.f;
-                    const float4* b4 = reinterpret_cast<const float4*>(bias + h * 128);
+                    const float4* b4 = reinterpret_cast<const float4*>(bias_s + h * 128);
 #pragma unroll
                     for (int j4 = 0; j4 < 32; ++j4) {
-                        const float4 b = __ldg(b4 + j4);
+                        const float4 b = b4[j4];
                         v[4 * j4 + 0] = silu_fast(v[4 * j4 + 0] + b.x);
                         v[4 * j4 + 1] = silu_fast(v[4 * j4 + 1] + b.y);
                         v[4 * j4 + 2] = silu_fast(v[4 * j4 + 2] + b.z);
@@ -281,40 +300,60 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
                     g.c_scales[static_cast<size_t>(ti.c_row + r_local) * (g.N / 128) + n_blk / 128] = sc;
                 }
             } else {
-                // second layer: bias, bf16 output; the two overlapping chunks first
+                // second layer: bias, bf16 output.  Chunks of 32 columns, the
+                // overlapping ones first; the tensor-memory load of the next
+                // chunk is in flight while a chunk is converted and stored.
                 __nv_bfloat16* crow = static_cast<__nv_bfloat16*>(g.C) +
                                       static_cast<size_t>(ti.c_row + r_local) * g.N + ti.n0;
                 const int n_valid = min(BN, g.N - ti.n0);
-#pragma unroll 1
-                for (int ci = 0; ci < BN / 32; ++ci) {
-                    const int c = (abuf || !L::OVERLAP) ? ci : (ci + 6) & 7;
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(acc + static_cast<uint32_t>(c * 32), r);
-                    tmem_ld_wait();
-                    if (L::OVERLAP && ci == 1) {                 // overlap read: the next tile may start
+                constexpr int NCH = BN / 32;
+                auto col_of = [&](int ci) { return (abuf || !L::OVERLAP) ? ci : (ci + 6) & 7; };
+                auto store_chunk = [&](const uint32_t (&r)[32], int c) {
+                    if (!row_ok || c * 32 >= n_valid) return;
+                    uint32_t packed[16];
+                    const float4* b4 = reinterpret_cast<const float4*>(bias_s + c * 32);
+#pragma unroll
+                    for (int j4 = 0; j4 < 8; ++j4) {
+                        const float4 b = b4[j4];
+                        __nv_bfloat162 lo = __floats2bfloat162_rn(__uint_as_float(r[4 * j4 + 0]) + b.x,
+                                                                  __uint_as_float(r[4 * j4 + 1]) + b.y);
+                        __nv_bfloat162 hi = __floats2bfloat162_rn(__uint_as_float(r[4 * j4 + 2]) + b.z,
+                                                                  __uint_as_float(r[4 * j4 + 3]) + b.w);
+                        packed[2 * j4] = *reinterpret_cast<uint32_t*>(&lo);
+                        packed[2 * j4 + 1] = *reinterpret_cast<uint32_t*>(&hi);
+                    }
+                    uint4* dst = reinterpret_cast<uint4*>(crow + c * 32);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+                };
+                // once chunk `loaded` is in registers: after the two overlapping
+                // chunks the next tile may start, after the last the
+                // accumulator is free
+                auto loaded = [&](int ci) {
+                    if (L::OVERLAP && ci == 1) {
                         tc_fence_before();
                         mbar_arrive(ovl);
-                    } else if (ci == BN / 32 - 1) {              // accumulator fully read: release it
+                    } else if (ci == NCH - 1) {
                         tc_fence_before();
                         mbar_arrive(&acce[abuf]);
                     }
-                    if (row_ok && c * 32 < n_valid) {
-                        uint32_t packed[16];
-                        const float4* b4 = reinterpret_cast<const float4*>(bias + c * 32);
-#pragma unroll
-                        for (int j4 = 0; j4 < 8; ++j4) {
-                            const float4 b = __ldg(b4 + j4);
-                            __nv_bfloat162 lo = __floats2bfloat162_rn(__uint_as_float(r[4 * j4 + 0]) + b.x,
-                                                                      __uint_as_float(r[4 * j4 + 1]) + b.y);
-                            __nv_bfloat162 hi = __floats2bfloat162_rn(__uint_as_float(r[4 * j4 + 2]) + b.z,
-                                                                      __uint_as_float(r[4 * j4 + 3]) + b.w);
-                            packed[2 * j4] = *reinterpret_cast<uint32_t*>(&lo);
-                            packed[2 * j4 + 1] = *reinterpret_cast<uint32_t*>(&hi);
-                        }
-                        uint4* dst = reinterpret_cast<uint4*>(crow + c * 32);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+                };
+                uint32_t r0[32], r1[32];
+                tmem_ld_32x32b_x32(acc + static_cast<uint32_t>(col_of(0) * 32), r0);
+                tmem_ld_wait_regs(r0);
+                loaded(0);
+#pragma unroll 1
+                for (int ci = 0; ci < NCH; ci += 2) {
+                    tmem_ld_32x32b_x32(acc + static_cast<uint32_t>(col_of(ci + 1) * 32), r1);
+                    store_chunk(r0, col_of(ci));
+                    tmem_ld_wait_regs(r1);
+                    loaded(ci + 1);
+                    if (ci + 2 < NCH) tmem_ld_32x32b_x32(acc + static_cast<uint32_t>(col_of(ci + 2) * 32), r0);
+                    store_chunk(r1, col_of(ci + 1));
+                    if (ci + 2 < NCH) {
+                        tmem_ld_wait_regs(r0);
+                        loaded(ci + 2);
                     }
                 }
             }
@@ -419,15 +458,12 @@ cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
 
 }  // namespace
 
-// Weight tiles 128 wide when the batch averages fewer than 64 rows per
-// routed expert (decode-like: every tile streams its weights once and the
-// tile count sets the balance over the SMs), else 256 wide.
-int fp8_weight_tile(const Dims& dm) {
-    return static_cast<long long>(dm.T) * dm.K < 64LL * dm.E ? 128 : 256;
-}
-
-cudaError_t launch_grouped_ffn_fp8(const Dims& dm, const GemmArgs& a, cudaStream_t st) {
-    return fp8_weight_tile(dm) == 128 ? launch_bn<128>(a, st) : launch_bn<256>(a, st);
+// Weight tiles are 256 wide.  128-wide tiles (FCfg<128>) double the tile
+// count on decode-sized batches, which evens out the last wave, but measured
+// slower on the V3 decode batch (0.293 against 0.269 ms): the per-stage cost
+// of the block-scaled MMA is nearly the same at N = 128 as at N = 256.
+cudaError_t launch_grouped_ffn_fp8(const Dims&, const GemmArgs& a, cudaStream_t st) {
+    return launch_bn<256>(a, st);
 }
 
 }  // namespace moe

@@ -81,9 +81,9 @@ struct RouterScratch {
 };
 
 // Tile plan of the tensor-core router: m-tiles of 128 tokens, nt tiles of bn
-// experts, ksplit splits of K = 3 d.
+// experts, ksplit splits of K = 3 d; pair: m-tiles two at a time on CTA pairs.
 struct RouterTcPlan {
-    int mt, nt, bn, ksplit;
+    int mt, nt, bn, ksplit, pair;
 };
 
 bool router_uses_small(const Dims& dm);
@@ -143,8 +143,6 @@ cudaError_t launch_grouped_ffn_bf16_pair(const Dims& dm, const GemmArgs& a, cuda
 // CTA-pair kernels are used unless the environment variable MOE_GEMM_PAIR is "0".
 bool gemm_pairs_enabled();
 cudaError_t launch_grouped_ffn_fp8(const Dims& dm, const GemmArgs& a, cudaStream_t st);
-// Weight-tile width (128 or 256) the FP8 grouped GEMM uses for this shape.
-int fp8_weight_tile(const Dims& dm);
 
 cudaError_t launch_wait_selftest(int64_t timeout_ns, int32_t* status, cudaStream_t st);
 

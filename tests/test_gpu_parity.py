@@ -30,6 +30,11 @@ CASES = {
     "bf16-e24-small-router": MoEShape("b7", 300, 256, 24, 3, 256, dtype=DTYPE_BF16),
     "bf16-e128-tc-router": MoEShape("b8", 600, 256, 128, 4, 128, n_shared=1, d_ff_shared=128,
                                     dtype=DTYPE_BF16),
+    # tensor-core router on CTA pairs with a 128-wide expert tile (nine token
+    # tiles: the last pair has one), and with 8 experts too wide for the
+    # shared-memory router (d = 5632) in a 64-wide tile padded with zero rows
+    "bf16-e128-pair-router": MoEShape("b9", 1100, 256, 128, 4, 128, dtype=DTYPE_BF16),
+    "bf16-e8-wide-pair-router": MoEShape("b10", 300, 5632, 8, 2, 128, dtype=DTYPE_BF16),
     "fp8-ragged-shared": MoEShape("f1", 300, 512, 16, 4, 256, n_shared=1, d_ff_shared=384, dtype=DTYPE_FP8),
     "fp8-decode-skewed": MoEShape("f2", 37, 1024, 256, 8, 256, n_shared=1, d_ff_shared=256,
                                   dtype=DTYPE_FP8, zipf_logit_bias=True),
