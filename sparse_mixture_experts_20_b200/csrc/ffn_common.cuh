@@ -38,6 +38,7 @@ struct GroupDev {
 struct __align__(64) TcParams {
     CUtensorMap a_map[2];
     CUtensorMap b_map[2];
+    CUtensorMap c_map[2];     // outputs, for TMA stores (FP8 engine)
     GroupDev g[2];
     int silu;
     int out_fp8;
@@ -151,8 +152,10 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // Host: fills the parameter block of both groups; elem = operand bytes,
-// bn = weight rows per tile.  Returns false if a tensor map cannot be encoded.
-inline bool fill_params(TcParams& p, const GemmArgs& a, int elem, int bn, uint64_t timeout_ns) {
+// bn = weight rows per tile, out_elem > 0: also the output maps for TMA
+// stores of 64-byte x 32-row boxes (out_elem = output element bytes).
+// Returns false if a tensor map cannot be encoded.
+inline bool fill_params(TcParams& p, const GemmArgs& a, int elem, int bn, uint64_t timeout_ns, int out_elem = 0) {
     std::memset(&p, 0, sizeof(p));
     for (int gi = 0; gi < 2; ++gi) {
         const GemmGroup& g = a.g[gi];
@@ -174,6 +177,7 @@ inline bool fill_params(TcParams& p, const GemmArgs& a, int elem, int bn, uint64
         d.a_rows = g.a_rows;
         if (!encode_tma_2d(&p.a_map[gi], g.A, g.a_rows, g.K, elem, BM)) return false;
         if (!encode_tma_3d(&p.b_map[gi], g.B, g.n_mats, g.N, g.K, elem, bn)) return false;
+        if (out_elem > 0 && !encode_tma_2d_store64(&p.c_map[gi], g.C, g.c_rows, g.N, out_elem, 32)) return false;
     }
     p.silu = a.silu;
     p.out_fp8 = a.out_fp8;

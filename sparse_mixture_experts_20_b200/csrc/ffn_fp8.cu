@@ -82,12 +82,17 @@ template <int BN_> struct FCfg {
     // per epilogue warp, 2 x BN fp32: the biases of its two tiles in flight
     // (read and written as float4: 16-byte aligned)
     static constexpr int OFF_BIAS = (OFF_SEG + SegTable::SEG_INTS * 4 + 15) & ~15;
-    static constexpr int TOTAL = OFF_BIAS + 4 * 2 * BN * 4;
+    // per epilogue warp, two 2 KB staging buffers (32 rows x 64 bytes, 64-byte
+    // swizzled) for the TMA stores of its output rows
+    static constexpr int OFF_STAGE = (OFF_BIAS + 4 * 2 * BN * 4 + 1023) & ~1023;
+    static constexpr int STAGE_BUF = 32 * 64;
+    static constexpr int TOTAL = OFF_STAGE + 4 * 2 * STAGE_BUF;
     static constexpr int ALLOC = TOTAL + 1024;
     static_assert(OFF_BIAS % 16 == 0 && (BN * 4) % 16 == 0, "float4 access to the bias buffers");
     static_assert(OFF_A % 1024 == 0 && OFF_B % 1024 == 0 && A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0,
                   "128-byte-swizzled TMA tiles start on 1024-byte boundaries");
     static_assert(OFF_BAR % 8 == 0, "mbarriers are 8-byte aligned");
+    static_assert(OFF_STAGE % 1024 == 0, "64-byte-swizzled TMA boxes start on 512-byte boundaries");
 };
 
 // A positive power-of-two fp32 scale as a UE8M0 byte (its biased exponent),
@@ -101,7 +106,10 @@ struct ItemIt {
     TileInfo ti;
 };
 
-template <int BN>
+// OUT_FP8: the first layer (bias, SiLU, e4m3 re-quantisation of h) or the
+// second (bias, bf16 y); one instance each, so that neither carries the
+// other's registers and code.
+template <int BN, bool OUT_FP8>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
     using L = FCfg<BN>;
@@ -226,10 +234,40 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
         int abuf = 0;
         uint32_t fph0 = 0, fph1 = 0;
+        // Output rows leave through shared memory and TMA stores: the warp
+        // writes its 32 rows x 64 bytes into one of its two staging buffers
+        // (16-byte chunk q of row r at chunk q ^ ((r >> 1) & 3): the 64-byte
+        // swizzle, which also spreads the writes over the banks) and one lane
+        // stores the box.  A buffer is rewritten only after the store issued
+        // from it two boxes earlier has read it.
+        uint8_t* stg = smem + L::OFF_STAGE + quad * 2 * L::STAGE_BUF;
+        int sbuf = 0;
+        // the warp's next staging buffer, free to write; this lane's row in it
+        auto stage_begin = [&]() -> uint8_t* {
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+            return stg + sbuf * L::STAGE_BUF + lane * 64;
+        };
+        auto stage_put = [&](uint8_t* row, int q, const uint4& v) {
+            *reinterpret_cast<uint4*>(row + ((q ^ ((lane >> 1) & 3)) << 4)) = v;
+        };
+        auto stage_end = [&](const void* map, int x, int y) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_2d(map, stg + sbuf * L::STAGE_BUF, x, y);
+                bulk_commit();
+            }
+            sbuf ^= 1;
+        };
         for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
             const TileInfo ti = decode_tile<BN, BK>(tile, p, seg, nseg);
             const GroupDev& g = p.g[ti.grp];
             const bool row_ok = r_local < ti.rows_left;
+            // all 32 rows of this warp lie in the segment: TMA stores; else the
+            // valid rows are stored one by one (a box would reach into the
+            // next segment's rows)
+            const bool full_warp = ti.rows_left >= quad * 32 + 32;
             // the tile's BN biases into this warp's shared-memory buffer while the
             // tile's MMAs run (each warp keeps its own copy, so only the warp
             // itself synchronises); the buffer of tile i is rewritten for tile
@@ -250,7 +288,7 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
             // this tile's accumulator; its overlapping columns are 192..255 of
             // buffer 0 (the second half) or 0..63 of buffer 1 (the first half)
             const uint32_t acc = lane_base + (abuf ? L::ACC1_COL : 0u);
-            if (p.out_fp8) {
+            if constexpr (OUT_FP8) {
                 // first layer: bias + SiLU, then one e4m3 block per 128 columns
                 // per row; the half holding the overlap goes first
 #pragma unroll 1
@@ -286,16 +324,24 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
                     const float inv = inv_pow2(sc);          // exact: sc is a power of two
                     uint8_t* crow = static_cast<uint8_t*>(g.C) + static_cast<size_t>(ti.c_row + r_local) * g.N + n_blk;
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        uint32_t w[4];
+                    for (int sub = 0; sub < 2; ++sub) {            // 64 columns (64 bytes) at a time
+                        uint8_t* srow = full_warp ? stage_begin() : nullptr;
 #pragma unroll
-                        for (int hh = 0; hh < 4; ++hh) {
-                            const int j = q * 16 + hh * 4;
-                            const uint32_t lo = f32x2_to_e4m3x2(v[j] * inv, v[j + 1] * inv);
-                            const uint32_t hi = f32x2_to_e4m3x2(v[j + 2] * inv, v[j + 3] * inv);
-                            w[hh] = lo | (hi << 16);
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            const int q = sub * 4 + q4;
+                            uint32_t w[4];
+#pragma unroll
+                            for (int hh = 0; hh < 4; ++hh) {
+                                const int j = q * 16 + hh * 4;
+                                const uint32_t lo = f32x2_to_e4m3x2(v[j] * inv, v[j + 1] * inv);
+                                const uint32_t hi = f32x2_to_e4m3x2(v[j + 2] * inv, v[j + 3] * inv);
+                                w[hh] = lo | (hi << 16);
+                            }
+                            const uint4 val = make_uint4(w[0], w[1], w[2], w[3]);
+                            if (full_warp) stage_put(srow, q4, val);
+                            else reinterpret_cast<uint4*>(crow)[q] = val;
                         }
-                        reinterpret_cast<uint4*>(crow)[q] = make_uint4(w[0], w[1], w[2], w[3]);
+                        if (full_warp) stage_end(&p.c_map[ti.grp], n_blk + 64 * sub, ti.c_row + quad * 32);
                     }
                     g.c_scales[static_cast<size_t>(ti.c_row + r_local) * (g.N / 128) + n_blk / 128] = sc;
                 }
@@ -309,7 +355,7 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
                 constexpr int NCH = BN / 32;
                 auto col_of = [&](int ci) { return (abuf || !L::OVERLAP) ? ci : (ci + 6) & 7; };
                 auto store_chunk = [&](const uint32_t (&r)[32], int c) {
-                    if (!row_ok || c * 32 >= n_valid) return;
+                    if (c * 32 >= n_valid || !(full_warp || row_ok)) return;
                     uint32_t packed[16];
                     const float4* b4 = reinterpret_cast<const float4*>(bias_s + c * 32);
 #pragma unroll
@@ -322,10 +368,19 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
                         packed[2 * j4] = *reinterpret_cast<uint32_t*>(&lo);
                         packed[2 * j4 + 1] = *reinterpret_cast<uint32_t*>(&hi);
                     }
-                    uint4* dst = reinterpret_cast<uint4*>(crow + c * 32);
+                    if (full_warp) {
+                        uint8_t* srow = stage_begin();
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+                        for (int q = 0; q < 4; ++q)
+                            stage_put(srow, q, make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2],
+                                                          packed[4 * q + 3]));
+                        stage_end(&p.c_map[ti.grp], ti.n0 + c * 32, ti.c_row + quad * 32);
+                    } else {
+                        uint4* dst = reinterpret_cast<uint4*>(crow + c * 32);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+                    }
                 };
                 // once chunk `loaded` is in registers: after the two overlapping
                 // chunks the next tile may start, after the last the
@@ -359,6 +414,9 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
             }
             abuf ^= 1;
         }
+        // the stores have read their buffers and landed before the CTA exits
+        if (lane == 0) bulk_wait<0>();
+        __syncwarp();
     } else {
         // ================= scale-factor writers (warps 6..9)
         const int quad = warp & 3;
@@ -401,39 +459,41 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
         for (int j = 0; j < LOOKAHEAD; ++j) {
             if (valid(ahead)) { load(ahead, ra[j], rb[j]); advance(ahead); }
         }
-        // Item i of the stream uses stage i % STAGES and ring slot i % LOOKAHEAD,
-        // the same index: the loop is unrolled over one turn of the ring, so a
-        // slot's scales (loaded LOOKAHEAD items earlier) are converted and the
-        // slot reloaded in place, with no register moves that would wait on a
-        // load still in flight.
-        static_assert(STAGES == LOOKAHEAD, "one ring slot per stage");
+        // Item i of the stream uses ring slot i % LOOKAHEAD and stage
+        // i % STAGES; LOOKAHEAD is a multiple of STAGES and the loop is
+        // unrolled over one turn of the ring, so both indices are constants:
+        // a slot's scales (loaded LOOKAHEAD items earlier) are converted and
+        // the slot reloaded in place, with no register moves that would wait
+        // on a load still in flight.
+        static_assert(LOOKAHEAD % STAGES == 0, "a turn of the ring is whole turns of the stages");
         uint32_t phase = 0;
         bool aborted = false;
 #pragma unroll 1
         while (valid(cur) && !aborted) {
 #pragma unroll
             for (int j = 0; j < LOOKAHEAD; ++j) {
+                const int stage = j % STAGES;
                 if (!valid(cur)) break;
                 const uint32_t wa0 = ue8m0_x4(ra[j][0]), wa1 = ue8m0_x4(ra[j][1]);
                 const uint32_t wa2 = ue8m0_x4(ra[j][2]), wa3 = ue8m0_x4(ra[j][3]);
                 const uint32_t wb0 = ue8m0_x4(rb[j][0]), wb1 = ue8m0_x4(rb[j][1]);
                 if (valid(ahead)) { load(ahead, ra[j], rb[j]); advance(ahead); }
-                if (!warp_wait(&empty[j], phase ^ 1u, abort_flag, p.status, p.timeout_ns, lane)) {
+                if (!warp_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, p.timeout_ns, lane)) {
                     aborted = true;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t slot = sf_base + static_cast<uint32_t>(j) * SF_STRIDE;
+                const uint32_t slot = sf_base + static_cast<uint32_t>(stage) * SF_STRIDE;
                 tmem_st_32x32b_x4(slot, wa0, wa1, wa2, wa3);
                 tmem_st_32x32b_x4(slot + 4, wb0, wb0, wb0, wb0);
                 if (BN == 256) tmem_st_32x32b_x4(slot + 8, wb1, wb1, wb1, wb1);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&full[j]);
+                if (lane == 0) mbar_arrive(&full[stage]);
+                if (stage == STAGES - 1) phase ^= 1u;
                 advance(cur);
             }
-            phase ^= 1u;
         }
     }
 
@@ -445,15 +505,16 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
     }
 }
 
-template <int BN>
+template <int BN, bool OUT_FP8>
 cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
     TcParams p;
-    if (!fill_params(p, a, 1, BN, kWaitTimeoutNs)) return cudaErrorInvalidValue;
+    if (!fill_params(p, a, 1, BN, kWaitTimeoutNs, OUT_FP8 ? 1 : 2)) return cudaErrorInvalidValue;
     constexpr int smem = FCfg<BN>::ALLOC;
     static_assert(smem <= 227 * 1024, "shared memory budget");
-    cudaError_t e = cudaFuncSetAttribute(grouped_ffn_fp8_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    auto kernel = grouped_ffn_fp8_kernel<BN, OUT_FP8>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(grouped_ffn_fp8_kernel<BN>, dim3(device_sm_count()), dim3(NUM_THREADS), smem, st, 1, p);
+    return launch_pdl(kernel, dim3(device_sm_count()), dim3(NUM_THREADS), smem, st, 1, p);
 }
 
 }  // namespace
@@ -463,7 +524,7 @@ cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
 // slower on the V3 decode batch (0.293 against 0.269 ms): the per-stage cost
 // of the block-scaled MMA is nearly the same at N = 128 as at N = 256.
 cudaError_t launch_grouped_ffn_fp8(const Dims&, const GemmArgs& a, cudaStream_t st) {
-    return launch_bn<256>(a, st);
+    return a.out_fp8 ? launch_bn<256, true>(a, st) : launch_bn<256, false>(a, st);
 }
 
 }  // namespace moe
