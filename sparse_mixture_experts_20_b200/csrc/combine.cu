@@ -10,8 +10,9 @@
 // output row, gathers the token's kept expert rows (loads issued together,
 // accumulated in ascending k) with 16-byte loads, accumulates g * y in fp32,
 // adds the shared experts' rows (ascending s) and rounds once.
-// balance_kernel: one block; chunked sums in a fixed order, so f, P and the
-// loss are bit-reproducible.
+// balance_kernel: one block running balance_block (balance.cuh): chunked sums
+// in a fixed order, so f, P and the loss are bit-reproducible.
+#include "balance.cuh"
 #include "common.cuh"
 #include "internal.h"
 
@@ -128,59 +129,15 @@ combine_kernel(const void* __restrict__ y_, const float* __restrict__ gates,
     }
 }
 
-// One block of 1024 threads.  Thread (c, j) = (tid / E, tid % E) sums the
-// per-block partial sums of s of expert j over its chunk c of the router
-// blocks, eight loads in flight at a time; the C chunk sums of each expert
-// are then added in chunk order and the products f_j P_j in a fixed tree, so
-// f, P and the loss are bit-reproducible.
-constexpr int BAL_THREADS = 1024;
-
-__global__ void __launch_bounds__(BAL_THREADS)
+__global__ void __launch_bounds__(BALANCE_THREADS)
 balance_kernel(const int32_t* __restrict__ counts, const float* __restrict__ psum, int blocks,
                int T, int E, int K, float alpha, float* __restrict__ f, float* __restrict__ P,
                float* __restrict__ loss) {
-    __shared__ float part[BAL_THREADS];
+    __shared__ float part[BALANCE_THREADS];
     __shared__ float fp[256];
     pdl_wait();
     pdl_allow_next();
-    const int tid = threadIdx.x;
-    const int C = BAL_THREADS / E;                       // >= 4: E <= 256
-    const int c = tid / E, j = tid - c * E;
-    if (c < C) {
-        const int b0 = static_cast<int>(static_cast<long long>(c) * blocks / C);
-        const int b1 = static_cast<int>(static_cast<long long>(c + 1) * blocks / C);
-        float s = 0.f;
-        int b = b0;
-        for (; b + 8 <= b1; b += 8) {
-            float v[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = __ldg(psum + static_cast<size_t>(b + u) * E + j);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) s += v[u];
-        }
-        for (; b < b1; ++b) s += __ldg(psum + static_cast<size_t>(b) * E + j);
-        part[tid] = s;
-    }
-    __syncthreads();
-    if (tid < 256) {
-        float prod = 0.f;
-        if (tid < E) {
-            float s = 0.f;
-            for (int q = 0; q < C; ++q) s += part[q * E + tid];
-            const float fj = static_cast<float>(counts[tid]) / static_cast<float>(T * K);
-            const float pj = s / static_cast<float>(T);
-            f[tid] = fj;
-            P[tid] = pj;
-            prod = fj * pj;
-        }
-        fp[tid] = prod;
-    }
-    __syncthreads();
-    for (int w = 128; w > 0; w >>= 1) {
-        if (tid < w) fp[tid] += fp[tid + w];
-        __syncthreads();
-    }
-    if (tid == 0) *loss = alpha * static_cast<float>(E) * fp[0];
+    balance_block(counts, psum, blocks, T, E, K, alpha, f, P, loss, part, fp);
 }
 
 }  // namespace
@@ -209,7 +166,7 @@ cudaError_t launch_combine(const Dims& dm, const void* y, const float* gates,
 
 cudaError_t launch_balance(const Dims& dm, const int32_t* counts, const float* psum,
                            float* f, float* P, float* loss, cudaStream_t st) {
-    return launch_pdl(balance_kernel, dim3(1), dim3(BAL_THREADS), 0, st, 1, counts, psum, dm.route_blocks, dm.T, dm.E,
+    return launch_pdl(balance_kernel, dim3(1), dim3(BALANCE_THREADS), 0, st, 1, counts, psum, dm.route_blocks, dm.T, dm.E,
                       dm.K, dm.alpha, f, P, loss);
 }
 

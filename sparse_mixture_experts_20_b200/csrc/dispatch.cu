@@ -22,6 +22,7 @@
 //      writes slot_row / row_slot; then the warp copies (bf16/fp32) or
 //      quantises to e4m3 (FP8) the token's row into each kept destination
 //      with 16-byte accesses.
+#include "balance.cuh"
 #include "common.cuh"
 #include "internal.h"
 
@@ -96,10 +97,13 @@ bitmap_kernel(const int32_t* __restrict__ topk_idx, int T, int E, int K, int t_w
 // written; and an exclusive scan of kept over the experts for the offsets.
 constexpr int SCAN_CACHE = 32;
 
+// With bal.f non-null the block then computes the balance statistics of the
+// batch as well (balance_block: the same arithmetic as the balance kernel),
+// which saves moe_layer_forward that kernel.
 __global__ void __launch_bounds__(1024)
 scan_kernel(const uint32_t* __restrict__ bitmap, int E, int n_words, int capacity,
             int32_t* __restrict__ word_base, int32_t* __restrict__ counts,
-            int32_t* __restrict__ kept, int32_t* __restrict__ offsets) {
+            int32_t* __restrict__ kept, int32_t* __restrict__ offsets, BalanceArgs bal) {
     __shared__ int part[1024];
     __shared__ int kept_s[256];
     pdl_wait();
@@ -182,6 +186,11 @@ scan_kernel(const uint32_t* __restrict__ bitmap, int E, int n_words, int capacit
         kept[tid] = kv;
         offsets[tid] = incl - kv;
         if (tid == E - 1) offsets[E] = incl;
+    }
+    if (bal.f != nullptr) {
+        __syncthreads();                                   // counts written, kept_s and part free
+        balance_block(counts, bal.psum, bal.blocks, bal.T, E, bal.K, bal.alpha, bal.f, bal.P, bal.loss,
+                      reinterpret_cast<float*>(part), reinterpret_cast<float*>(kept_s));
     }
 }
 
@@ -326,7 +335,7 @@ cudaError_t launch_dispatch(const Dims& dm, const void* x, const int32_t* topk_i
                             int32_t* counts, int32_t* kept, int32_t* offsets,
                             int32_t* slot_row, int32_t* row_slot, void* x_disp,
                             float* x_disp_scales, uint32_t* bitmap, int32_t* word_base,
-                            int32_t* status, cudaStream_t st) {
+                            int32_t* status, cudaStream_t st, const BalanceArgs* bal) {
     // warps per block: up to 8, with at most 32 KB of masks in shared memory
     const int words = dm.planes * dm.E;
     int wpb = 8;
@@ -337,8 +346,9 @@ cudaError_t launch_dispatch(const Dims& dm, const void* x, const int32_t* topk_i
     if (e != cudaSuccess) return e;
     // the scan runs over the (plane, word) sequence: token order within a
     // plane, planes in slot order
+    BalanceArgs none{};
     e = launch_pdl(scan_kernel, dim3(1), dim3(1024), 0, st, 1, bitmap, dm.E, dm.planes * dm.t_words, dm.capacity,
-                   word_base, counts, kept, offsets);
+                   word_base, counts, kept, offsets, bal ? *bal : none);
     if (e != cudaSuccess) return e;
     const int shared_copy = (dm.dtype == MOE_FP8_E4M3_BLOCK && dm.S > 0) ? 1 : 0;
     // warps per token: enough warps in flight to fill the GPU at small T

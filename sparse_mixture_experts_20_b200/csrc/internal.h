@@ -96,11 +96,22 @@ cudaError_t launch_router(const Dims& dm, const void* x, const float* W_r, const
                           int32_t* topk_idx, float* gates, float* logits_out, float* psum,
                           const RouterScratch& rs, cudaStream_t st);
 
+// Balance statistics computed by the dispatch scan (moe_layer_forward): the
+// router's per-block partial sums of s and the outputs; f == nullptr: none.
+struct BalanceArgs {
+    const float* psum;
+    int blocks, T, K;
+    float alpha;
+    float* f;
+    float* P;
+    float* loss;
+};
+
 cudaError_t launch_dispatch(const Dims& dm, const void* x, const int32_t* topk_idx,
                             int32_t* counts, int32_t* kept, int32_t* offsets,
                             int32_t* slot_row, int32_t* row_slot, void* x_disp,
                             float* x_disp_scales, uint32_t* bitmap, int32_t* word_base,
-                            int32_t* status, cudaStream_t st);
+                            int32_t* status, cudaStream_t st, const BalanceArgs* bal = nullptr);
 
 cudaError_t launch_combine(const Dims& dm, const void* y, const float* gates,
                            const int32_t* slot_row, const void* x, void* out, cudaStream_t st);

@@ -444,16 +444,17 @@ int moe_layer_forward(const moe_config* cfg, const void* x, const float* W_r, co
     cudaError_t e = launch_router(dm, x, W_r, logit_bias, idx, g, nullptr, at<float>(ws, L.psum),
                                   router_scratch(ws, L), st);
     if (e != cudaSuccess) return cuda_status(e);
+    // the balance statistics come out of the dispatch scan (same arithmetic
+    // as moe_balance_stats, one kernel fewer)
+    const BalanceArgs bal{at<float>(ws, L.psum), dm.route_blocks, dm.T, dm.K, dm.alpha, f, P, loss};
     e = launch_dispatch(dm, x, idx, cnt, at<int32_t>(ws, L.kept), offsets, slot_row, at<int32_t>(ws, L.row_slot),
                         x_disp, x_disp_sc, at<uint32_t>(ws, L.bitmap), at<int32_t>(ws, L.word_base),
-                        at<int32_t>(ws, L.status), st);
+                        at<int32_t>(ws, L.status), st, &bal);
     if (e != cudaSuccess) return cuda_status(e);
     const int r = run_expert_ffn(dm, L, x, x_disp, x_disp_sc, offsets, W1, W1_scales, b1, W2, W2_scales, b2,
                                  Ws1, Ws1_scales, bs1, Ws2, Ws2_scales, bs2, y, ws, st);
     if (r != MOE_OK) return r;
-    e = launch_combine(dm, y, g, slot_row, x, out, st);
-    if (e != cudaSuccess) return cuda_status(e);
-    return cuda_status(launch_balance(dm, cnt, at<float>(ws, L.psum), f, P, loss, st));
+    return cuda_status(launch_combine(dm, y, g, slot_row, x, out, st));
 }
 
 int moe_backward_workspace_size(const moe_config* cfg, size_t* bytes) {

@@ -426,13 +426,12 @@ RouterTcPlan router_tc_plan(const Dims& dm) {
     }
     pl.nt = (dm.E + pl.bn - 1) / pl.bn;
     // CTA pairs once there are two token tiles to pair (an odd last tile is
-    // paired with a tile of zero rows past T); a pair tile is at least 64
-    // experts wide (rows past N_r read as zeros)
-    pl.pair = pl.mt >= 2 ? 1 : 0;
-    if (pl.pair && pl.bn < 64) {
-        pl.bn = 64;
-        pl.nt = (dm.E + pl.bn - 1) / pl.bn;
-    }
+    // paired with a tile of zero rows past T) and the expert tile is at least
+    // 128 wide
+    // (the pair halves the plane bytes a CTA stages, which is what fills a
+    // stage once the expert tile is 128 wide or more; with narrower tiles the
+    // x block dominates and single CTAs measured faster)
+    pl.pair = (pl.mt >= 2 && pl.bn >= 128) ? 1 : 0;
     const int ctas_per_split = (pl.pair ? 2 * ((pl.mt + 1) / 2) : pl.mt) * pl.nt;
     int ks = target / ctas_per_split;
     if (ks < 1) ks = 1;
@@ -461,11 +460,7 @@ cudaError_t launch_router_tc(const Dims& dm, const RouterTcPlan& plan, const voi
     p.timeout_ns = kRouterWaitNs;
     if (plan.pair) {
         if (!encode_tma_2d(&p.b_map, w3, dm.E, 3 * dm.d, 2, plan.bn / 2)) return cudaErrorInvalidValue;
-        switch (plan.bn) {
-            case 64: return launch_bn2<64>(plan, p, st);
-            case 128: return launch_bn2<128>(plan, p, st);
-            default: return launch_bn2<256>(plan, p, st);
-        }
+        return plan.bn == 128 ? launch_bn2<128>(plan, p, st) : launch_bn2<256>(plan, p, st);
     }
     switch (plan.bn) {
         case 32: return launch_bn<32>(dm, plan, p, st);
