@@ -321,7 +321,10 @@ MOE_EXPORT int moe_dispatch_noalloc(const moe_config* cfg, const void* x, const 
  *     z = W1 x + b1 is recomputed; dz = (W2^T dy) * SiLU'(z); dW2 = dy SiLU(z)^T,
  *     dW1 = dz x^T, db1 / db2 the sums of dz / dy; dx gets W1^T dz of each
  *     kept slot, and g * dout_t of each slot dropped with pass-through.
- * MOE_FP8_E4M3_BLOCK returns MOE_ERR_UNSUPPORTED.  Every reduction runs in a
+ * MOE_FP8_E4M3_BLOCK returns MOE_ERR_UNSUPPORTED.  bf16 layers run every
+ * expert GEMM (the recompute of z, dh, dx, dW1, dW2) on the tensor cores with
+ * fp32 accumulation over bf16 copies of dy = g * dout, SiLU(z), SiLU'(z) and
+ * dz; fp32 layers run fp32 arithmetic throughout.  Every reduction runs in a
  * fixed order (bit-reproducible).  Inputs are the forward's inputs and the
  * results of its stages on the same batch; outputs are fp32 and written in
  * full (experts no slot reached get zero gradients).  All pointers are device
@@ -370,7 +373,11 @@ MOE_EXPORT int moe_backward_workspace_size(const moe_config* cfg, size_t* bytes)
 
 /* Enqueues the backward on `stream`.  lam: weight of the balance loss in J
  * (finite).  bws: caller scratch of moe_backward_workspace_size() bytes,
- * 256-byte aligned, any contents (fully rewritten before it is read). */
+ * 256-byte aligned, any contents (fully rewritten before it is read).  The
+ * first 4 bytes of bws receive this call's device status word (0, or
+ * MOE_DEV_TIMEOUT when a bounded wait of a tensor-core kernel gave up, the
+ * gradients then being incomplete); moe_get_device_status(cfg, bws, ...)
+ * reads it like a forward workspace's. */
 MOE_EXPORT int moe_layer_backward(const moe_config* cfg, float lam, const moe_backward_io* io,
                                   void* bws, void* stream);
 

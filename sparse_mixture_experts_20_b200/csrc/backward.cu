@@ -1,5 +1,31 @@
-// GPU executor of the layer backward: each step of bwd::run_backward runs as
-// one grid-stride kernel of 256 threads, one output element per iteration.
+// GPU executor of the layer backward.
+//
+// fp32 layers: each step of bwd::run_backward (backward.cuh) runs as one
+// grid-stride kernel of 256 threads, one output element per iteration.
+//
+// bf16 layers: the router and gate steps are the same fixed-order functors
+// (the gate gradients one warp per slot); every expert GEMM runs on the
+// tensor cores (bwd_gemm.cu) over padded row segments:
+//   1. poff: each routed expert's row count rounded up to 16, scanned;
+//   2. padded rows: x_p[pr] = x_disp[r], dy_p[pr] = g * dout[t] (bf16), zero
+//      rows in each expert's padding;
+//   3. recompute  z = x_p W1^T + b1          -> SiLU(z), SiLU'(z)  (bf16)
+//   4. dgrad      dz = (dy_p W2) * SiLU'(z)  -> bf16
+//   5. dgrad      dx rows = dz W1            -> fp32
+//   6. wgrad      dW2 = dy_p^T SiLU(z), dW1 = dz^T x_p (fp32, contraction
+//      over each expert's padded rows; the padding rows are zero in dy_p and
+//      dz, so they add nothing)
+//   shared experts in the same launches (rows = the T tokens, dy = dout; the
+//   shared hidden activations of all shared experts side by side in one
+//   (T, n_shared * d_ff_shared) matrix, so dx and dW1 of all shared experts
+//   are one GEMM each);
+//   7. bias gradients: column sums in two fixed-order passes (16-row chunk
+//      partials, then the chunks of each segment in order);
+//   8. dx = router part + shared part + the kept slots' rows (+ g * dout for
+//      slots passed through).
+// Every reduction has a fixed order: the result is bit-reproducible.
+#include <algorithm>
+#include <cstring>
 #include "backward.cuh"
 
 namespace moe {
@@ -16,23 +42,441 @@ struct GpuExec {
     cudaStream_t st;
     cudaError_t err;
     int launches;
+    int max_blocks;
     template <class F> void run(size_t n, const F& f) {
         if (err != cudaSuccess || n == 0) return;
         size_t blocks = (n + 255) / 256;
-        if (blocks > 148 * 16) blocks = 148 * 16;       // 16 blocks per SM, then the loop strides
+        if (blocks > static_cast<size_t>(max_blocks)) blocks = max_blocks;   // then the loop strides
         for_each_kernel<F><<<static_cast<unsigned>(blocks), 256, 0, st>>>(n, f);
         ++launches;
         err = cudaGetLastError();
     }
 };
 
+// ------------------------------------------------------------ bf16 path
+
+// a[slot] = <dout_t, y_row> (kept), <dout_t, x_t> (passed through), else 0:
+// one warp per slot, 16-byte loads, lanes own fixed column chunks, fixed
+// butterfly order.
+template <typename XT>
+__global__ void __launch_bounds__(256) gate_grad_warp_kernel(int TK, int K, int d, int passthrough,
+                                                              const int32_t* slot_row, const XT* dout,
+                                                              const XT* y, const XT* x, float* a) {
+    constexpr int V = 16 / sizeof(XT);
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (blockDim.x >> 5);
+    for (int slot = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); slot < TK; slot += warps) {
+        const int t = slot / K;
+        const int row = slot_row[slot];
+        const XT* other = row >= 0 ? y + static_cast<size_t>(row) * d
+                                   : ((row == -1 && passthrough) ? x + static_cast<size_t>(t) * d : nullptr);
+        float acc = 0.f;
+        if (other) {
+            const XT* dr = dout + static_cast<size_t>(t) * d;
+            for (int c = lane * V; c < d; c += 32 * V) {
+                const uint4 pa = *reinterpret_cast<const uint4*>(dr + c);
+                const uint4 pb = *reinterpret_cast<const uint4*>(other + c);
+                const XT* ea = reinterpret_cast<const XT*>(&pa);
+                const XT* eb = reinterpret_cast<const XT*>(&pb);
+#pragma unroll
+                for (int j = 0; j < V; ++j) acc += bwd::ld(ea, j) * bwd::ld(eb, j);
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) a[slot] = acc;
+    }
+}
+
+// poff[e] = sum over e' < e of roundup16(offsets[e'+1] - offsets[e']);
+// also clears the status word.  One warp.
+__global__ void pad_offsets_kernel(const int32_t* offsets, int E, int32_t* poff, int32_t* status) {
+    const int lane = threadIdx.x;
+    if (lane == 0) *status = 0;
+    int carry = 0;
+    for (int base = 0; base < E; base += 32) {
+        const int e = base + lane;
+        int v = e < E ? ((offsets[e + 1] - offsets[e] + 15) & ~15) : 0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, v, off);
+            if (lane >= off) v += o;
+        }
+        if (e < E) poff[e + 1] = v + carry;
+        carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+    if (lane == 0) poff[0] = 0;
+}
+
+// Padded rows (one warp each): x_p[pr] = x_disp[r], dy_p[pr] = g * dout[t]
+// for the rows of an expert's segment, zeros in its padding.
+__global__ void __launch_bounds__(256) pad_rows_kernel(int E, int K, int d, int rows_cap, const int32_t* offsets,
+                                                       const int32_t* poff, const int32_t* row_slot,
+                                                       const float* gates, const __nv_bfloat16* dout,
+                                                       const __nv_bfloat16* x_disp, __nv_bfloat16* x_p,
+                                                       __nv_bfloat16* dy_p) {
+    __shared__ int s_off[257], s_poff[257];
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) { s_off[i] = offsets[i]; s_poff[i] = poff[i]; }
+    __syncthreads();
+    const int total = s_poff[E];
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (blockDim.x >> 5);
+    for (int pr = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); pr < total && pr < rows_cap; pr += warps) {
+        int lo = 0, hi = E - 1;                         // last e with poff[e] <= pr
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (s_poff[mid] <= pr) lo = mid; else hi = mid - 1;
+        }
+        const int e = lo, i = pr - s_poff[e];
+        uint4* xo = reinterpret_cast<uint4*>(x_p + static_cast<size_t>(pr) * d);
+        uint4* yo = reinterpret_cast<uint4*>(dy_p + static_cast<size_t>(pr) * d);
+        if (i < s_off[e + 1] - s_off[e]) {
+            const int r = s_off[e] + i;
+            const int slot = row_slot[r];
+            const float g = gates[slot];
+            const uint4* xi = reinterpret_cast<const uint4*>(x_disp + static_cast<size_t>(r) * d);
+            const uint4* di = reinterpret_cast<const uint4*>(dout + static_cast<size_t>(slot / K) * d);
+            for (int c = lane; c < d / 8; c += 32) {
+                xo[c] = xi[c];
+                uint4 v = di[c];
+                uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+                    __nv_bfloat162 o = __floats2bfloat162_rn(g * f.x, g * f.y);
+                    w[j] = *reinterpret_cast<uint32_t*>(&o);
+                }
+                yo[c] = v;
+            }
+        } else {
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+            for (int c = lane; c < d / 8; c += 32) { xo[c] = z; yo[c] = z; }
+        }
+    }
+}
+
+// part[ch][c] = sum of rows ch*CH .. min(ch*CH + CH, n_rows) - 1 of column c
+// (bf16 matrix, row stride ld); n_rows from *n_rows_dev when given.
+template <int CH>
+__global__ void __launch_bounds__(256) colsum_chunks_kernel(const __nv_bfloat16* M, int ld, int ncols,
+                                                            const int32_t* n_rows_dev, int n_rows, float* part) {
+    const int rows = n_rows_dev ? *n_rows_dev : n_rows;
+    const int c = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+    if (c >= ncols) return;
+    for (int ch = blockIdx.y; ch * CH < rows; ch += gridDim.y) {
+        const int r0 = ch * CH, r1 = min(r0 + CH, rows);
+        float s0 = 0.f, s1 = 0.f;
+        for (int r = r0; r < r1; ++r) {
+            const float2 f = __bfloat1622float2(
+                *reinterpret_cast<const __nv_bfloat162*>(M + static_cast<size_t>(r) * ld + c));
+            s0 += f.x;
+            s1 += f.y;
+        }
+        *reinterpret_cast<float2*>(part + static_cast<size_t>(ch) * ncols + c) = make_float2(s0, s1);
+    }
+}
+
+// out[copy * copy_stride + s * ncols + c] = sum over the chunks of segment s
+// of part[ch][c], in chunk order.  Segment s spans rows seg[s] .. seg[s+1]-1
+// (multiples of CH) or, with seg == nullptr, rows 0 .. fixed_rows-1.
+template <int CH>
+__global__ void __launch_bounds__(256) colsum_segments_kernel(const float* part, int ncols, const int32_t* seg,
+                                                              int nseg, int fixed_rows, float* out, int copies,
+                                                              int copy_stride) {
+    const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (i >= static_cast<size_t>(nseg) * ncols) return;
+    const int s = static_cast<int>(i / ncols), c = static_cast<int>(i % ncols);
+    const int ch0 = seg ? seg[s] / CH : 0;
+    const int ch1 = seg ? seg[s + 1] / CH : (fixed_rows + CH - 1) / CH;
+    float acc = 0.f;
+    for (int ch = ch0; ch < ch1; ++ch) acc += part[static_cast<size_t>(ch) * ncols + c];
+    for (int k = 0; k < copies; ++k) out[static_cast<size_t>(k) * copy_stride + i] = acc;
+}
+
+// dx[t][c] = dx_router[t][c] + dx_shared[t][c] + sum_k (kept: dx rows of
+// the slot's padded row; passed through: g * dout[t][c]).
+__global__ void __launch_bounds__(256) dx_final_kernel(int T, int K, int d, int passthrough, const float* dx_router,
+                                                       const float* dx_shared, const int32_t* slot_row,
+                                                       const int32_t* topk_idx, const int32_t* offsets,
+                                                       const int32_t* poff, const float* gates, const float* dxr_p,
+                                                       const __nv_bfloat16* dout, float* dx) {
+    const size_t n = static_cast<size_t>(T) * d;
+    for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        const size_t t = i / d, c = i % d;
+        float v = dx_router[i];
+        if (dx_shared) v += dx_shared[i];
+        for (int k = 0; k < K; ++k) {
+            const int row = slot_row[t * K + k];
+            if (row >= 0) {
+                const int e = topk_idx[t * K + k];
+                const size_t pr = static_cast<size_t>(row - offsets[e] + poff[e]);
+                v += dxr_p[pr * d + c];
+            } else if (row == -1 && passthrough) {
+                v += gates[t * K + k] * __bfloat162float(dout[i]);
+            }
+        }
+        dx[i] = v;
+    }
+}
+
+struct TcLayout {
+    size_t status, a, dl, dxacc, poff, x_p, dy_p, h_p, sp_p, dz_p, dxr_p, h_s, sp_s, dz_s, dx_s, part, total;
+    int rows_cap;   // padded routed rows
+};
+
+constexpr int kChunkRouted = 16;    // row chunk of the routed column sums (the padding unit)
+constexpr int kChunkShared = 128;
+
+TcLayout tc_layout(const Dims& dm) {
+    TcLayout L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = (off + bytes + 255) & ~static_cast<size_t>(255);
+        return o;
+    };
+    const size_t T = dm.T, d = dm.d, E = dm.E, K = dm.K, dff = dm.dff;
+    const size_t sw = static_cast<size_t>(dm.S) * dm.dffs;
+    const size_t Rp = (static_cast<size_t>(dm.r_cap) + 15 * E + 15) & ~static_cast<size_t>(15);
+    L.rows_cap = static_cast<int>(Rp);
+    L.status = take(256);
+    L.a = take(T * K * 4);
+    L.dl = take(T * E * 4);
+    L.dxacc = take(T * d * 4);
+    L.poff = take((E + 1) * 4);
+    L.x_p = take(Rp * d * 2);
+    L.dy_p = take(Rp * d * 2);
+    L.h_p = take(Rp * dff * 2);
+    L.sp_p = take(Rp * dff * 2);
+    L.dz_p = take(Rp * dff * 2);
+    L.dxr_p = take(Rp * d * 4);
+    L.h_s = take(T * sw * 2);
+    L.sp_s = take(T * sw * 2);
+    L.dz_s = take(T * sw * 2);
+    L.dx_s = take(sw ? T * d * 4 : 0);
+    const size_t pr = (Rp / kChunkRouted) * (d > dff ? d : dff);
+    const size_t ps = ((T + kChunkShared - 1) / kChunkShared) * (d > sw ? d : sw);
+    L.part = take((pr > ps ? pr : ps) * 4);
+    L.total = off;
+    return L;
+}
+
+BwdGemmGroup group0() {
+    BwdGemmGroup g;
+    std::memset(&g, 0, sizeof(g));
+    return g;
+}
+
+cudaError_t run_backward_bf16(const Dims& dm, float lam, const moe_backward_io& io, void* bws, cudaStream_t st,
+                              int& launches) {
+    using bf = __nv_bfloat16;
+    const TcLayout L = tc_layout(dm);
+    uint8_t* base = static_cast<uint8_t*>(bws);
+    auto F = [&](size_t o) { return reinterpret_cast<float*>(base + o); };
+    auto B = [&](size_t o) { return reinterpret_cast<bf*>(base + o); };
+    int32_t* status = reinterpret_cast<int32_t*>(base + L.status);
+    int32_t* poff = reinterpret_cast<int32_t*>(base + L.poff);
+    float *a = F(L.a), *dl = F(L.dl), *dxacc = F(L.dxacc), *dxr_p = F(L.dxr_p), *dx_s = F(L.dx_s), *part = F(L.part);
+    bf *x_p = B(L.x_p), *dy_p = B(L.dy_p), *h_p = B(L.h_p), *sp_p = B(L.sp_p), *dz_p = B(L.dz_p);
+    bf *h_s = B(L.h_s), *sp_s = B(L.sp_s), *dz_s = B(L.dz_s);
+    const int T = dm.T, d = dm.d, E = dm.E, K = dm.K, dff = dm.dff, S = dm.S, dffs = dm.dffs, Rp = L.rows_cap;
+    const int sw = S * dffs;
+    const bf* x = static_cast<const bf*>(io.x);
+    const bf* dout = static_cast<const bf*>(io.dout);
+    const int sms = device_sm_count();
+    GpuExec ex{st, cudaSuccess, 0, sms * 16};
+    auto check = [&](cudaError_t e) { if (ex.err == cudaSuccess && e != cudaSuccess) ex.err = e; };
+
+    // router and gates
+    pad_offsets_kernel<<<1, 32, 0, st>>>(io.offsets, E, poff, status);
+    check(cudaGetLastError());
+    ++ex.launches;
+    {
+        const int TK = T * K;
+        const int blocks = std::min((TK + 7) / 8, sms * 8);
+        gate_grad_warp_kernel<bf><<<blocks, 256, 0, st>>>(TK, K, d, dm.passthrough, io.slot_row, dout,
+                                                         static_cast<const bf*>(io.y), x, a);
+        check(cudaGetLastError());
+        ++ex.launches;
+    }
+    const float bal = lam * dm.alpha * static_cast<float>(dm.E) /
+                      (static_cast<float>(dm.T) * static_cast<float>(dm.T) * static_cast<float>(dm.K));
+    ex.run(T, bwd::RouterGrad{dm.T, dm.E, dm.K, bal, io.logits, io.topk_idx, io.gates, a, io.counts, dl});
+    ex.run(static_cast<size_t>(E) * d, bwd::RouterWGrad<bf>{dm.T, dm.E, dm.d, dl, x, io.dW_r});
+    if (io.d_logit_bias) {
+        if (dm.bias_mode == 0) ex.run(E, bwd::ColSum{bwd::Seg{nullptr, dm.T}, dm.E, dl, io.d_logit_bias});
+        else ex.run(E, bwd::Fill{0.f, io.d_logit_bias});
+    }
+    ex.run(static_cast<size_t>(T) * d, bwd::RouterDx{dm.E, dm.d, dl, io.W_r, dxacc});
+    if (ex.err != cudaSuccess) { launches = ex.launches; return ex.err; }
+
+    // padded routed rows
+    {
+        const int blocks = std::min((Rp + 7) / 8, sms * 8);
+        pad_rows_kernel<<<blocks, 256, 0, st>>>(E, K, d, Rp, io.offsets, poff, io.row_slot, io.gates, dout,
+                                                static_cast<const bf*>(io.x_disp), x_p, dy_p);
+        check(cudaGetLastError());
+        ++ex.launches;
+    }
+    // 3. recompute: SiLU(z), SiLU'(z)
+    {
+        BwdGemmArgs ga;
+        ga.g[0] = group0();
+        ga.g[1] = group0();
+        ga.status = status;
+        BwdGemmGroup& r = ga.g[0];
+        r.n_mats = E; r.seg = poff; r.N = dff; r.K = d;
+        r.A = x_p; r.a_rows = Rp; r.a_cols = d;
+        r.B = io.W1; r.b_mats = E; r.b_rows = dff; r.b_cols = d; r.b_z_mat = 1;
+        r.bias = io.b1; r.out0 = h_p; r.out1 = sp_p; r.ldc = dff;
+        if (S > 0) {
+            BwdGemmGroup& s = ga.g[1];
+            s.n_mats = 1; s.fixed = T; s.N = sw; s.K = d;
+            s.A = x; s.a_rows = T; s.a_cols = d;
+            s.B = io.Ws1; s.b_mats = 1; s.b_rows = sw; s.b_cols = d;
+            s.bias = io.bs1; s.out0 = h_s; s.out1 = sp_s; s.ldc = sw;
+        }
+        check(launch_bwd_gemm(BWD_RECOMPUTE, ga, st));    // counts its own launch
+    }
+    // 4. dz = (dy W2) * SiLU'(z)
+    {
+        BwdGemmArgs ga;
+        ga.g[0] = group0();
+        ga.g[1] = group0();
+        ga.status = status;
+        BwdGemmGroup& r = ga.g[0];
+        r.n_mats = E; r.seg = poff; r.N = dff; r.K = d;
+        r.A = dy_p; r.a_rows = Rp; r.a_cols = d;
+        r.B = io.W2; r.b_mats = E; r.b_rows = d; r.b_cols = dff; r.b_z_mat = 1;
+        r.aux = sp_p; r.out0 = dz_p; r.ldc = dff;
+        if (S > 0) {
+            BwdGemmGroup& s = ga.g[1];
+            s.n_mats = S; s.fixed = T; s.N = dffs; s.K = d;
+            s.A = dout; s.a_rows = T; s.a_cols = d;
+            s.B = io.Ws2; s.b_mats = S; s.b_rows = d; s.b_cols = dffs; s.b_z_mat = 1;
+            s.aux = sp_s; s.out0 = dz_s; s.ldc = sw; s.c_col_stride = dffs;
+        }
+        check(launch_bwd_gemm(BWD_DGRAD_SILU, ga, st));
+    }
+    // 5. dx rows = dz W1 (routed, per padded row), dz_s Ws1 (shared, all at once)
+    {
+        BwdGemmArgs ga;
+        ga.g[0] = group0();
+        ga.g[1] = group0();
+        ga.status = status;
+        BwdGemmGroup& r = ga.g[0];
+        r.n_mats = E; r.seg = poff; r.N = d; r.K = dff;
+        r.A = dz_p; r.a_rows = Rp; r.a_cols = dff;
+        r.B = io.W1; r.b_mats = E; r.b_rows = dff; r.b_cols = d; r.b_z_mat = 1;
+        r.out0 = dxr_p; r.ldc = d;
+        if (S > 0) {
+            BwdGemmGroup& s = ga.g[1];
+            s.n_mats = 1; s.fixed = T; s.N = d; s.K = sw;
+            s.A = dz_s; s.a_rows = T; s.a_cols = sw;
+            s.B = io.Ws1; s.b_mats = 1; s.b_rows = sw; s.b_cols = d;
+            s.out0 = dx_s; s.ldc = d;
+        }
+        check(launch_bwd_gemm(BWD_DGRAD_F32, ga, st));
+    }
+    // 6a. dW2 = dy^T SiLU(z)
+    {
+        BwdGemmArgs ga;
+        ga.g[0] = group0();
+        ga.g[1] = group0();
+        ga.status = status;
+        BwdGemmGroup& r = ga.g[0];
+        r.n_mats = E; r.seg = poff; r.M = d; r.N = dff;
+        r.A = dy_p; r.a_rows = Rp; r.a_cols = d;
+        r.B = h_p; r.b_mats = 1; r.b_rows = Rp; r.b_cols = dff;
+        r.out0 = io.dW2; r.ldc = dff; r.c_mat_elems = static_cast<long long>(d) * dff;
+        if (S > 0) {
+            BwdGemmGroup& s = ga.g[1];
+            s.n_mats = S; s.fixed = T; s.M = d; s.N = dffs;
+            s.A = dout; s.a_rows = T; s.a_cols = d;
+            s.B = h_s; s.b_mats = 1; s.b_rows = T; s.b_cols = sw; s.b_col_stride = dffs;
+            s.out0 = io.dWs2; s.ldc = dffs; s.c_mat_elems = static_cast<long long>(d) * dffs;
+        }
+        check(launch_bwd_gemm(BWD_WGRAD, ga, st));
+    }
+    // 6b. dW1 = dz^T x
+    {
+        BwdGemmArgs ga;
+        ga.g[0] = group0();
+        ga.g[1] = group0();
+        ga.status = status;
+        BwdGemmGroup& r = ga.g[0];
+        r.n_mats = E; r.seg = poff; r.M = dff; r.N = d;
+        r.A = dz_p; r.a_rows = Rp; r.a_cols = dff;
+        r.B = x_p; r.b_mats = 1; r.b_rows = Rp; r.b_cols = d;
+        r.out0 = io.dW1; r.ldc = d; r.c_mat_elems = static_cast<long long>(dff) * d;
+        if (S > 0) {
+            BwdGemmGroup& s = ga.g[1];
+            s.n_mats = 1; s.fixed = T; s.M = sw; s.N = d;
+            s.A = dz_s; s.a_rows = T; s.a_cols = sw;
+            s.B = x; s.b_mats = 1; s.b_rows = T; s.b_cols = d;
+            s.out0 = io.dWs1; s.ldc = d;
+        }
+        check(launch_bwd_gemm(BWD_WGRAD, ga, st));
+    }
+    if (ex.err != cudaSuccess) { launches = ex.launches; return ex.err; }
+
+    // 7. bias gradients
+    auto colsum_routed = [&](const bf* M, int ncols, float* out) {
+        const dim3 g1((ncols / 2 + 255) / 256, std::min(Rp / kChunkRouted, 65535));
+        colsum_chunks_kernel<kChunkRouted><<<g1, 256, 0, st>>>(M, ncols, ncols, poff + E, 0, part);
+        check(cudaGetLastError());
+        const size_t n = static_cast<size_t>(E) * ncols;
+        colsum_segments_kernel<kChunkRouted><<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
+            part, ncols, poff, E, 0, out, 1, 0);
+        check(cudaGetLastError());
+        ex.launches += 2;
+    };
+    auto colsum_shared = [&](const bf* M, int ncols, float* out, int copies, int copy_stride) {
+        const dim3 g1((ncols / 2 + 255) / 256, std::min((T + kChunkShared - 1) / kChunkShared, 65535));
+        colsum_chunks_kernel<kChunkShared><<<g1, 256, 0, st>>>(M, ncols, ncols, nullptr, T, part);
+        check(cudaGetLastError());
+        colsum_segments_kernel<kChunkShared><<<static_cast<unsigned>((ncols + 255) / 256), 256, 0, st>>>(
+            part, ncols, nullptr, 1, T, out, copies, copy_stride);
+        check(cudaGetLastError());
+        ex.launches += 2;
+    };
+    colsum_routed(dy_p, d, io.db2);
+    colsum_routed(dz_p, dff, io.db1);
+    if (S > 0) {
+        colsum_shared(dout, d, io.dbs2, S, d);
+        colsum_shared(dz_s, sw, io.dbs1, 1, 0);
+    }
+
+    // 8. dx
+    {
+        const size_t n = static_cast<size_t>(T) * d;
+        const int blocks = static_cast<int>(std::min<size_t>((n + 255) / 256, static_cast<size_t>(sms) * 16));
+        dx_final_kernel<<<blocks, 256, 0, st>>>(T, K, d, dm.passthrough, dxacc, S > 0 ? dx_s : nullptr,
+                                                io.slot_row, io.topk_idx, io.offsets, poff, io.gates, dxr_p,
+                                                dout, io.dx);
+        check(cudaGetLastError());
+        ++ex.launches;
+    }
+    launches = ex.launches;
+    return ex.err;
+}
+
 }  // namespace
 
-size_t backward_ws_bytes(const Dims& dm) { return bwd::bwd_layout(dm).total; }
+size_t backward_ws_bytes(const Dims& dm) {
+    return dm.dtype == MOE_BF16 ? tc_layout(dm).total : bwd::bwd_layout(dm).total;
+}
 
 cudaError_t launch_backward(const Dims& dm, float lam, const moe_backward_io& io, void* bws,
                             cudaStream_t st) {
-    GpuExec ex{st, cudaSuccess, 0};
+    if (dm.dtype == MOE_BF16) {
+        int launches = 0;
+        const cudaError_t e = run_backward_bf16(dm, lam, io, bws, st, launches);
+        count_launches(launches);
+        return e;
+    }
+    GpuExec ex{st, cudaSuccess, 0, device_sm_count() * 16};
     bwd::run_backward(ex, dm, lam, io, bws);
     count_launches(ex.launches);
     return ex.err;

@@ -316,7 +316,7 @@ template <typename XT> struct DxFinal {
 // ------------------------------------------------------------ workspace
 
 struct BwdLayout {
-    size_t a, dl, dyr, zr, dzr, dxr, dys, zs, dzs, dxacc, total;
+    size_t status, a, dl, dyr, zr, dzr, dxr, dys, zs, dzs, dxacc, total;
 };
 
 inline BwdLayout bwd_layout(const Dims& dm) {
@@ -328,6 +328,7 @@ inline BwdLayout bwd_layout(const Dims& dm) {
         return o;
     };
     const size_t T = dm.T, R = dm.r_cap;
+    L.status = take(64);
     L.a = take(T * dm.K);
     L.dl = take(T * dm.E);
     L.dyr = take(R * dm.d);
@@ -355,6 +356,7 @@ void run_backward_t(Exec& ex, const Dims& dm, float lam, const moe_backward_io& 
     const XT* dout = static_cast<const XT*>(io.dout);
     const XT* xd = static_cast<const XT*>(io.x_disp);
 
+    ex.run(1, Fill{0.f, F(L.status)});                     // device status word: no waits here
     ex.run(T * K, GateGrad<XT>{dm.K, dm.d, dm.passthrough, io.slot_row, dout, static_cast<const XT*>(io.y), x, a});
     const float bal = lam * dm.alpha * static_cast<float>(dm.E) /
                       (static_cast<float>(dm.T) * static_cast<float>(dm.T) * static_cast<float>(dm.K));

@@ -169,6 +169,47 @@ void note_cuda_error(int err);
 // Adds n to the process-wide kernel launch counter (moe_kernel_launches).
 void count_launches(int n = 1);
 
+// One group of a grouped GEMM of the backward (bwd_gemm.cu), bf16 operands.
+// M-ragged kinds: C[rows of segment i, N] = A[rows, K] op(B_i); K-ragged
+// (BWD_WGRAD): C_i[M, N] = A[K rows of i, M]^T B[K rows of i, N].
+struct BwdGemmGroup {
+    int n_mats;              // segments (matrices); 0: group unused
+    const int32_t* seg;      // (n_mats + 1) device row offsets (16-row multiples apart), or nullptr
+    int fixed;               // rows of every segment when seg is nullptr
+    int M, N, K;             // M-ragged: N, K; K-ragged: M, N
+    const void* A;           // (a_rows, a_cols) row-major
+    int a_rows, a_cols;
+    int a_row_base;          // first A row (K row when K-ragged) of segment 0
+    int a_mat_stride;        // fixed segments: rows between segments
+    const void* B;           // (b_mats, b_rows, b_cols) row-major
+    int b_mats, b_rows, b_cols;
+    int b_col_stride;        // K-ragged: B column offset of matrix i
+    int b_z_mat;             // 1: B matrix index = segment index; 0: matrix 0
+    const float* bias;       // recompute: (n_mats, N)
+    const void* aux;         // dgrad-SiLU: SiLU'(z) bf16, addressed like out0
+    void* out0;
+    void* out1;              // recompute: SiLU'(z)
+    int c_row_base;          // M-ragged: first output row of segment 0 (routed) or of all
+    int c_mat_rows;          // fixed segments: output rows between segments
+    int c_col_stride;        // M-ragged: output column offset of segment i
+    int ldc;                 // output row stride (elements)
+    long long c_mat_elems;   // K-ragged: elements between the matrices' outputs
+};
+
+struct BwdGemmArgs {
+    BwdGemmGroup g[2];       // routed, shared (n_mats == 0 if none)
+    int32_t* status;
+};
+
+enum BwdGemmKind {
+    BWD_RECOMPUTE = 0,       // M-ragged, B K-major; out0 = SiLU(v), out1 = SiLU'(v), v = acc + bias (bf16)
+    BWD_DGRAD_SILU = 1,      // M-ragged, B MN-major; out0 = acc * aux (bf16)
+    BWD_DGRAD_F32 = 2,       // M-ragged, B MN-major; out0 = acc (fp32)
+    BWD_WGRAD = 3,           // K-ragged, A and B MN-major; out0 = acc (fp32), zeros for K = 0
+};
+
+cudaError_t launch_bwd_gemm(BwdGemmKind kind, const BwdGemmArgs& a, cudaStream_t st);
+
 // Layer backward (backward.cu): scratch bytes and the launch sequence.
 size_t backward_ws_bytes(const Dims& dm);
 cudaError_t launch_backward(const Dims& dm, float lam, const moe_backward_io& io, void* bws,

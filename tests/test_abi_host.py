@@ -9,7 +9,7 @@ import pytest
 
 import oracle as O
 import sparse_mixture_experts_20_b200 as M
-from synthetic import WORKLOADS
+from synthetic import DTYPE_F32, WORKLOADS
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -143,12 +143,33 @@ def test_fp8_requires_scales():
     assert L.moe_dispatch(ctypes.byref(cfg), *args) == M.MOE_ERR_INVALID_ARG
 
 
+def _r256(n):
+    return (n + 255) // 256 * 256
+
+
 def _bwd_layout_bytes(T, d, E, K, dff, S, dffs, r_cap):
-    """Closed form of the backward scratch: fp32 regions, each rounded up to
-    256 bytes, in the order a, dl, dy, z, dz, dx rows, shared dy, z, dz, dx."""
-    regions = [T * K, T * E, r_cap * d, r_cap * dff, r_cap * dff, r_cap * d,
+    """Closed form of the fp32 layers' backward scratch: fp32 regions, each
+    rounded up to 256 bytes, in the order status, a, dl, dy, z, dz, dx rows,
+    shared dy, z, dz, dx."""
+    regions = [64, T * K, T * E, r_cap * d, r_cap * dff, r_cap * dff, r_cap * d,
                T * d if S else 0, T * dffs if S else 0, T * dffs if S else 0, T * d]
-    return sum((n * 4 + 255) // 256 * 256 for n in regions)
+    return sum(_r256(n * 4) for n in regions)
+
+
+def _bwd_tc_layout_bytes(T, d, E, K, dff, S, dffs, r_cap):
+    """Closed form of the bf16 layers' backward scratch: status word; fp32 a,
+    dl, router dx; padded row offsets; routed rows padded to 16 per expert
+    (r_cap + 15 E, rounded to 16): bf16 x, dy, SiLU(z), SiLU'(z), dz and fp32
+    dx rows; shared bf16 SiLU(z), SiLU'(z), dz of width n_shared * d_ff_shared
+    and fp32 dx; fp32 column-sum partials (16-row chunks of the routed rows,
+    128-row chunks of the tokens)."""
+    rp = (r_cap + 15 * E + 15) // 16 * 16
+    sw = S * dffs
+    part = max((rp // 16) * max(d, dff), ((T + 127) // 128) * max(d, sw))
+    regions = [256, T * K * 4, T * E * 4, T * d * 4, (E + 1) * 4,
+               rp * d * 2, rp * d * 2, rp * dff * 2, rp * dff * 2, rp * dff * 2, rp * d * 4,
+               T * sw * 2, T * sw * 2, T * sw * 2, T * d * 4 if sw else 0, part * 4]
+    return sum(_r256(n) for n in regions)
 
 
 @pytest.mark.parametrize("cid", [1, 2, 3])
@@ -156,7 +177,8 @@ def test_backward_workspace_closed_form(cid):
     sh = WORKLOADS[cid]
     cfg = M.make_config(sh)
     _, r_cap, _, _ = M.moe_buffer_rows(cfg)
-    assert M.moe_backward_workspace_size(cfg) == _bwd_layout_bytes(
+    form = _bwd_layout_bytes if sh.dtype == DTYPE_F32 else _bwd_tc_layout_bytes
+    assert M.moe_backward_workspace_size(cfg) == form(
         sh.T, sh.d_model, sh.n_routed, sh.top_k, sh.d_ff, sh.n_shared, sh.d_ff_shared, r_cap)
 
 
