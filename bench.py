@@ -21,7 +21,10 @@ value counts the tokens of all ranks.
 One JSON line on rank 0: tokens/s plus the grouped-GEMM roofline, the
 per-stage HBM fractions, the CPU oracle baseline (rank 0, N=1), an end-to-end
 figure through the public API with host buffers, and the SM clocks sampled
-during the timed region; the same fields per nested workload.
+during the timed region; the same fields per nested workload.  For the fp32
+and bf16 workloads the run also times the layer backward on the same batch
+("backward": tokens/s, and for bf16 its expert GEMMs' TFLOP/s against the
+tensor peak).
 
 --impl reference times the CPU oracle (the reference implementation of this
 repository: a plain fp64 restatement of the pages) on bounded token samples
@@ -443,6 +446,11 @@ def measure_workload(args, cid, sh, dev, world, rank, local, peaks, peak_src, cp
     counts = b["counts"].cpu().numpy()
     status = M.moe_get_device_status(cfg, ws) | layer.device_status()
     assert torch.equal(layer.topk_idx, b["topk_idx"]), "the layer call and the stage calls route alike"
+    bwd = None
+    if sh.dtype != 2:
+        bwd = measure_backward(args, sh, cfg, inp, b, ws, dev, world, local, stream, flush, int(kept.sum()),
+                               peaks, peak_src)
+        sampler.mark()
     del b
 
     # ---- end to end through the public API: pinned host x in, out + loss back
@@ -517,6 +525,8 @@ def measure_workload(args, cid, sh, dev, world, rank, local, peaks, peak_src, cp
         "device_status": status,
         "clocks": clocks,
     }
+    if bwd is not None:
+        res["backward"] = bwd
     if cpu_baseline and rank == 0 and world == 1:
         host = oracle_inputs_on_host(inp)
         # passes over the sample until about 10 s of host work (at least one)
@@ -533,6 +543,80 @@ def measure_workload(args, cid, sh, dev, world, rank, local, peaks, peak_src, cp
     del inp
     torch.cuda.synchronize(dev)
     torch.cuda.empty_cache()
+    return res
+
+
+def backward_flops(sh, kept_sum):
+    """Tensor-core work of one layer backward: per routed row and per shared
+    expert's token five d x d_ff products (recompute of z, dh, dx, dW2, dW1)
+    of 2 flop per multiply-add."""
+    return 10.0 * sh.d_model * (kept_sum * sh.d_ff + sh.n_shared * sh.T * sh.d_ff_shared)
+
+
+def measure_backward(args, sh, cfg, inp, b, ws, dev, world, local, stream, flush, kept_sum, peaks, peak_src):
+    """K timed calls of moe_layer_backward on the forward results of this
+    batch (fp32 gradients of <dout, out> + L_balance), L2 flushed between
+    calls outside the events; tokens/s and the expert GEMMs' flops over the
+    whole call against the bf16 tensor peak."""
+    import numpy as np
+    import torch
+
+    import sparse_mixture_experts_20_b200 as M
+    T, d, E = sh.T, sh.d_model, sh.n_routed
+    f32 = dict(dtype=torch.float32, device=dev)
+    logits = torch.empty((T, E), **f32)
+    M.moe_route(cfg, inp["x"], inp.get("W_r"), inp.get("logit_bias"), b["topk_idx"], b["gates"], logits, ws)
+    gen = torch.Generator(device=dev).manual_seed(args.seed + 17)
+    dout = torch.randn((T, d), generator=gen, device=dev, dtype=torch.float32).to(inp["x"].dtype)
+    t = {k: inp.get(k) for k in ("x", "W_r", "W1", "b1", "W2", "b2", "Ws1", "bs1", "Ws2", "bs2")}
+    t.update({k: b[k] for k in ("topk_idx", "gates", "counts", "offsets", "slot_row", "row_slot", "x_disp", "y")})
+    t.update(logits=logits, dout=dout, dx=torch.empty((T, d), **f32), dW_r=torch.empty((E, d), **f32),
+             dW1=torch.empty(inp["W1"].shape, **f32), db1=torch.empty(inp["b1"].shape, **f32),
+             dW2=torch.empty(inp["W2"].shape, **f32), db2=torch.empty(inp["b2"].shape, **f32))
+    if inp.get("logit_bias") is not None:
+        t["d_logit_bias"] = torch.empty(E, **f32)
+    if sh.n_shared:
+        for k in ("Ws1", "bs1", "Ws2", "bs2"):
+            t["d" + k] = torch.empty(inp[k].shape, **f32)
+    bws = torch.empty(M.moe_backward_workspace_size(cfg), dtype=torch.uint8, device=dev)
+    for _ in range(max(3, min(args.warmup, 5))):
+        flush.zero_()
+        M.moe_layer_backward(cfg, 1.0, t, bws)
+    torch.cuda.synchronize(dev)
+    assert bws[:4].view(torch.int32).item() == 0, "backward device status after warm-up"
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world, local)
+    torch.cuda.synchronize(dev)
+    l0 = M.moe_kernel_launches()
+    for k in range(args.steps):
+        flush.zero_()
+        ev[k][0].record(stream)
+        M.moe_layer_backward(cfg, 1.0, t, bws)
+        ev[k][1].record(stream)
+    torch.cuda.synchronize(dev)
+    launches = M.moe_kernel_launches() - l0
+    barrier(world, local)
+    ms = np.array([a.elapsed_time(c) for a, c in ev])
+    total = max_over_ranks(float(ms.sum()), world, dev)
+    status = int(bws[:4].view(torch.int32).item())
+    flops = backward_flops(sh, kept_sum)
+    per = total / args.steps
+    ach = flops / (per * 1e-3) / 1e12
+    res = {"value": round(job_throughput(T, world, args.steps, total), 1), "unit": "tokens/s",
+           "ms_per_step": round(per, 4),
+           "what": "moe_layer_backward per step (gradients of x, W_r, bias, every expert's weights and biases, "
+                   "fp32) on this batch's forward results; CUDA events around the call",
+           "gpu_launches": launches, "device_status": status}
+    if sh.dtype == 1:
+        res["roofline"] = {"bound": "tensor", "achieved": round(ach, 1), "peak": peaks["bf16_tflops"],
+                           "unit": "TFLOP/s", "frac": round(ach / peaks["bf16_tflops"], 4),
+                           "peak_source": f"{peak_src} (bf16 burst)",
+                           "frac_of_sustained_peak": round(ach / peaks["bf16_tflops_sustained"], 4)
+                           if peaks.get("bf16_tflops_sustained") else None,
+                           "kernel": "bwd_gemm_kernel (five launches: recompute, dz, dx, dW2, dW1); achieved = "
+                                     "their algorithmic flops over the whole backward call",
+                           "algorithmic": {"flops": flops}, "traffic": None}
+    del t, bws, logits, dout
     return res
 
 
@@ -612,7 +696,7 @@ def run_ours(args):
                 "data": "synthetic (seeded N(0,1) activations, N(0,1/fan_in) weights, N(0,0.01) biases)",
                 "config": head["config"], "impl": "ours"}
         for k in ("timing", "stages_ms", "grouped_gemm_tflops", "stages_hbm", "roofline", "e2e", "gpu_launches",
-                  "routing", "device_status", "clocks", "cpu_baseline"):
+                  "routing", "device_status", "clocks", "cpu_baseline", "backward"):
             if k in head:
                 line[k] = head[k]
         line["peaks"] = {"source": peak_src, "hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"]}

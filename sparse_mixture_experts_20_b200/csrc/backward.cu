@@ -88,6 +88,106 @@ __global__ void __launch_bounds__(256) gate_grad_warp_kernel(int TK, int K, int 
     }
 }
 
+// dl[t][j] = dJ/dl of token t (softmax of its logits, the gates' and the
+// balance loss's share of ds), one warp per token, lanes over experts; also
+// the bf16 copy dl_b (row stride Epad, zero columns E .. Epad-1) that the
+// tensor-core router gradients read.  Reductions in fixed butterfly order.
+__global__ void __launch_bounds__(256) router_grad_warp_kernel(int T, int E, int K, int Epad, float bal,
+                                                                const float* logits, const int32_t* topk_idx,
+                                                                const float* gates, const float* a,
+                                                                const int32_t* counts, float* dl,
+                                                                __nv_bfloat16* dl_b) {
+    constexpr int JMAX = 8;                          // E <= 256
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (blockDim.x >> 5);
+    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
+        const float* l = logits + static_cast<size_t>(t) * E;
+        float lv[JMAX];
+        float m = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < JMAX; ++i) {
+            const int j = lane + 32 * i;
+            lv[i] = j < E ? l[j] : -INFINITY;
+            m = fmaxf(m, lv[i]);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        float z = 0.f;
+#pragma unroll
+        for (int i = 0; i < JMAX; ++i) {
+            lv[i] = (lane + 32 * i) < E ? expf(lv[i] - m) : 0.f;
+            z += lv[i];
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+        // S = sum of s over the chosen experts; common = sum_k a_k g_k (same order on every lane)
+        float S = 0.f, common = 0.f;
+        for (int k = 0; k < K; ++k) {
+            const int j = topk_idx[static_cast<size_t>(t) * K + k];
+            if (j >= 0 && j < E) S += expf(l[j] - m) / z;
+            common += a[static_cast<size_t>(t) * K + k] * gates[static_cast<size_t>(t) * K + k];
+        }
+        float ds[JMAX];
+        float sds = 0.f;
+#pragma unroll
+        for (int i = 0; i < JMAX; ++i) {
+            const int j = lane + 32 * i;
+            float v = 0.f;
+            if (j < E) {
+                v = bal * static_cast<float>(counts[j]);
+                for (int k = 0; k < K; ++k)
+                    if (topk_idx[static_cast<size_t>(t) * K + k] == j) v += (a[static_cast<size_t>(t) * K + k] - common) / S;
+                lv[i] = lv[i] / z;                   // s_j
+            }
+            ds[i] = v;
+            sds += lv[i] * v;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sds += __shfl_xor_sync(0xffffffffu, sds, off);
+#pragma unroll
+        for (int i = 0; i < JMAX; ++i) {
+            const int j = lane + 32 * i;
+            if (j < E) {
+                const float v = lv[i] * (ds[i] - sds);
+                dl[static_cast<size_t>(t) * E + j] = v;
+                dl_b[static_cast<size_t>(t) * Epad + j] = __float2bfloat16_rn(v);
+            } else if (j < Epad) {
+                dl_b[static_cast<size_t>(t) * Epad + j] = __float2bfloat16_rn(0.f);
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256) f32_to_bf16_kernel(size_t n, const float* in, __nv_bfloat16* out) {
+    for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x)
+        out[i] = __float2bfloat16_rn(in[i]);
+}
+
+// out[i] = sum over s of part[s * n + i], in split order.
+__global__ void __launch_bounds__(256) sum_splits_kernel(size_t n, int splits, const float* part, float* out) {
+    for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        float acc = 0.f;
+        for (int s2 = 0; s2 < splits; ++s2) acc += part[static_cast<size_t>(s2) * n + i];
+        out[i] = acc;
+    }
+}
+
+// part[ch][c] = sum of rows ch*CH .. of column c of an fp32 (rows, ncols)
+// matrix (any ncols); one column per thread.
+template <int CH>
+__global__ void __launch_bounds__(256) colsum_chunks_f32_kernel(const float* M, int ncols, int n_rows, float* part) {
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= ncols) return;
+    for (int ch = blockIdx.y; ch * CH < n_rows; ch += gridDim.y) {
+        const int r0 = ch * CH, r1 = min(r0 + CH, n_rows);
+        float acc = 0.f;
+        for (int r = r0; r < r1; ++r) acc += M[static_cast<size_t>(r) * ncols + c];
+        part[static_cast<size_t>(ch) * ncols + c] = acc;
+    }
+}
+
 // poff[e] = sum over e' < e of roundup16(offsets[e'+1] - offsets[e']);
 // also clears the status word.  One warp.
 __global__ void pad_offsets_kernel(const int32_t* offsets, int E, int32_t* poff, int32_t* status) {
@@ -193,37 +293,78 @@ __global__ void __launch_bounds__(256) colsum_segments_kernel(const float* part,
     for (int k = 0; k < copies; ++k) out[static_cast<size_t>(k) * copy_stride + i] = acc;
 }
 
-// dx[t][c] = dx_router[t][c] + dx_shared[t][c] + sum_k (kept: dx rows of
-// the slot's padded row; passed through: g * dout[t][c]).
+// dx[t][c] = dx_router[t][c] + dx_shared[t][c] + sum_k (kept: the bf16 dx
+// row of the slot's padded row; passed through: g * dout[t][c]), one warp per
+// token: the slots' rows are looked up once, lanes take 8 columns at a time.
 __global__ void __launch_bounds__(256) dx_final_kernel(int T, int K, int d, int passthrough, const float* dx_router,
                                                        const float* dx_shared, const int32_t* slot_row,
                                                        const int32_t* topk_idx, const int32_t* offsets,
-                                                       const int32_t* poff, const float* gates, const float* dxr_p,
-                                                       const __nv_bfloat16* dout, float* dx) {
-    const size_t n = static_cast<size_t>(T) * d;
-    for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-        const size_t t = i / d, c = i % d;
-        float v = dx_router[i];
-        if (dx_shared) v += dx_shared[i];
-        for (int k = 0; k < K; ++k) {
-            const int row = slot_row[t * K + k];
+                                                       const int32_t* poff, const float* gates,
+                                                       const __nv_bfloat16* dxr_p, const __nv_bfloat16* dout,
+                                                       float* dx) {
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (blockDim.x >> 5);
+    for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += warps) {
+        // lane k < K: padded row of slot k (>= 0), -1 passed through, -2 nothing
+        long long my_row = -2;
+        float my_g = 0.f;
+        if (lane < K) {
+            const int row = slot_row[static_cast<size_t>(t) * K + lane];
             if (row >= 0) {
-                const int e = topk_idx[t * K + k];
-                const size_t pr = static_cast<size_t>(row - offsets[e] + poff[e]);
-                v += dxr_p[pr * d + c];
+                const int e = topk_idx[static_cast<size_t>(t) * K + lane];
+                my_row = row - offsets[e] + poff[e];
             } else if (row == -1 && passthrough) {
-                v += gates[t * K + k] * __bfloat162float(dout[i]);
+                my_row = -1;
+                my_g = gates[static_cast<size_t>(t) * K + lane];
             }
         }
-        dx[i] = v;
+        const size_t base = static_cast<size_t>(t) * d;
+        for (int c = lane * 8; c < d; c += 256) {
+            float v[8];
+            const float4 r0 = *reinterpret_cast<const float4*>(dx_router + base + c);
+            const float4 r1 = *reinterpret_cast<const float4*>(dx_router + base + c + 4);
+            v[0] = r0.x; v[1] = r0.y; v[2] = r0.z; v[3] = r0.w; v[4] = r1.x; v[5] = r1.y; v[6] = r1.z; v[7] = r1.w;
+            if (dx_shared) {
+                const float4 s0 = *reinterpret_cast<const float4*>(dx_shared + base + c);
+                const float4 s1 = *reinterpret_cast<const float4*>(dx_shared + base + c + 4);
+                v[0] += s0.x; v[1] += s0.y; v[2] += s0.z; v[3] += s0.w;
+                v[4] += s1.x; v[5] += s1.y; v[6] += s1.z; v[7] += s1.w;
+            }
+            for (int k = 0; k < K; ++k) {
+                const long long row = __shfl_sync(0xffffffffu, my_row, k);
+                const float gk = __shfl_sync(0xffffffffu, my_g, k);
+                if (row == -2) continue;
+                const __nv_bfloat16* src = row >= 0 ? dxr_p + static_cast<size_t>(row) * d + c : dout + base + c;
+                const float w = row >= 0 ? 1.f : gk;
+                const uint4 q = *reinterpret_cast<const uint4*>(src);
+                const uint32_t qw[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qw[j]));
+                    v[2 * j] += w * f.x;
+                    v[2 * j + 1] += w * f.y;
+                }
+            }
+            *reinterpret_cast<float4*>(dx + base + c) = make_float4(v[0], v[1], v[2], v[3]);
+            *reinterpret_cast<float4*>(dx + base + c + 4) = make_float4(v[4], v[5], v[6], v[7]);
+        }
     }
 }
 
 struct TcLayout {
-    size_t status, a, dl, dxacc, poff, x_p, dy_p, h_p, sp_p, dz_p, dxr_p, h_s, sp_s, dz_s, dx_s, part, total;
+    size_t status, a, dl, dl_b, w_rb, rw_part, dxacc, poff, x_p, dy_p, h_p, sp_p, dz_p, dxr_p, h_s, sp_s, dz_s,
+        dx_s, part, total;
     int rows_cap;   // padded routed rows
+    int epad;       // row stride of dl_b
+    int rw_splits;  // token splits of the router weight gradient
+    int rw_chunk;   // tokens per split
 };
+
+// The router weight gradient (M = N_r, N = d, K = T) has few output tiles:
+// its tokens are split so that about this many tiles run at once (a fixed
+// number, so that the workspace and the summation order do not depend on
+// the device).
+constexpr int kRouterSplitTiles = 296;
 
 constexpr int kChunkRouted = 16;    // row chunk of the routed column sums (the padding unit)
 constexpr int kChunkShared = 128;
@@ -240,9 +381,23 @@ TcLayout tc_layout(const Dims& dm) {
     const size_t sw = static_cast<size_t>(dm.S) * dm.dffs;
     const size_t Rp = (static_cast<size_t>(dm.r_cap) + 15 * E + 15) & ~static_cast<size_t>(15);
     L.rows_cap = static_cast<int>(Rp);
+    L.epad = static_cast<int>((E + 7) & ~static_cast<size_t>(7));
+    {
+        const int tiles = static_cast<int>(((E + 127) / 128) * ((d + 255) / 256));
+        int splits = (kRouterSplitTiles + tiles - 1) / tiles;
+        const int max_splits = (dm.T + 255) / 256;
+        if (splits > max_splits) splits = max_splits;
+        if (splits < 1) splits = 1;
+        const int chunk = ((dm.T + splits - 1) / splits + 15) & ~15;
+        L.rw_chunk = chunk;
+        L.rw_splits = (dm.T + chunk - 1) / chunk;
+    }
     L.status = take(256);
     L.a = take(T * K * 4);
     L.dl = take(T * E * 4);
+    L.dl_b = take(T * static_cast<size_t>(L.epad) * 2);
+    L.w_rb = take(E * d * 2);
+    L.rw_part = take(L.rw_splits > 1 ? static_cast<size_t>(L.rw_splits) * E * d * 4 : 0);
     L.dxacc = take(T * d * 4);
     L.poff = take((E + 1) * 4);
     L.x_p = take(Rp * d * 2);
@@ -250,13 +405,14 @@ TcLayout tc_layout(const Dims& dm) {
     L.h_p = take(Rp * dff * 2);
     L.sp_p = take(Rp * dff * 2);
     L.dz_p = take(Rp * dff * 2);
-    L.dxr_p = take(Rp * d * 4);
+    L.dxr_p = take(Rp * d * 2);
     L.h_s = take(T * sw * 2);
     L.sp_s = take(T * sw * 2);
     L.dz_s = take(T * sw * 2);
     L.dx_s = take(sw ? T * d * 4 : 0);
     const size_t pr = (Rp / kChunkRouted) * (d > dff ? d : dff);
-    const size_t ps = ((T + kChunkShared - 1) / kChunkShared) * (d > sw ? d : sw);
+    size_t ps = ((T + kChunkShared - 1) / kChunkShared) * (d > sw ? d : sw);
+    if (((T + kChunkShared - 1) / kChunkShared) * E > ps) ps = ((T + kChunkShared - 1) / kChunkShared) * E;
     L.part = take((pr > ps ? pr : ps) * 4);
     L.total = off;
     return L;
@@ -277,7 +433,9 @@ cudaError_t run_backward_bf16(const Dims& dm, float lam, const moe_backward_io& 
     auto B = [&](size_t o) { return reinterpret_cast<bf*>(base + o); };
     int32_t* status = reinterpret_cast<int32_t*>(base + L.status);
     int32_t* poff = reinterpret_cast<int32_t*>(base + L.poff);
-    float *a = F(L.a), *dl = F(L.dl), *dxacc = F(L.dxacc), *dxr_p = F(L.dxr_p), *dx_s = F(L.dx_s), *part = F(L.part);
+    float *a = F(L.a), *dl = F(L.dl), *dxacc = F(L.dxacc), *dx_s = F(L.dx_s), *part = F(L.part);
+    float* rw_part = F(L.rw_part);
+    bf *dl_b = B(L.dl_b), *w_rb = B(L.w_rb), *dxr_p = B(L.dxr_p);
     bf *x_p = B(L.x_p), *dy_p = B(L.dy_p), *h_p = B(L.h_p), *sp_p = B(L.sp_p), *dz_p = B(L.dz_p);
     bf *h_s = B(L.h_s), *sp_s = B(L.sp_s), *dz_s = B(L.dz_s);
     const int T = dm.T, d = dm.d, E = dm.E, K = dm.K, dff = dm.dff, S = dm.S, dffs = dm.dffs, Rp = L.rows_cap;
@@ -302,13 +460,66 @@ cudaError_t run_backward_bf16(const Dims& dm, float lam, const moe_backward_io& 
     }
     const float bal = lam * dm.alpha * static_cast<float>(dm.E) /
                       (static_cast<float>(dm.T) * static_cast<float>(dm.T) * static_cast<float>(dm.K));
-    ex.run(T, bwd::RouterGrad{dm.T, dm.E, dm.K, bal, io.logits, io.topk_idx, io.gates, a, io.counts, dl});
-    ex.run(static_cast<size_t>(E) * d, bwd::RouterWGrad<bf>{dm.T, dm.E, dm.d, dl, x, io.dW_r});
-    if (io.d_logit_bias) {
-        if (dm.bias_mode == 0) ex.run(E, bwd::ColSum{bwd::Seg{nullptr, dm.T}, dm.E, dl, io.d_logit_bias});
-        else ex.run(E, bwd::Fill{0.f, io.d_logit_bias});
+    {
+        const int blocks = std::min((T + 7) / 8, sms * 8);
+        router_grad_warp_kernel<<<blocks, 256, 0, st>>>(T, E, K, L.epad, bal, io.logits, io.topk_idx, io.gates, a,
+                                                       io.counts, dl, dl_b);
+        check(cudaGetLastError());
+        const size_t n = static_cast<size_t>(E) * d;
+        f32_to_bf16_kernel<<<static_cast<unsigned>(std::min<size_t>((n + 255) / 256, sms * 8)), 256, 0, st>>>(
+            n, io.W_r, w_rb);
+        check(cudaGetLastError());
+        ex.launches += 2;
     }
-    ex.run(static_cast<size_t>(T) * d, bwd::RouterDx{dm.E, dm.d, dl, io.W_r, dxacc});
+    // dW_r = dl^T x: a weight gradient over the T tokens, split in token
+    // chunks (partials summed in split order)
+    {
+        BwdGemmArgs ga;
+        ga.g[0] = group0();
+        ga.g[1] = group0();
+        ga.status = status;
+        BwdGemmGroup& r = ga.g[0];
+        r.n_mats = L.rw_splits; r.fixed = L.rw_chunk; r.M = E; r.N = d;
+        r.A = dl_b; r.a_rows = T; r.a_cols = L.epad; r.a_mat_stride = L.rw_chunk;
+        r.B = x; r.b_mats = 1; r.b_rows = T; r.b_cols = d;
+        r.out0 = L.rw_splits > 1 ? static_cast<void*>(rw_part) : static_cast<void*>(io.dW_r);
+        r.ldc = d; r.c_mat_elems = static_cast<long long>(E) * d;
+        check(launch_bwd_gemm(BWD_WGRAD, ga, st));
+        if (L.rw_splits > 1) {
+            const size_t n = static_cast<size_t>(E) * d;
+            sum_splits_kernel<<<static_cast<unsigned>(std::min<size_t>((n + 255) / 256, sms * 8)), 256, 0, st>>>(
+                n, L.rw_splits, rw_part, io.dW_r);
+            check(cudaGetLastError());
+            ++ex.launches;
+        }
+    }
+    if (io.d_logit_bias) {
+        if (dm.bias_mode == 0) {
+            const int nch = (T + kChunkShared - 1) / kChunkShared;
+            colsum_chunks_f32_kernel<kChunkShared><<<dim3((E + 255) / 256, std::min(nch, 65535)), 256, 0, st>>>(
+                dl, E, T, part);
+            check(cudaGetLastError());
+            colsum_segments_kernel<kChunkShared><<<(E + 255) / 256, 256, 0, st>>>(part, E, nullptr, 1, T,
+                                                                                 io.d_logit_bias, 1, 0);
+            check(cudaGetLastError());
+            ex.launches += 2;
+        } else {
+            ex.run(E, bwd::Fill{0.f, io.d_logit_bias});
+        }
+    }
+    // router part of dx: dl W_r (K = N_r, zero-filled to a multiple of 64)
+    {
+        BwdGemmArgs ga;
+        ga.g[0] = group0();
+        ga.g[1] = group0();
+        ga.status = status;
+        BwdGemmGroup& r = ga.g[0];
+        r.n_mats = 1; r.fixed = T; r.N = d; r.K = (E + 63) & ~63;
+        r.A = dl_b; r.a_rows = T; r.a_cols = L.epad;
+        r.B = w_rb; r.b_mats = 1; r.b_rows = E; r.b_cols = d;
+        r.out0 = dxacc; r.ldc = d;
+        check(launch_bwd_gemm(BWD_DGRAD_F32, ga, st));
+    }
     if (ex.err != cudaSuccess) { launches = ex.launches; return ex.err; }
 
     // padded routed rows
@@ -369,7 +580,7 @@ cudaError_t run_backward_bf16(const Dims& dm, float lam, const moe_backward_io& 
         r.n_mats = E; r.seg = poff; r.N = d; r.K = dff;
         r.A = dz_p; r.a_rows = Rp; r.a_cols = dff;
         r.B = io.W1; r.b_mats = E; r.b_rows = dff; r.b_cols = d; r.b_z_mat = 1;
-        r.out0 = dxr_p; r.ldc = d;
+        r.out0 = dxr_p; r.ldc = d; r.out_bf16 = 1;
         if (S > 0) {
             BwdGemmGroup& s = ga.g[1];
             s.n_mats = 1; s.fixed = T; s.N = d; s.K = sw;

@@ -30,7 +30,8 @@
 // two warps per lane quadrant split the 256 columns).  Epilogues:
 //   SILU_PAIR  v = acc + bias: SiLU(v) and SiLU'(v) as bf16 (recompute);
 //   DSILU      acc * SiLU'(z) read from the recompute's output, as bf16 (dz);
-//   F32        acc as fp32 (dx rows, weight gradients).
+//   F32        acc as fp32 (dx rows, weight gradients), or bf16 for dx rows
+//              when the group asks for it.
 // K is consumed in 16-row steps: a K-ragged segment issues only the steps
 // inside its (16-padded) row count, so rows of the next segment that share
 // the last TMA box are never multiplied.  Every wait is bounded (2 s); on
@@ -73,6 +74,7 @@ struct GroupDev {
     void* out1;
     int c_row_base, c_mat_rows, c_col_stride, ldc;
     long long c_mat_elems;
+    int out_bf16;
 };
 
 struct __align__(64) Params {
@@ -451,6 +453,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
                         uint4* dz = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out0) + off);
 #pragma unroll
                         for (int q = 0; q < 4; ++q) dz[q] = make_uint4(po[4 * q], po[4 * q + 1], po[4 * q + 2], po[4 * q + 3]);
+                    } else if (MODE == MODE_DX && g.out_bf16) {
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out0) + off);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            dst[q] = make_uint4(
+                                pack_bf16x2(__uint_as_float(r[u][8 * q + 0]), __uint_as_float(r[u][8 * q + 1])),
+                                pack_bf16x2(__uint_as_float(r[u][8 * q + 2]), __uint_as_float(r[u][8 * q + 3])),
+                                pack_bf16x2(__uint_as_float(r[u][8 * q + 4]), __uint_as_float(r[u][8 * q + 5])),
+                                pack_bf16x2(__uint_as_float(r[u][8 * q + 6]), __uint_as_float(r[u][8 * q + 7])));
                     } else {
                         float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out0) + off);
 #pragma unroll
@@ -497,6 +508,7 @@ bool fill_group(Params& p, int gi, const BwdGemmGroup& h, bool a_mn, bool b_mn) 
     d.c_col_stride = h.c_col_stride;
     d.ldc = h.ldc;
     d.c_mat_elems = h.c_mat_elems;
+    d.out_bf16 = h.out_bf16;
     // A (a_rows, a_cols): K-major boxes of 64 K x 128 rows, MN-major boxes of
     // 64 M x 64 K rows; B (b_mats, b_rows, b_cols): K-major boxes of 64 K x
     // 256 rows of N, MN-major boxes of 64 N x 64 rows of K

@@ -194,6 +194,7 @@ struct BwdGemmGroup {
     int c_col_stride;        // M-ragged: output column offset of segment i
     int ldc;                 // output row stride (elements)
     long long c_mat_elems;   // K-ragged: elements between the matrices' outputs
+    int out_bf16;            // BWD_DGRAD_F32: write bf16 instead of fp32
 };
 
 struct BwdGemmArgs {
@@ -204,7 +205,7 @@ struct BwdGemmArgs {
 enum BwdGemmKind {
     BWD_RECOMPUTE = 0,       // M-ragged, B K-major; out0 = SiLU(v), out1 = SiLU'(v), v = acc + bias (bf16)
     BWD_DGRAD_SILU = 1,      // M-ragged, B MN-major; out0 = acc * aux (bf16)
-    BWD_DGRAD_F32 = 2,       // M-ragged, B MN-major; out0 = acc (fp32)
+    BWD_DGRAD_F32 = 2,       // M-ragged, B MN-major; out0 = acc (fp32, or bf16 with out_bf16)
     BWD_WGRAD = 3,           // K-ragged, A and B MN-major; out0 = acc (fp32), zeros for K = 0
 };
 

@@ -158,16 +158,27 @@ def _bwd_layout_bytes(T, d, E, K, dff, S, dffs, r_cap):
 
 def _bwd_tc_layout_bytes(T, d, E, K, dff, S, dffs, r_cap):
     """Closed form of the bf16 layers' backward scratch: status word; fp32 a,
-    dl, router dx; padded row offsets; routed rows padded to 16 per expert
-    (r_cap + 15 E, rounded to 16): bf16 x, dy, SiLU(z), SiLU'(z), dz and fp32
-    dx rows; shared bf16 SiLU(z), SiLU'(z), dz of width n_shared * d_ff_shared
-    and fp32 dx; fp32 column-sum partials (16-row chunks of the routed rows,
-    128-row chunks of the tokens)."""
+    dl; bf16 dl (row stride N_r rounded up to 8) and W_r; fp32 partials of the
+    router weight gradient when its tokens are split (about 296 output tiles
+    at once, at most one split per 256 tokens, chunks of a multiple of 16
+    tokens); fp32 router dx; padded row offsets; routed rows padded to 16 per
+    expert (r_cap + 15 N_r, rounded to 16): bf16 x, dy, SiLU(z), SiLU'(z), dz
+    and dx rows; shared bf16 SiLU(z), SiLU'(z), dz of width n_shared *
+    d_ff_shared and fp32 dx; fp32 column-sum partials (16-row chunks of the
+    routed rows, 128-row chunks of the tokens)."""
     rp = (r_cap + 15 * E + 15) // 16 * 16
     sw = S * dffs
-    part = max((rp // 16) * max(d, dff), ((T + 127) // 128) * max(d, sw))
-    regions = [256, T * K * 4, T * E * 4, T * d * 4, (E + 1) * 4,
-               rp * d * 2, rp * d * 2, rp * dff * 2, rp * dff * 2, rp * dff * 2, rp * d * 4,
+    epad = (E + 7) // 8 * 8
+    tiles = ((E + 127) // 128) * ((d + 255) // 256)
+    splits = min(-(-296 // tiles), (T + 255) // 256)
+    splits = max(splits, 1)
+    chunk = (-(-T // splits) + 15) // 16 * 16
+    splits = -(-T // chunk)
+    nch = (T + 127) // 128
+    part = max((rp // 16) * max(d, dff), nch * max(d, sw), nch * E)
+    regions = [256, T * K * 4, T * E * 4, T * epad * 2, E * d * 2, splits * E * d * 4 if splits > 1 else 0,
+               T * d * 4, (E + 1) * 4,
+               rp * d * 2, rp * d * 2, rp * dff * 2, rp * dff * 2, rp * dff * 2, rp * d * 2,
                T * sw * 2, T * sw * 2, T * sw * 2, T * d * 4 if sw else 0, part * 4]
     return sum(_r256(n) for n in regions)
 
