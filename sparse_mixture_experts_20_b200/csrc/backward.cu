@@ -517,7 +517,7 @@ cudaError_t run_backward_bf16(const Dims& dm, float lam, const moe_backward_io& 
         r.n_mats = 1; r.fixed = T; r.N = d; r.K = (E + 63) & ~63;
         r.A = dl_b; r.a_rows = T; r.a_cols = L.epad;
         r.B = w_rb; r.b_mats = 1; r.b_rows = E; r.b_cols = d;
-        r.out0 = dxacc; r.ldc = d;
+        r.out0 = dxacc; r.ldc = d; r.c_rows = T;
         check(launch_bwd_gemm(BWD_DGRAD_F32, ga, st));
     }
     if (ex.err != cudaSuccess) { launches = ex.launches; return ex.err; }
@@ -540,13 +540,13 @@ cudaError_t run_backward_bf16(const Dims& dm, float lam, const moe_backward_io& 
         r.n_mats = E; r.seg = poff; r.N = dff; r.K = d;
         r.A = x_p; r.a_rows = Rp; r.a_cols = d;
         r.B = io.W1; r.b_mats = E; r.b_rows = dff; r.b_cols = d; r.b_z_mat = 1;
-        r.bias = io.b1; r.out0 = h_p; r.out1 = sp_p; r.ldc = dff;
+        r.bias = io.b1; r.out0 = h_p; r.out1 = sp_p; r.ldc = dff; r.c_rows = Rp;
         if (S > 0) {
             BwdGemmGroup& s = ga.g[1];
             s.n_mats = 1; s.fixed = T; s.N = sw; s.K = d;
             s.A = x; s.a_rows = T; s.a_cols = d;
             s.B = io.Ws1; s.b_mats = 1; s.b_rows = sw; s.b_cols = d;
-            s.bias = io.bs1; s.out0 = h_s; s.out1 = sp_s; s.ldc = sw;
+            s.bias = io.bs1; s.out0 = h_s; s.out1 = sp_s; s.ldc = sw; s.c_rows = T;
         }
         check(launch_bwd_gemm(BWD_RECOMPUTE, ga, st));    // counts its own launch
     }
@@ -560,13 +560,13 @@ cudaError_t run_backward_bf16(const Dims& dm, float lam, const moe_backward_io& 
         r.n_mats = E; r.seg = poff; r.N = dff; r.K = d;
         r.A = dy_p; r.a_rows = Rp; r.a_cols = d;
         r.B = io.W2; r.b_mats = E; r.b_rows = d; r.b_cols = dff; r.b_z_mat = 1;
-        r.aux = sp_p; r.out0 = dz_p; r.ldc = dff;
+        r.aux = sp_p; r.out0 = dz_p; r.ldc = dff; r.c_rows = Rp;
         if (S > 0) {
             BwdGemmGroup& s = ga.g[1];
             s.n_mats = S; s.fixed = T; s.N = dffs; s.K = d;
             s.A = dout; s.a_rows = T; s.a_cols = d;
             s.B = io.Ws2; s.b_mats = S; s.b_rows = d; s.b_cols = dffs; s.b_z_mat = 1;
-            s.aux = sp_s; s.out0 = dz_s; s.ldc = sw; s.c_col_stride = dffs;
+            s.aux = sp_s; s.out0 = dz_s; s.ldc = sw; s.c_col_stride = dffs; s.c_rows = T;
         }
         check(launch_bwd_gemm(BWD_DGRAD_SILU, ga, st));
     }
@@ -580,13 +580,13 @@ cudaError_t run_backward_bf16(const Dims& dm, float lam, const moe_backward_io& 
         r.n_mats = E; r.seg = poff; r.N = d; r.K = dff;
         r.A = dz_p; r.a_rows = Rp; r.a_cols = dff;
         r.B = io.W1; r.b_mats = E; r.b_rows = dff; r.b_cols = d; r.b_z_mat = 1;
-        r.out0 = dxr_p; r.ldc = d; r.out_bf16 = 1;
+        r.out0 = dxr_p; r.ldc = d; r.out_bf16 = 1; r.c_rows = Rp;
         if (S > 0) {
             BwdGemmGroup& s = ga.g[1];
             s.n_mats = 1; s.fixed = T; s.N = d; s.K = sw;
             s.A = dz_s; s.a_rows = T; s.a_cols = sw;
             s.B = io.Ws1; s.b_mats = 1; s.b_rows = sw; s.b_cols = d;
-            s.out0 = dx_s; s.ldc = d;
+            s.out0 = dx_s; s.ldc = d; s.c_rows = T;
         }
         check(launch_bwd_gemm(BWD_DGRAD_F32, ga, st));
     }

@@ -1,14 +1,14 @@
 // Grouped GEMMs of the layer backward in bf16 on the 5th-generation tensor
 // cores: the recompute of z = x W1^T + b1, the two data-gradient GEMMs
 // (dh = dy W2, dx = dz W1) and the two weight-gradient GEMMs (dW2 = dy^T
-// SiLU(z), dW1 = dz^T x) of every routed and shared expert.
+// SiLU(z), dW1 = dz^T x) of every routed and shared expert, plus the
+// router's own gradients (dW_r = dl^T x, dl W_r).
 //
 // The forward these differentiate is "論文解説: DeepSeekMoE" §アルゴリズム (each
 // expert Linear(d, d_ff) + bias -> SiLU -> Linear(d_ff, d) + bias) and
 // §共有エキスパート機構 (routed experts on their tokens, shared experts on all).
 //
-// Two tile schedules over the same warp-specialised engine (320 threads, one
-// CTA per SM, persistent):
+// Two tile schedules over the same warp-specialised engine:
 //   M-ragged  C[rows of a segment, N] = A[rows, K] * op(B_mat): the segment
 //             rows are an expert's dispatched rows (device-side offsets, the
 //             backward pads each expert's row count to a multiple of 16) or a
@@ -24,19 +24,36 @@
 // (instruction descriptor transpose bits; shared-memory descriptor with the
 // 64-element blocks LBO bytes apart and 8-row groups 1024 bytes apart).
 //
-// Roles: warp 0 TMA producer (ring of 4 stages of 16 KB A + 32 KB B), warp 1
-// MMA issuer (M=128, N=256, K=16 per instruction, fp32 accumulators in
-// tensor memory, two 256-column buffers), warps 2..9 epilogue (thread = row,
-// two warps per lane quadrant split the 256 columns).  Epilogues:
+// CTA pairs (clusters of two SMs, tcgen05 cta_group::2): one MMA instruction
+// computes a 256 x 256 x 16 block with A rows 0..127 in the first CTA's
+// shared memory and 128..255 in the second's, and the 256 output columns'
+// B operand split the same way, so each SM stages half the B bytes of a
+// single-CTA 128 x 256 tile.  A scheduled tile is two 128-row m-tiles and
+// one 256-wide n-tile; an odd last m-tile runs as an M = 128 pair MMA (64
+// rows per CTA; its accumulator folds the columns: lanes 0..63 hold columns
+// 0..127, lanes 64..127 columns 128..255), a last n-tile with at most 128
+// valid columns as an N = 128 pair MMA.  Both CTAs' TMA loads signal the
+// first CTA's stage barrier, where the pair's single MMA-issuing thread
+// waits; tcgen05.commit with a CTA mask frees the stage in both CTAs and
+// hands a finished accumulator to both epilogues.
+//
+// Per CTA (320 threads, one CTA per SM): warp 0 TMA producer (ring of 4
+// stages of 16 KB A + 16 KB B), warp 1 MMA issuer (first CTA of the pair),
+// warps 2..9 epilogue (two warps per tensor-memory lane quadrant).
+// Epilogues:
 //   SILU_PAIR  v = acc + bias: SiLU(v) and SiLU'(v) as bf16 (recompute);
 //   DSILU      acc * SiLU'(z) read from the recompute's output, as bf16 (dz);
 //   F32        acc as fp32 (dx rows, weight gradients), or bf16 for dx rows
 //              when the group asks for it.
+// Output chunks of 32 rows x 32 columns leave through shared memory and TMA
+// bulk stores (per-thread stores of a thread's 128-byte fp32 row pieces kept
+// the weight-gradient kernel waiting on its store queue); rows past a
+// segment's end are stored one by one.
 // K is consumed in 16-row steps: a K-ragged segment issues only the steps
 // inside its (16-padded) row count, so rows of the next segment that share
 // the last TMA box are never multiplied.  Every wait is bounded (2 s); on
-// expiry the CTA drains its copies and MMAs, frees tensor memory, exits and
-// leaves MOE_DEV_TIMEOUT in the status word.
+// expiry the CTA stops, the MMA thread waits for its issued MMAs, tensor
+// memory is freed and MOE_DEV_TIMEOUT is left in the status word.
 #include <cuda.h>
 #include <cstring>
 #include "common.cuh"
@@ -45,13 +62,15 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4, ACC_BUFS = 2;
-constexpr int NUM_THREADS = 320, EPI_THREADS = 256;
+constexpr int BM = 128;                 // rows of A per CTA (M = 256 per pair)
+constexpr int BN = 256, BN_HALF = 128;  // output columns per pair tile, B rows/columns per CTA
+constexpr int BK = 64, STAGES = 4, ACC_BUFS = 2;
+constexpr int NUM_THREADS = 320, EPI_WARPS = 8;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int MAX_SEGS = 256 + 8;
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;
 constexpr uint64_t kDrainTimeoutNs = 200000000ull;
-constexpr int BOX_BYTES = 64 * 64 * 2;       // one MN-major box: 64 elements x 64 K rows
+constexpr int BOX_BYTES = 64 * 64 * 2;  // one MN-major box: 64 elements x 64 K rows
 
 enum Mode { MODE_RECOMP = 0, MODE_DSILU = 1, MODE_DX = 2, MODE_WGRAD = 3 };
 
@@ -80,6 +99,7 @@ struct GroupDev {
 struct __align__(64) Params {
     CUtensorMap a_map[2];
     CUtensorMap b_map[2];
+    CUtensorMap c_map[2][2];       // outputs out0 / out1 of each group, for TMA stores
     GroupDev g[2];
     int tiles0, tiles_total;       // K-ragged schedule (host-known)
     int32_t* status;
@@ -88,10 +108,15 @@ struct __align__(64) Params {
 
 struct Smem {
     static constexpr int A_BYTES = BM * BK * 2;
-    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int B_BYTES = BN_HALF * BK * 2;
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-    static constexpr int OFF_BAR = OFF_B + STAGES * B_BYTES;
+    // per epilogue warp two staging buffers of one 32 x 32 output chunk
+    // (fp32: a 4 KB box in the 128-byte swizzle; bf16: 2 KB boxes in the
+    // 64-byte swizzle, two of them for the recompute's two outputs)
+    static constexpr int STG_BYTES = 4096;
+    static constexpr int OFF_STAGE = OFF_B + STAGES * B_BYTES;
+    static constexpr int OFF_BAR = OFF_STAGE + EPI_WARPS * 2 * STG_BYTES;
     static constexpr int N_BARS = 2 * STAGES + 2 * ACC_BUFS + 1;
     static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
     static constexpr int OFF_SEG = OFF_MISC + 16;
@@ -99,9 +124,11 @@ struct Smem {
     static constexpr int TOTAL = OFF_SEG + SEG_INTS * 4;
     static constexpr int ALLOC = TOTAL + 1024;
 };
-static_assert(Smem::A_BYTES == 2 * BOX_BYTES && Smem::B_BYTES == 4 * BOX_BYTES, "box layout");
+static_assert(Smem::A_BYTES == 2 * BOX_BYTES && Smem::B_BYTES == 2 * BOX_BYTES, "box layout");
 static_assert(Smem::OFF_B % 1024 == 0 && Smem::A_BYTES % 1024 == 0 && Smem::B_BYTES % 1024 == 0,
               "stages start on 1024-byte swizzle atoms");
+static_assert(Smem::OFF_STAGE % 1024 == 0 && Smem::STG_BYTES % 1024 == 0,
+              "staging boxes start on 1024-byte swizzle atoms");
 static_assert(Smem::ALLOC <= 227 * 1024, "shared memory budget");
 
 // Shared-memory descriptor of an MN-major operand in the 128-byte swizzled
@@ -121,7 +148,8 @@ __device__ __forceinline__ uint64_t smem_desc_mn_sw128(const void* tile, uint32_
 
 __device__ __forceinline__ int cdiv(int a, int b) { return (a + b - 1) / b; }
 
-// M-ragged segment table (shared memory).
+// M-ragged segment table (shared memory); a segment's tiles are its pairs of
+// m-tiles times its n-tiles.
 struct SegTable {
     int* start;   // first tile of each segment; start[nseg] = total
     int* rows;
@@ -149,7 +177,7 @@ __device__ int build_seg_table(const Params& p, SegTable& t) {
         t.crow[s] = g.c_row_base + (g.seg ? lo : i * g.c_mat_rows);
         t.ccol[s] = i * g.c_col_stride;
         t.mat[s] = (gi << 16) | i;
-        t.start[s + 1] = cdiv(rows, BM) * cdiv(g.N, BN);
+        t.start[s + 1] = cdiv(cdiv(rows, BM), 2) * cdiv(g.N, BN);
     }
     __syncthreads();
     if (warp == 0) {
@@ -170,19 +198,23 @@ __device__ int build_seg_table(const Params& p, SegTable& t) {
     return nseg;
 }
 
+// One pair tile as seen by CTA `rank`.
 struct Tile {
     int grp, mat;
-    int m0;          // K-ragged: first output row (of M); M-ragged: 0
-    int rows_ok;     // valid output rows of the tile (<= 128)
-    int a_row;       // M-ragged: first A row; K-ragged: first K row (A and B)
-    int n0;
+    bool m128;       // odd last m-tile: an M = 128 pair MMA, 64 rows per CTA
+    bool n128;       // last n-tile with at most 128 valid columns: an N = 128 pair MMA
+    int m0;          // K-ragged: this CTA's first output row (of M)
+    int rows_ok;     // valid output rows of this CTA (<= 128, <= 64 with m128)
+    int a_row;       // M-ragged: this CTA's first A row; K-ragged: first K row (A and B)
+    int n0;          // first output column of the pair tile
     int ksteps, kblocks;
-    long long c_off; // element offset of the tile's (row 0, column n0) in out0 / out1 / aux
+    long long c_off; // element offset of this CTA's (row 0, column n0) in out0 / out1 / aux
     int ldc;
+    int crow, ccol;  // the same as coordinates of the output's 2-D tensor map
 };
 
 template <bool KRAG>
-__device__ __forceinline__ Tile decode(int tile, const Params& p, const SegTable& t, int nseg) {
+__device__ __forceinline__ Tile decode(int tile, const Params& p, const SegTable& t, int nseg, int rank) {
     Tile ti;
     if constexpr (!KRAG) {
         int lo = 0, hi = nseg - 1;
@@ -191,29 +223,34 @@ __device__ __forceinline__ Tile decode(int tile, const Params& p, const SegTable
             if (t.start[mid] <= tile) lo = mid; else hi = mid - 1;
         }
         const int s = lo, local = tile - t.start[s];
-        const int mt_n = cdiv(t.rows[s], BM);
-        const int nt = local / mt_n, mt = local % mt_n;
+        const int mt_n = cdiv(t.rows[s], BM), mg_n = cdiv(mt_n, 2);
+        const int nt = local / mg_n, mg = local % mg_n;
         ti.grp = t.mat[s] >> 16;
         ti.mat = t.mat[s] & 0xFFFF;
         const GroupDev& g = p.g[ti.grp];
+        ti.m128 = (2 * mg + 1 == mt_n);
+        const int off = mg * 2 * BM + rank * (ti.m128 ? BM / 2 : BM);
         ti.m0 = 0;
-        ti.rows_ok = min(BM, t.rows[s] - mt * BM);
-        ti.a_row = t.arow[s] + mt * BM;
+        ti.rows_ok = min(ti.m128 ? BM / 2 : BM, t.rows[s] - off);
+        ti.a_row = t.arow[s] + off;
         ti.n0 = nt * BN;
         ti.ksteps = g.K / 16;
         ti.ldc = g.ldc;
-        ti.c_off = static_cast<long long>(t.crow[s] + mt * BM) * g.ldc + t.ccol[s] + ti.n0;
+        ti.crow = t.crow[s] + off;
+        ti.ccol = t.ccol[s] + ti.n0;
+        ti.n128 = !ti.m128 && g.N - ti.n0 <= BN_HALF;
     } else {
         const int gi = tile >= p.tiles0 ? 1 : 0;
         const GroupDev& g = p.g[gi];
         const int local = tile - (gi ? p.tiles0 : 0);
-        const int mt_n = cdiv(g.M, BM), nt_n = cdiv(g.N, BN);
-        const int mat = local / (mt_n * nt_n), r = local % (mt_n * nt_n);
-        const int nt = r / mt_n, mt = r % mt_n;
+        const int mt_n = cdiv(g.M, BM), mg_n = cdiv(mt_n, 2), nt_n = cdiv(g.N, BN);
+        const int mat = local / (mg_n * nt_n), r = local % (mg_n * nt_n);
+        const int nt = r / mg_n, mg = r % mg_n;
         ti.grp = gi;
         ti.mat = mat;
-        ti.m0 = mt * BM;
-        ti.rows_ok = min(BM, g.M - ti.m0);
+        ti.m128 = (2 * mg + 1 == mt_n);
+        ti.m0 = mg * 2 * BM + rank * (ti.m128 ? BM / 2 : BM);
+        ti.rows_ok = min(ti.m128 ? BM / 2 : BM, g.M - ti.m0);
         int lo, cnt;
         if (g.seg) { lo = g.seg[mat]; cnt = g.seg[mat + 1] - lo; }
         else { lo = mat * g.a_mat_stride; cnt = g.fixed; }
@@ -221,8 +258,11 @@ __device__ __forceinline__ Tile decode(int tile, const Params& p, const SegTable
         ti.n0 = nt * BN;
         ti.ksteps = cdiv(cnt, 16);
         ti.ldc = g.ldc;
-        ti.c_off = static_cast<long long>(mat) * g.c_mat_elems + static_cast<long long>(ti.m0) * g.ldc + ti.n0;
+        ti.crow = mat * g.M + ti.m0;     // the matrices' outputs stacked as rows (c_mat_elems = M * ldc)
+        ti.ccol = ti.n0;
+        ti.n128 = !ti.m128 && g.N - ti.n0 <= BN_HALF;
     }
+    ti.c_off = static_cast<long long>(ti.crow) * ti.ldc + ti.ccol;
     ti.kblocks = cdiv(ti.ksteps, 4);
     return ti;
 }
@@ -262,11 +302,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
     SegTable seg(reinterpret_cast<int*>(smem + L::OFF_SEG));
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = cluster_ctarank();          // 0: issues the MMAs of the pair
+    const int pair_id = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
 
-    if (warp == 0) tmem_alloc<TMEM_COLS>(tmem_slot);
+    if (warp == 0) tmem_alloc_pair<TMEM_COLS>(tmem_slot);
     if (warp == 1 && lane == 0) {
         for (int i = 0; i < STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-        for (int i = 0; i < ACC_BUFS; ++i) { mbar_init(&accf[i], 1); mbar_init(&acce[i], EPI_THREADS); }
+        for (int i = 0; i < ACC_BUFS; ++i) { mbar_init(&accf[i], 1); mbar_init(&acce[i], 2 * EPI_WARPS); }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -281,69 +323,74 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
     if constexpr (!TR::krag) nseg = build_seg_table(p, seg);
     tc_fence_before();
     __syncthreads();
+    cluster_sync();                                   // barriers of both CTAs initialised
     tc_fence_after();
     if constexpr (!TR::krag) total_tiles = seg.start[nseg];
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
-        // ================= TMA producer
+        // ================= TMA producer (both CTAs)
         if (lane == 0) {
-            int stage = 0, issued = 0;
+            int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-                const Tile ti = decode<TR::krag>(tile, p, seg, nseg);
+            for (int tile = pair_id; tile < total_tiles && ok; tile += n_pairs) {
+                const Tile ti = decode<TR::krag>(tile, p, seg, nseg, static_cast<int>(rank));
                 const GroupDev& g = p.g[ti.grp];
                 const void* amap = &p.a_map[ti.grp];
                 const void* bmap = &p.b_map[ti.grp];
                 const int bz = g.b_z_mat ? ti.mat : 0;
-                const int bcol = ti.n0 + (TR::krag ? ti.mat * g.b_col_stride : 0);
+                // this CTA's B rows (K-major) or columns (MN-major): half of
+                // the pair's 256, or 64 of an N = 128 tile (whose box reads 128)
+                const int bhalf = ti.n0 + static_cast<int>(rank) * (ti.n128 ? BN_HALF / 2 : BN_HALF);
+                const int bcol = bhalf + (TR::krag ? ti.mat * g.b_col_stride : 0);
                 for (int kb = 0; kb < ti.kblocks; ++kb) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&full[stage], L::A_BYTES + L::B_BYTES);
+                    const uint32_t bar0 = mapa_shared(smem_u32(&full[stage]), 0);
+                    if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (L::A_BYTES + L::B_BYTES));
                     uint8_t* sa = smem + L::OFF_A + stage * L::A_BYTES;
                     uint8_t* sb = smem + L::OFF_B + stage * L::B_BYTES;
                     const int k0 = kb * BK;
                     if constexpr (TR::a_mn) {
-                        tma_load_2d(sa, amap, &full[stage], ti.m0, ti.a_row + k0);
-                        tma_load_2d(sa + BOX_BYTES, amap, &full[stage], ti.m0 + 64, ti.a_row + k0);
+                        tma_load_2d_pair(sa, amap, bar0, ti.m0, ti.a_row + k0);
+                        tma_load_2d_pair(sa + BOX_BYTES, amap, bar0, ti.m0 + 64, ti.a_row + k0);
                     } else {
-                        tma_load_2d(sa, amap, &full[stage], k0, ti.a_row);
+                        tma_load_2d_pair(sa, amap, bar0, k0, ti.a_row);
                     }
                     if constexpr (TR::b_mn) {
                         const int krow = TR::krag ? ti.a_row + k0 : k0;
-#pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            tma_load_3d(sb + j * BOX_BYTES, bmap, &full[stage], bcol + 64 * j, krow, bz);
+                        tma_load_3d_pair(sb, bmap, bar0, bcol, krow, bz);
+                        tma_load_3d_pair(sb + BOX_BYTES, bmap, bar0, bcol + 64, krow, bz);
                     } else {
-                        tma_load_3d(sb, bmap, &full[stage], k0, ti.n0, bz);
+                        tma_load_3d_pair(sb, bmap, bar0, k0, bhalf, bz);
                     }
-                    ++issued;
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
             if (!ok) {
-                int s = stage;
-                uint32_t ph = phase;
-                const int pending = issued < STAGES ? issued : STAGES;
-                for (int i = 0; i < pending; ++i) {
-                    if (--s < 0) { s = STAGES - 1; ph ^= 1u; }
-                    volatile int no_abort = 0;
-                    mbar_wait_bounded(&full[s], ph, &no_abort, nullptr, kDrainTimeoutNs);
-                }
+                // unwinding: copies still in flight land within microseconds
+                const uint64_t t0 = global_timer_ns();
+                while (global_timer_ns() - t0 < 100000ull) { }
             }
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ================= MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc = make_idesc(1, BM, BN) | (TR::a_mn ? (1u << 15) : 0u) |
-                                       (TR::b_mn ? (1u << 16) : 0u);
+        // ================= MMA issuer (first CTA of the pair)
+        if (rank == 0 && lane == 0) {
+            constexpr uint32_t tbits = (TR::a_mn ? (1u << 15) : 0u) | (TR::b_mn ? (1u << 16) : 0u);
+            constexpr uint32_t idesc256 = make_idesc(1, 2 * BM, BN) | tbits;
+            constexpr uint32_t idesc128 = make_idesc(1, BM, BN) | tbits;
+            constexpr uint32_t idesc256n = make_idesc(1, 2 * BM, BN_HALF) | tbits;
+            // K step of 16: 32 bytes along a K-major row, or 16 rows (2048
+            // bytes) of an MN-major block; descriptor units of 16 B
+            constexpr uint64_t a_step = TR::a_mn ? 128 : 2;
+            constexpr uint64_t b_step = TR::b_mn ? 128 : 2;
             int stage = 0, abuf = 0;
             uint32_t phase = 0, aphase = 0;
             bool ok = true, issued_any = false;
-            for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-                const Tile ti = decode<TR::krag>(tile, p, seg, nseg);
+            for (int tile = pair_id; tile < total_tiles && ok; tile += n_pairs) {
+                const Tile ti = decode<TR::krag>(tile, p, seg, nseg, 0);
+                const uint32_t idesc = ti.m128 ? idesc128 : (ti.n128 ? idesc256n : idesc256);
                 if (!mbar_wait_bounded(&acce[abuf], aphase ^ 1u, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(abuf * BN);
@@ -354,49 +401,82 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
                     const uint8_t* sb = smem + L::OFF_B + stage * L::B_BYTES;
                     const uint64_t adesc = TR::a_mn ? smem_desc_mn_sw128(sa, BOX_BYTES) : smem_desc_k_sw128(sa);
                     const uint64_t bdesc = TR::b_mn ? smem_desc_mn_sw128(sb, BOX_BYTES) : smem_desc_k_sw128(sb);
-                    // K step of 16: 32 bytes along a K-major row, or 16 rows
-                    // (2048 bytes) of an MN-major block; descriptor units of 16 B
-                    constexpr uint64_t a_step = TR::a_mn ? 128 : 2;
-                    constexpr uint64_t b_step = TR::b_mn ? 128 : 2;
                     const int steps = min(4, ti.ksteps - kb * 4);
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
                         if (k < steps)
-                            umma_f16(d_tmem, adesc + a_step * k, bdesc + b_step * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                            umma_f16_pair(d_tmem, adesc + a_step * k, bdesc + b_step * k, idesc,
+                                          (kb > 0 || k > 0) ? 1u : 0u);
                     issued_any = true;
-                    umma_commit(&empty[stage]);
+                    umma_commit_pair(&empty[stage], 0x3);   // stage free in both CTAs
                     if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
-                umma_commit(&accf[abuf]);
+                umma_commit_pair(&accf[abuf], 0x3);         // accumulator ready in both CTAs
                 if (++abuf == ACC_BUFS) { abuf = 0; aphase ^= 1u; }
             }
             if (!ok && issued_any) {
-                umma_commit(drain);
+                umma_commit_pair(drain, 0x1);
                 volatile int no_abort = 0;
                 mbar_wait_bounded(drain, 0, &no_abort, nullptr, kDrainTimeoutNs);
             }
         }
         __syncwarp();
     } else {
-        // ================= epilogue (warps 2..9; TMEM lane quadrant = warp % 4)
+        // ================= epilogue (warps 2..9, both CTAs; TMEM lane quadrant = warp % 4)
         const int quad = warp & 3;
         const int half = (warp - 2) >> 2;
-        const int r_local = quad * 32 + lane;
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+        // A chunk of 32 rows x 32 columns whose rows all lie in the tile's
+        // valid rows leaves through shared memory and a TMA store: the warp
+        // writes it into one of its two staging buffers (fp32 rows of 128
+        // bytes, 16-byte chunk q at q ^ (row & 7); bf16 rows of 64 bytes,
+        // chunk q at q ^ ((row >> 1) & 3): the swizzles of the boxes, which
+        // also spread the writes over the banks) and one lane stores it.  A
+        // buffer is rewritten only after the store issued from it two chunks
+        // earlier has read it.  Other rows are stored by their threads.
+        uint8_t* stg = smem + L::OFF_STAGE + (warp - 2) * 2 * L::STG_BYTES;
+        int sbuf = 0;
+        auto stage_begin = [&]() -> uint8_t* {
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+            return stg + sbuf * L::STG_BYTES;
+        };
+        auto stage_end = [&](const void* map0, const void* map1, int x, int y) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_2d(map0, stg + sbuf * L::STG_BYTES, x, y);
+                if (map1) tma_store_2d(map1, stg + sbuf * L::STG_BYTES + 2048, x, y);
+                bulk_commit();
+            }
+            sbuf ^= 1;
+        };
         int abuf = 0;
         uint32_t aphase = 0;
-        for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-            const Tile ti = decode<TR::krag>(tile, p, seg, nseg);
+        for (int tile = pair_id; tile < total_tiles; tile += n_pairs) {
+            const Tile ti = decode<TR::krag>(tile, p, seg, nseg, static_cast<int>(rank));
             const GroupDev& g = p.g[ti.grp];
-            const bool row_ok = r_local < ti.rows_ok;
+            // M = 256: quadrant = 32 rows, warp half = 128 columns (4 chunks);
+            // M = 128: quadrants 0, 1 = rows 0..63 of columns 0..127,
+            // quadrants 2, 3 = the same rows of columns 128..255, warp half =
+            // 64 columns; N = 128: quadrant = 32 rows, warp half = 64 columns
+            const int r_row0 = ti.m128 ? (quad & 1) * 32 : quad * 32;   // the warp's first row
+            const int r_loc = r_row0 + lane;
+            const int n_base = (ti.m128 && quad >= 2) ? BN_HALF : 0;
+            const bool narrow = ti.m128 || ti.n128;
+            const int chunk0 = narrow ? half * 2 : half * 4;
+            const int n_iter = narrow ? 1 : 2;
+            const bool row_ok = r_loc < ti.rows_ok;
+            const bool full_rows = ti.rows_ok >= r_row0 + 32;            // warp-uniform
             const int n_valid = g.N - ti.n0;
+            const bool f32_out = (MODE == MODE_WGRAD) || (MODE == MODE_DX && !g.out_bf16);
             if (!warp_wait(&accf[abuf], aphase, abort_flag, p.status, p.timeout_ns, lane)) break;
             tc_fence_after();
-            const long long row_off = ti.c_off + static_cast<long long>(r_local) * ti.ldc;
+            const long long row_off = ti.c_off + static_cast<long long>(r_loc) * ti.ldc;
 #pragma unroll 1
-            for (int cc = 0; cc < 2; ++cc) {
-                const int c0 = half * 4 + cc * 2;
+            for (int cc = 0; cc < n_iter; ++cc) {
+                const int c0 = chunk0 + cc * 2;
                 uint32_t r[2][32];
                 if (ti.ksteps > 0) {
                     tmem_ld_32x32b_x32(lane_base + static_cast<uint32_t>(abuf * BN + c0 * 32), r[0]);
@@ -409,12 +489,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
                 }
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
-                    const int c = c0 + u;
-                    if (!row_ok || c * 32 >= n_valid) continue;
-                    const long long off = row_off + c * 32;
+                    const int col = n_base + (c0 + u) * 32;            // output column within the tile
+                    if (col >= n_valid) continue;                      // warp-uniform
+                    if (!full_rows && !row_ok) continue;
+                    const long long off = row_off + col;
+                    uint32_t o0[16], o1[16];                           // bf16 results, two per word
                     if constexpr (MODE == MODE_RECOMP) {
-                        const float* bias = g.bias + static_cast<long long>(ti.mat) * g.N + ti.n0 + c * 32;
-                        uint32_t ph[16], pd[16];
+                        const float* bias = g.bias + static_cast<long long>(ti.mat) * g.N + ti.n0 + col;
 #pragma unroll
                         for (int j4 = 0; j4 < 8; ++j4) {
                             const float4 b4 = __ldg(reinterpret_cast<const float4*>(bias) + j4);
@@ -422,71 +503,94 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
                             const float v1 = __uint_as_float(r[u][4 * j4 + 1]) + b4.y;
                             const float v2 = __uint_as_float(r[u][4 * j4 + 2]) + b4.z;
                             const float v3 = __uint_as_float(r[u][4 * j4 + 3]) + b4.w;
-                            ph[2 * j4] = pack_bf16x2(silu_fast(v0), silu_fast(v1));
-                            ph[2 * j4 + 1] = pack_bf16x2(silu_fast(v2), silu_fast(v3));
-                            pd[2 * j4] = pack_bf16x2(dsilu_fast(v0), dsilu_fast(v1));
-                            pd[2 * j4 + 1] = pack_bf16x2(dsilu_fast(v2), dsilu_fast(v3));
-                        }
-                        uint4* dh = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out0) + off);
-                        uint4* dd = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out1) + off);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            dh[q] = make_uint4(ph[4 * q], ph[4 * q + 1], ph[4 * q + 2], ph[4 * q + 3]);
-                            dd[q] = make_uint4(pd[4 * q], pd[4 * q + 1], pd[4 * q + 2], pd[4 * q + 3]);
+                            o0[2 * j4] = pack_bf16x2(silu_fast(v0), silu_fast(v1));
+                            o0[2 * j4 + 1] = pack_bf16x2(silu_fast(v2), silu_fast(v3));
+                            o1[2 * j4] = pack_bf16x2(dsilu_fast(v0), dsilu_fast(v1));
+                            o1[2 * j4 + 1] = pack_bf16x2(dsilu_fast(v2), dsilu_fast(v3));
                         }
                     } else if constexpr (MODE == MODE_DSILU) {
                         const uint4* sp = reinterpret_cast<const uint4*>(g.aux + off);
-                        uint32_t po[16];
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             const uint4 s4 = __ldg(sp + q);
                             const uint32_t sw[4] = {s4.x, s4.y, s4.z, s4.w};
 #pragma unroll
                             for (int w = 0; w < 4; ++w) {
-                                const __nv_bfloat162 s2 = *reinterpret_cast<const __nv_bfloat162*>(&sw[w]);
-                                const float2 sf = __bfloat1622float2(s2);
+                                const float2 sf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sw[w]));
                                 const int j = 8 * q + 2 * w;
-                                po[4 * q + w] = pack_bf16x2(__uint_as_float(r[u][j]) * sf.x,
+                                o0[4 * q + w] = pack_bf16x2(__uint_as_float(r[u][j]) * sf.x,
                                                             __uint_as_float(r[u][j + 1]) * sf.y);
                             }
                         }
-                        uint4* dz = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out0) + off);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) dz[q] = make_uint4(po[4 * q], po[4 * q + 1], po[4 * q + 2], po[4 * q + 3]);
-                    } else if (MODE == MODE_DX && g.out_bf16) {
-                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out0) + off);
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            dst[q] = make_uint4(
-                                pack_bf16x2(__uint_as_float(r[u][8 * q + 0]), __uint_as_float(r[u][8 * q + 1])),
-                                pack_bf16x2(__uint_as_float(r[u][8 * q + 2]), __uint_as_float(r[u][8 * q + 3])),
-                                pack_bf16x2(__uint_as_float(r[u][8 * q + 4]), __uint_as_float(r[u][8 * q + 5])),
-                                pack_bf16x2(__uint_as_float(r[u][8 * q + 6]), __uint_as_float(r[u][8 * q + 7])));
                     } else {
+#pragma unroll
+                        for (int w = 0; w < 16; ++w)
+                            o0[w] = pack_bf16x2(__uint_as_float(r[u][2 * w]), __uint_as_float(r[u][2 * w + 1]));
+                    }
+                    if (full_rows) {
+                        uint8_t* buf = stage_begin();
+                        if (f32_out) {
+                            uint8_t* row = buf + lane * 128;
+#pragma unroll
+                            for (int q = 0; q < 8; ++q)
+                                *reinterpret_cast<uint4*>(row + ((q ^ (lane & 7)) << 4)) =
+                                    make_uint4(r[u][4 * q], r[u][4 * q + 1], r[u][4 * q + 2], r[u][4 * q + 3]);
+                        } else {
+                            uint8_t* row = buf + lane * 64;
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                *reinterpret_cast<uint4*>(row + ((q ^ ((lane >> 1) & 3)) << 4)) =
+                                    make_uint4(o0[4 * q], o0[4 * q + 1], o0[4 * q + 2], o0[4 * q + 3]);
+                            if constexpr (MODE == MODE_RECOMP) {
+#pragma unroll
+                                for (int q = 0; q < 4; ++q)
+                                    *reinterpret_cast<uint4*>(row + 2048 + ((q ^ ((lane >> 1) & 3)) << 4)) =
+                                        make_uint4(o1[4 * q], o1[4 * q + 1], o1[4 * q + 2], o1[4 * q + 3]);
+                            }
+                        }
+                        stage_end(&p.c_map[ti.grp][0], MODE == MODE_RECOMP ? &p.c_map[ti.grp][1] : nullptr,
+                                  ti.ccol + col, ti.crow + r_row0);
+                    } else if (f32_out) {
                         float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out0) + off);
 #pragma unroll
                         for (int q = 0; q < 8; ++q)
                             dst[q] = make_float4(__uint_as_float(r[u][4 * q]), __uint_as_float(r[u][4 * q + 1]),
                                                  __uint_as_float(r[u][4 * q + 2]), __uint_as_float(r[u][4 * q + 3]));
+                    } else {
+                        uint4* d0 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out0) + off);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) d0[q] = make_uint4(o0[4 * q], o0[4 * q + 1], o0[4 * q + 2], o0[4 * q + 3]);
+                        if constexpr (MODE == MODE_RECOMP) {
+                            uint4* d1 = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out1) + off);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) d1[q] = make_uint4(o1[4 * q], o1[4 * q + 1], o1[4 * q + 2], o1[4 * q + 3]);
+                        }
                     }
                 }
             }
             tc_fence_before();
-            mbar_arrive(&acce[abuf]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&acce[abuf]), 0));
             if (++abuf == ACC_BUFS) { abuf = 0; aphase ^= 1u; }
         }
+        // the stores have read their buffers and landed before the CTA exits
+        if (lane == 0) bulk_wait<0>();
+        __syncwarp();
     }
 
+    // ---- teardown: both CTAs are done with tensor memory and with each
+    // other's barriers before either frees or exits
     tc_fence_before();
     __syncthreads();
+    cluster_sync();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc<TMEM_COLS>(tmem_base);
+        tmem_dealloc_pair<TMEM_COLS>(tmem_base);
     }
 }
 
 // Host: device copy of a group and its tensor maps.
-bool fill_group(Params& p, int gi, const BwdGemmGroup& h, bool a_mn, bool b_mn) {
+bool fill_group(Params& p, int gi, const BwdGemmGroup& h, bool a_mn, bool b_mn, bool krag, bool out_f32) {
     GroupDev& d = p.g[gi];
     d.n_mats = h.n_mats;
     if (h.n_mats == 0) return true;
@@ -511,9 +615,19 @@ bool fill_group(Params& p, int gi, const BwdGemmGroup& h, bool a_mn, bool b_mn) 
     d.out_bf16 = h.out_bf16;
     // A (a_rows, a_cols): K-major boxes of 64 K x 128 rows, MN-major boxes of
     // 64 M x 64 K rows; B (b_mats, b_rows, b_cols): K-major boxes of 64 K x
-    // 256 rows of N, MN-major boxes of 64 N x 64 rows of K
+    // 128 rows of N, MN-major boxes of 64 N x 64 rows of K
     if (!encode_tma_2d(&p.a_map[gi], h.A, h.a_rows, h.a_cols, 2, a_mn ? 64 : BM)) return false;
-    if (!encode_tma_3d(&p.b_map[gi], h.B, h.b_mats, h.b_rows, h.b_cols, 2, b_mn ? 64 : BN)) return false;
+    if (!encode_tma_3d(&p.b_map[gi], h.B, h.b_mats, h.b_rows, h.b_cols, 2, b_mn ? 64 : BN_HALF)) return false;
+    // outputs as 2-D (rows, ldc) tensors for 32 x 32 TMA store boxes; the
+    // weight gradients' matrices stacked as rows
+    const int rows = krag ? h.n_mats * h.M : h.c_rows;
+    for (int o = 0; o < 2; ++o) {
+        void* out = o == 0 ? h.out0 : h.out1;
+        if (!out) continue;
+        const bool ok = out_f32 ? encode_tma_2d_store128(&p.c_map[gi][o], out, rows, h.ldc, 4, 32)
+                                : encode_tma_2d_store64(&p.c_map[gi][o], out, rows, h.ldc, 2, 32);
+        if (!ok) return false;
+    }
     return true;
 }
 
@@ -523,11 +637,14 @@ cudaError_t launch_mode(const BwdGemmArgs& a, cudaStream_t st) {
     Params p;
     std::memset(&p, 0, sizeof(p));
     for (int gi = 0; gi < 2; ++gi)
-        if (!fill_group(p, gi, a.g[gi], TR::a_mn, TR::b_mn)) return cudaErrorInvalidValue;
+        if (!fill_group(p, gi, a.g[gi], TR::a_mn, TR::b_mn, TR::krag,
+                        MODE == MODE_WGRAD || (MODE == MODE_DX && !a.g[gi].out_bf16)))
+            return cudaErrorInvalidValue;
     int tiles[2] = {0, 0};
     for (int gi = 0; gi < 2; ++gi) {
         const BwdGemmGroup& g = a.g[gi];
-        if (g.n_mats > 0 && TR::krag) tiles[gi] = g.n_mats * ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN);
+        if (g.n_mats > 0 && TR::krag)
+            tiles[gi] = g.n_mats * (((g.M + BM - 1) / BM + 1) / 2) * ((g.N + BN - 1) / BN);
     }
     p.tiles0 = tiles[0];
     p.tiles_total = tiles[0] + tiles[1];
@@ -536,7 +653,24 @@ cudaError_t launch_mode(const BwdGemmArgs& a, cudaStream_t st) {
     constexpr int smem = Smem::ALLOC;
     cudaError_t e = cudaFuncSetAttribute(bwd_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(bwd_gemm_kernel<MODE>, dim3(device_sm_count()), dim3(NUM_THREADS), smem, st, 1, p);
+    // persistent: as many pairs as fit on the device at once
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(device_sm_count() & ~1);
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&clusters, bwd_gemm_kernel<MODE>, &cfg);
+    if (e != cudaSuccess) return e;
+    if (clusters < 1) return cudaErrorLaunchOutOfResources;
+    return launch_pdl(bwd_gemm_kernel<MODE>, dim3(2 * clusters), dim3(NUM_THREADS), smem, st, 2, p);
 }
 
 }  // namespace

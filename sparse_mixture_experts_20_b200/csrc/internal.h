@@ -161,6 +161,7 @@ cudaError_t launch_wait_selftest(int64_t timeout_ns, int32_t* status, cudaStream
 bool encode_tma_2d(void* map, const void* base, int rows, int K, int elem, int box_rows);
 bool encode_tma_3d(void* map, const void* base, int n_mats, int N, int K, int elem, int box_rows);
 bool encode_tma_2d_store64(void* map, const void* base, int rows, int cols, int elem, int box_rows);
+bool encode_tma_2d_store128(void* map, const void* base, int rows, int cols, int elem, int box_rows);
 int device_sm_count();
 
 // Records a failed CUDA call for moe_last_cuda_error() on this thread.
@@ -189,6 +190,7 @@ struct BwdGemmGroup {
     const void* aux;         // dgrad-SiLU: SiLU'(z) bf16, addressed like out0
     void* out0;
     void* out1;              // recompute: SiLU'(z)
+    int c_rows;              // M-ragged: rows of the output matrices (for their TMA store maps)
     int c_row_base;          // M-ragged: first output row of segment 0 (routed) or of all
     int c_mat_rows;          // fixed segments: output rows between segments
     int c_col_stride;        // M-ragged: output column offset of segment i
