@@ -74,7 +74,7 @@ __all__ = [
     "router_logits", "softmax", "topk_select", "gates_of", "capacity_of",
     "dispatch_plan", "silu", "expert_ffn", "balance_stats", "topk_gap",
     "route", "layer_forward", "to_f64", "expert_weights",
-    "silu_grad", "expert_ffn_backward", "layer_backward",
+    "silu_grad", "expert_ffn_backward", "layer_backward", "layer_backward_sample",
 ]
 
 E4M3_MAX = 448.0
@@ -562,4 +562,102 @@ def layer_backward(shape, inputs, dout: np.ndarray, lam: float = 1.0,
     for k in d_exp:
         res[k] = np.stack(d_exp[k])
     res.update(shared)
+    return res
+
+
+def layer_backward_sample(shape, inputs, dout: np.ndarray, lam: float, routing: dict,
+                          experts, f_idx, c_idx, tokens, fs_idx=None) -> dict:
+    """Selected entries of layer_backward, each computed from the same
+    definitions with only the work it needs, so that layers of full size can
+    be checked:
+      "W1"[e]  dW1[e][f_idx, :]         "b1"[e]  db1[e][f_idx]
+      "W2"[e]  dW2[e][c_idx][:, f_idx]  "b2"[e]  db2[e][c_idx]
+    for each routed expert e in `experts`,
+      "Ws1"[s] dWs1[s][fs_idx, :]       "bs1"[s] dbs1[s][fs_idx]
+      "Ws2"[s] dWs2[s][c_idx][:, fs_idx] "bs2"[s] dbs2[s][c_idx]
+    for every shared expert s, and "x" = dx[tokens].  routing: the output of
+    route() for the whole batch (the balance term needs f over all tokens).
+    The derivative read is layer_backward's: a kept slot's expert sees
+    dy = g dout_t; a token's dx is its router part dl_t W_r, its kept slots'
+    W1^T dz, g dout_t for slots passed through and its shared experts'."""
+    if shape.dtype == 2:
+        raise ValueError("layer_backward_sample covers the fp32 and bf16 workloads")
+    rt = routing
+    T, K, N_r = shape.T, shape.top_k, shape.n_routed
+    f_idx, c_idx = np.asarray(f_idx), np.asarray(c_idx)
+    fs_idx = f_idx if fs_idx is None else np.asarray(fs_idx)
+    s, idx, g = rt["s"], rt["idx"].astype(np.int64), rt["gates"]
+    slot_row = rt["plan"]["slot_row"]
+    passthrough = getattr(shape, "overflow_mode", 0) == 1
+
+    def xrow(ts):
+        return to_f64(inputs["x"][np.asarray(ts)]) if len(ts) else np.zeros((0, shape.d_model))
+
+    def drow(ts):
+        return np.asarray(dout, np.float64)[np.asarray(ts)]
+
+    res = {k: {} for k in ("W1", "b1", "W2", "b2", "Ws1", "bs1", "Ws2", "bs2")}
+    for e in experts:
+        W1, b1, W2, b2 = expert_weights(inputs, "W", e, False)
+        slots = [(t, k) for t in range(T) for k in range(K) if idx[t, k] == e and slot_row[t, k] >= 0]
+        tt = [t for t, _ in slots]
+        xr = xrow(tt)
+        dy = np.array([g[t, k] for t, k in slots])[:, None] * drow(tt) if slots else np.zeros((0, shape.d_model))
+        z = xr @ W1[f_idx].T + b1[f_idx][None, :]
+        dz = (dy @ W2[:, f_idx]) * silu_grad(z)
+        res["W1"][e] = dz.T @ xr
+        res["b1"][e] = dz.sum(axis=0)
+        res["W2"][e] = dy[:, c_idx].T @ silu(z)
+        res["b2"][e] = dy[:, c_idx].sum(axis=0)
+    if shape.n_shared > 0:
+        xa = to_f64(inputs["x"])
+        da = np.asarray(dout, np.float64)
+        for si in range(shape.n_shared):
+            W1, b1, W2, b2 = expert_weights(inputs, "Ws", si, False)
+            z = xa @ W1[fs_idx].T + b1[fs_idx][None, :]
+            dz = (da @ W2[:, fs_idx]) * silu_grad(z)
+            res["Ws1"][si] = dz.T @ xa
+            res["bs1"][si] = dz.sum(axis=0)
+            res["Ws2"][si] = da[:, c_idx].T @ silu(z)
+            res["bs2"][si] = da[:, c_idx].sum(axis=0)
+    # dx of the chosen tokens: each expert's weights are widened once for all
+    # the chosen tokens' slots it serves
+    W_r = to_f64(inputs["W_r"])
+    f = rt["f"]
+    tokens = [int(t) for t in tokens]
+    xt_all = {t: to_f64(inputs["x"][t]) for t in tokens}
+    dt_all = {t: np.asarray(dout[t], np.float64) for t in tokens}
+    a = {t: np.zeros(K) for t in tokens}
+    v = {t: np.zeros(shape.d_model) for t in tokens}
+    by_expert = {}
+    for t in tokens:
+        for k in range(K):
+            if slot_row[t, k] >= 0:
+                by_expert.setdefault(int(idx[t, k]), []).append((t, k))
+            elif passthrough:
+                a[t][k] = float(dt_all[t] @ xt_all[t])
+                v[t] += g[t, k] * dt_all[t]
+    for e, slots_e in by_expert.items():
+        W1, b1, W2, b2 = expert_weights(inputs, "W", e, False)
+        for t, k in slots_e:
+            xt, dt = xt_all[t], dt_all[t]
+            a[t][k] = float(dt @ expert_ffn(xt[None, :], W1, b1, W2, b2)[0])
+            z = W1 @ xt + b1
+            v[t] += ((W2.T @ (g[t, k] * dt)) * silu_grad(z)) @ W1
+    for si in range(shape.n_shared):
+        W1, b1, W2, b2 = expert_weights(inputs, "Ws", si, False)
+        for t in tokens:
+            z = W1 @ xt_all[t] + b1
+            v[t] += ((W2.T @ dt_all[t]) * silu_grad(z)) @ W1
+    dx = []
+    for t in tokens:
+        S = s[t, idx[t]].sum()
+        ds = np.zeros(N_r)
+        common = float((a[t] * g[t]).sum())
+        for k in range(K):
+            ds[idx[t, k]] += (a[t][k] - common) / S
+        ds += lam * shape.alpha * N_r * f / T
+        dl = s[t] * (ds - float((s[t] * ds).sum()))
+        dx.append(v[t] + dl @ W_r)
+    res["x"] = np.array(dx).reshape(len(tokens), shape.d_model)
     return res

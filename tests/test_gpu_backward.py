@@ -15,7 +15,7 @@ tokens whose terms nearly cancel sits far below the typical row, and the
 bf16 roundings of its operands set its error on the typical row's scale).  The bf16 cases span several
 128-row and 256-column tiles with ragged tails, experts no token reaches
 (their gradients must be exact zeros) and shared experts of a width that is
-not a multiple of the tile.  Collected last."""
+not a multiple of the tile."""
 import numpy as np
 import pytest
 import torch

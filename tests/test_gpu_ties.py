@@ -6,7 +6,7 @@ The router-weight rows of a set Z of experts are zero and their logit bias is
 products plus +0); every other expert gets a bias of -50 and is never
 chosen.  Top-K must then be the K lowest indices of Z in ascending order,
 with equal gates 1/K -- on the small router (N_r = 8) and the tensor-core
-router (N_r = 64).  Collected last."""
+router (N_r = 64)."""
 import numpy as np
 import pytest
 import torch

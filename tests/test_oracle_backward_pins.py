@@ -172,3 +172,41 @@ def test_planted_mistakes_fail_the_central_differences(monkeypatch):
     monkeypatch.setattr(O, "layer_backward", no_balance)
     with pytest.raises(AssertionError):
         _fd_check(sh, seed=19, keys=["W_r"])
+
+
+@pytest.mark.parametrize("case", ["shared-capacity-pass", "bias-f32"])
+def test_sampled_backward_equals_the_full_one(case):
+    """layer_backward_sample (the full-size checks' oracle) gives exactly the
+    selected entries of layer_backward, which the finite differences above
+    pin: selected weight-gradient rows and blocks, bias entries and dx rows."""
+    if case == "shared-capacity-pass":
+        sh = MoEShape("sb1", 40, 64, 6, 2, 128, n_shared=2, d_ff_shared=64, capacity_factor=0.6,
+                      overflow_mode=1, dtype=1)
+    else:
+        sh = MoEShape("sb2", 30, 64, 5, 2, 128, zipf_logit_bias=True, dtype=DTYPE_F32)
+    inp = _inputs64(sh, 3)
+    rng = np.random.default_rng(11)
+    dout = rng.standard_normal((sh.T, sh.d_model))
+    rt = O.route(sh, inp)
+    full = O.layer_backward(sh, inp, dout, lam=LAM, routing=rt)
+    experts, f_idx, c_idx, tokens = [0, 2, sh.n_routed - 1], [0, 5, 127], [1, 63], [0, 7, sh.T - 1]
+    fs_idx = [0, 63]
+    smp = O.layer_backward_sample(sh, inp, dout, LAM, rt, experts, f_idx, c_idx, tokens, fs_idx=fs_idx)
+
+    def close(a, b):
+        assert np.allclose(a, b, rtol=1e-11, atol=1e-11 * (1.0 + np.abs(b).max()))
+
+    for e in experts:
+        close(smp["W1"][e], full["W1"][e][f_idx])
+        close(smp["b1"][e], full["b1"][e][f_idx])
+        close(smp["W2"][e], full["W2"][e][np.ix_(c_idx, f_idx)])
+        close(smp["b2"][e], full["b2"][e][c_idx])
+    for si in range(sh.n_shared):
+        close(smp["Ws1"][si], full["Ws1"][si][fs_idx])
+        close(smp["bs1"][si], full["bs1"][si][fs_idx])
+        close(smp["Ws2"][si], full["Ws2"][si][np.ix_(c_idx, fs_idx)])
+        close(smp["bs2"][si], full["bs2"][si][c_idx])
+    close(smp["x"], full["x"][tokens])
+    # the case reaches a dropped slot passed through and an expert with several rows
+    if case == "shared-capacity-pass":
+        assert (rt["plan"]["slot_row"] == -1).any()
