@@ -230,6 +230,38 @@ MOE_EXPORT int moe_expert_ffn(const moe_config* cfg, const void* x, const void* 
                    const void* Ws2, const float* Ws2_scales, const float* bs2,
                    void* y, void* ws, void* stream);
 
+/* ---- stage 3 over caller-made segments (expert parallelism) ----------------
+ * The grouped expert FFN of moe_expert_ffn over n_seg segments of x_rows that
+ * the caller lays out: rows seg_offsets[i] .. seg_offsets[i+1]-1 go through
+ * expert seg_expert[i] (0 <= seg_expert[i] < n_routed), and y row r is the
+ * output of x_rows row r.  Segments may name an expert more than once and in
+ * any order: an expert-parallel rank runs its experts on the rows every
+ * source rank sent it, in the order they arrived (one segment per source rank
+ * and expert), without regrouping them ("エキスパート並列（Expert
+ * Parallelism）" §推論フロー: each GPU computes the tokens routed to the
+ * experts it holds; "DeepSeek DeepEP" §DeepEP とは: FP8 dispatch, the rows
+ * arrive as e4m3 codes with their 1x128 scales).
+ *   cfg         n_routed = the experts held, top_k = 1, T = rows of x_rows and
+ *               y, n_shared = 0, no capacity (capacity_factor 0); d_model,
+ *               d_ff and dtype as the layer's
+ *   x_rows      (T, d_model) fp32 / bf16 rows, or e4m3 codes (FP8)
+ *   x_rows_scales (T, d_model/128) fp32 (FP8), else NULL
+ *   seg_offsets (n_seg+1) int32 device, non-decreasing, seg_offsets[n_seg] <= T
+ *   seg_expert  (n_seg) int32 device; 1 <= n_seg <= 256
+ *   W1 .. b2    the held experts' weights, as moe_expert_ffn
+ *   y           (T, d_model) fp32 (MOE_F32) or bf16; rows outside every
+ *               segment are not written
+ *   ws          moe_workspace_size(cfg) bytes (hidden activations, status word)
+ * A segment whose bounds lie outside [0, T] or whose expert is out of range is
+ * skipped and sets MOE_DEV_BAD_ROUTING in ws's status word.  Other argument
+ * errors return MOE_ERR_INVALID_ARG before anything is enqueued. */
+MOE_EXPORT int moe_expert_ffn_segments(const moe_config* cfg, const void* x_rows,
+                   const float* x_rows_scales, const int32_t* seg_offsets,
+                   const int32_t* seg_expert, int32_t n_seg,
+                   const void* W1, const float* W1_scales, const float* b1,
+                   const void* W2, const float* W2_scales, const float* b2,
+                   void* y, void* ws, void* stream);
+
 /* ---- stage 4: combine ------------------------------------------------------
  * out[t] = sum_{k ascending, slot_row[t,k] >= 0} gates[t,k] * y[slot_row[t,k]]
  *          (+ gates[t,k] * x[t] for slot_row[t,k] == -1 with MOE_OVERFLOW_PASS)

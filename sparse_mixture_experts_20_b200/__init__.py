@@ -38,6 +38,7 @@ EXPORTED = (
     "moe_last_cuda_error", "moe_status_string", "moe_route", "moe_dispatch", "moe_expert_ffn",
     "moe_combine", "moe_balance_stats", "moe_layer_forward", "moe_selftest_wait_timeout",
     "moe_dispatch_noalloc", "moe_kernel_launches", "moe_backward_workspace_size", "moe_layer_backward",
+    "moe_expert_ffn_segments",
 )
 
 
@@ -106,6 +107,7 @@ def lib() -> ctypes.CDLL:
             "moe_kernel_launches": [],
             "moe_backward_workspace_size": [cfgp, ctypes.POINTER(ctypes.c_size_t)],
             "moe_layer_backward": [cfgp, ctypes.c_float, ctypes.POINTER(moe_backward_io), P, P],
+            "moe_expert_ffn_segments": [cfgp, P, P, P, P, ctypes.c_int32] + [P] * 9,
         }
         restype = {"moe_status_string": ctypes.c_char_p, "moe_kernel_launches": ctypes.c_uint64}
         for name, args in sig.items():
@@ -204,6 +206,17 @@ def moe_expert_ffn(cfg, x, x_disp, x_disp_scales, offsets, W1, W1_scales, b1, W2
                                 _p(W1), _p(W1_scales), _p(b1), _p(W2), _p(W2_scales), _p(b2),
                                 _p(Ws1), _p(Ws1_scales), _p(bs1), _p(Ws2), _p(Ws2_scales), _p(bs2),
                                 _p(y), _p(ws), _stream(stream)), "moe_expert_ffn")
+
+
+def moe_expert_ffn_segments(cfg, x_rows, x_rows_scales, seg_offsets, seg_expert, n_seg: int,
+                            W1, W1_scales, b1, W2, W2_scales, b2, y, ws, stream=None):
+    """The grouped expert FFN over caller-made segments: rows seg_offsets[i] ..
+    seg_offsets[i+1]-1 of x_rows through expert seg_expert[i] (cfg: the held
+    experts, top_k 1, T = rows, no shared experts, no capacity)."""
+    _check(lib().moe_expert_ffn_segments(ctypes.byref(cfg), _p(x_rows), _p(x_rows_scales), _p(seg_offsets),
+                                         _p(seg_expert), int(n_seg), _p(W1), _p(W1_scales), _p(b1), _p(W2),
+                                         _p(W2_scales), _p(b2), _p(y), _p(ws), _stream(stream)),
+           "moe_expert_ffn_segments")
 
 
 def moe_combine(cfg, y, gates, slot_row, out, stream=None, x=None):

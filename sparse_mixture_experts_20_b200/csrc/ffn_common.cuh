@@ -3,7 +3,8 @@
 // dispatch offsets, tile decoding, and the host-side parameter fill.
 //
 // Segments: one per routed expert (rows offsets[e] .. offsets[e+1]-1 of A
-// and C), then one per shared expert (fixed_rows rows each).  A segment of
+// and C; with a segment map, segment i holds rows of expert seg_mat[i]), then
+// one per shared expert (fixed_rows rows each).  A segment of
 // `rows` rows has ceil(rows/128) m-tiles and ceil(N/BN) n-tiles; its tiles are
 // numbered n-tile-major with m fastest, so CTAs that run at the same time
 // work on the same weight tile.
@@ -33,6 +34,8 @@ struct GroupDev {
     float* c_scales;          // FP8 first layer (c_rows, N/128)
     int N, K;
     int a_rows;
+    const int32_t* seg_mat;   // routed: weight matrix of each segment, or nullptr
+    int n_weights;            // matrices seg_mat may name
 };
 
 struct __align__(64) TcParams {
@@ -79,9 +82,18 @@ __device__ __forceinline__ int build_seg_table(const TcParams& p, SegTable& t, i
             const GroupDev& g = p.g[0];
             const int o0 = g.offsets[s], o1 = g.offsets[s + 1];
             rows = o1 - o0;
+            if (g.seg_mat) {
+                // caller-made segments: one out of bounds, or naming no
+                // matrix, is skipped and reported
+                const int m = g.seg_mat[s];
+                if (o0 < 0 || rows < 0 || o1 > g.a_rows || m < 0 || m >= g.n_weights) {
+                    rows = 0;
+                    set_device_status(p.status, MOE_DEV_BAD_ROUTING);
+                }
+            }
             arow = g.a_row_base + o0;
             crow = g.c_row_base + o0;
-            packed = s;
+            packed = g.seg_mat ? g.seg_mat[s] : s;     // the segment's weight matrix
             N = g.N;
         } else {
             const GroupDev& g = p.g[1];
@@ -175,8 +187,11 @@ inline bool fill_params(TcParams& p, const GemmArgs& a, int elem, int bn, uint64
         d.N = g.N;
         d.K = g.K;
         d.a_rows = g.a_rows;
+        d.seg_mat = g.seg_mat;
+        d.n_weights = g.n_weights > 0 ? g.n_weights : g.n_mats;
         if (!encode_tma_2d(&p.a_map[gi], g.A, g.a_rows, g.K, elem, BM)) return false;
-        if (!encode_tma_3d(&p.b_map[gi], g.B, g.n_mats, g.N, g.K, elem, bn)) return false;
+        if (!encode_tma_3d(&p.b_map[gi], g.B, g.n_weights > 0 ? g.n_weights : g.n_mats, g.N, g.K, elem, bn))
+            return false;
         if (out_elem > 0 && !encode_tma_2d_store64(&p.c_map[gi], g.C, g.c_rows, g.N, out_elem, 32)) return false;
     }
     p.silu = a.silu;

@@ -20,8 +20,10 @@ constexpr int MAX_SEGS = 256 + 8;
 struct F32Group {
     int n_mats;
     const int32_t* offsets;
+    const int32_t* seg_mat;   // routed: weight matrix of each segment, or nullptr
     int fixed_rows;
     const float* A;
+    int a_rows;
     int a_row_base, a_seg_stride;
     const float* B;
     const float* bias;
@@ -33,6 +35,8 @@ struct F32Group {
 struct F32Params {
     F32Group g[2];
     int silu;
+    int n_weights;            // matrices the routed segment map may name
+    int32_t* status;
 };
 
 __global__ void __launch_bounds__(256)
@@ -46,7 +50,16 @@ ffn_f32_kernel(const __grid_constant__ F32Params p) {
     const int tid = threadIdx.x;
     const int n0segs = p.g[0].n_mats, nseg = n0segs + p.g[1].n_mats;
     for (int s = tid; s < nseg; s += 256) {
-        const int rows = (s < n0segs) ? p.g[0].offsets[s + 1] - p.g[0].offsets[s] : p.g[1].fixed_rows;
+        int rows = (s < n0segs) ? p.g[0].offsets[s + 1] - p.g[0].offsets[s] : p.g[1].fixed_rows;
+        if (s < n0segs && p.g[0].seg_mat) {
+            // caller-made segments: one out of bounds, or naming no matrix,
+            // is skipped and reported
+            const int o0 = p.g[0].offsets[s], m = p.g[0].seg_mat[s];
+            if (o0 < 0 || rows < 0 || o0 + rows > p.g[0].a_rows || m < 0 || m >= p.n_weights) {
+                rows = 0;
+                if (blockIdx.x == 0 && blockIdx.y == 0) set_device_status(p.status, MOE_DEV_BAD_ROUTING);
+            }
+        }
         seg_rows[s] = rows;
     }
     __syncthreads();
@@ -75,7 +88,8 @@ ffn_f32_kernel(const __grid_constant__ F32Params p) {
     }
     const int n0 = blockIdx.y * FBN;
     if (n0 >= g.N) return;
-    const float* Bm = g.B + static_cast<size_t>(mat) * g.N * g.K;
+    const int wmat = (grp == 0 && g.seg_mat) ? g.seg_mat[mat] : mat;    // the segment's weights
+    const float* Bm = g.B + static_cast<size_t>(wmat) * g.N * g.K;
 
     const int ty = tid / 16, tx = tid % 16;
     float acc[4][4] = {};
@@ -107,7 +121,7 @@ ffn_f32_kernel(const __grid_constant__ F32Params p) {
         for (int j = 0; j < 4; ++j) {
             const int n = n0 + tx * 4 + j;
             if (n >= g.N) continue;
-            float v = acc[i][j] + g.bias[static_cast<size_t>(mat) * g.N + n];
+            float v = acc[i][j] + g.bias[static_cast<size_t>(wmat) * g.N + n];
             if (p.silu) v = v / (1.0f + expf(-v));
             g.C[static_cast<size_t>(c_row + r) * g.N + n] = v;
         }
@@ -125,8 +139,10 @@ cudaError_t launch_grouped_ffn_f32(const Dims& dm, const GemmArgs& a, cudaStream
         d.n_mats = s.n_mats;
         if (s.n_mats == 0) continue;
         d.offsets = s.offsets;
+        d.seg_mat = s.seg_mat;
         d.fixed_rows = s.fixed_rows;
         d.A = static_cast<const float*>(s.A);
+        d.a_rows = s.a_rows;
         d.a_row_base = s.a_row_base;
         d.a_seg_stride = s.a_seg_stride;
         d.B = static_cast<const float*>(s.B);
@@ -138,7 +154,15 @@ cudaError_t launch_grouped_ffn_f32(const Dims& dm, const GemmArgs& a, cudaStream
         ntiles = max(ntiles, (s.N + FBN - 1) / FBN);
     }
     p.silu = a.silu;
-    const int mt_bound = (dm.r_cap + FBM - 1) / FBM + dm.E + dm.S * ((dm.T + FBM - 1) / FBM);
+    p.n_weights = a.g[0].n_weights > 0 ? a.g[0].n_weights : a.g[0].n_mats;
+    p.status = a.status;
+    // m-tiles: at most one per 64 rows of the routed rows plus one per segment
+    // (its ragged tail), and those of the fixed segments
+    int mt_bound = 0;
+    if (a.g[0].n_mats > 0) mt_bound += (a.g[0].a_rows + FBM - 1) / FBM + a.g[0].n_mats;
+    if (a.g[1].n_mats > 0) mt_bound += a.g[1].n_mats * ((a.g[1].fixed_rows + FBM - 1) / FBM);
+    if (mt_bound < 1) mt_bound = 1;
+    (void)dm;
     return launch_pdl(ffn_f32_kernel, dim3(mt_bound, ntiles), dim3(256), 0, st, 1, p);
 }
 

@@ -139,6 +139,11 @@ struct GemmGroup {
     // n_fixed segments of fixed_rows rows each.
     const int32_t* offsets; // (n_mats+1) or nullptr for a fixed group
     int fixed_rows;
+    // routed group: segment i uses the weights, biases and scales of matrix
+    // seg_mat[i] (device, n_mats entries) instead of matrix i, among n_weights
+    // matrices (0: n_mats); nullptr: segment i is matrix i
+    const int32_t* seg_mat;
+    int n_weights;
 };
 
 struct GemmArgs {

@@ -147,13 +147,16 @@ RouterScratch router_scratch(void* ws, const WsLayout& L) {
 }
 
 // Builds the two grouped-GEMM launches of the expert FFN and runs them.
+// seg_mat (device, n_seg entries) or nullptr: the routed group is n_seg
+// caller-made segments over x_disp (offsets has n_seg + 1 entries), segment i
+// computed with expert seg_mat[i] of the dm.E held.
 int run_expert_ffn(const Dims& dm, const WsLayout& L, const void* x, const void* x_disp,
                    const float* x_disp_scales, const int32_t* offsets,
                    const void* W1, const float* W1_scales, const float* b1,
                    const void* W2, const float* W2_scales, const float* b2,
                    const void* Ws1, const float* Ws1_scales, const float* bs1,
                    const void* Ws2, const float* Ws2_scales, const float* bs2,
-                   void* y, void* ws, cudaStream_t st) {
+                   void* y, void* ws, cudaStream_t st, const int32_t* seg_mat = nullptr, int n_seg = 0) {
     const bool fp8 = dm.dtype == MOE_FP8_E4M3_BLOCK;
     void* h_r = at<uint8_t>(ws, L.h_r);
     void* h_s = at<uint8_t>(ws, L.h_s);
@@ -172,6 +175,7 @@ int run_expert_ffn(const Dims& dm, const WsLayout& L, const void* x, const void*
         r.B = W1; r.n_mats = dm.E; r.b_scales = W1_scales; r.bias = b1;
         r.C = h_r; r.c_rows = dm.r_cap; r.c_row_base = 0; r.c_scales = h_r_sc;
         r.N = dm.dff; r.K = dm.d; r.offsets = offsets; r.fixed_rows = 0;
+        if (seg_mat) { r.n_mats = n_seg; r.seg_mat = seg_mat; r.n_weights = dm.E; }
     }
     if (dm.S > 0) {
         GemmGroup& s = g1.g[1];
@@ -192,6 +196,7 @@ int run_expert_ffn(const Dims& dm, const WsLayout& L, const void* x, const void*
         r.B = W2; r.n_mats = dm.E; r.b_scales = W2_scales; r.bias = b2;
         r.C = y; r.c_rows = dm.y_rows; r.c_row_base = 0; r.c_scales = nullptr;
         r.N = dm.d; r.K = dm.dff; r.offsets = offsets; r.fixed_rows = 0;
+        if (seg_mat) { r.n_mats = n_seg; r.seg_mat = seg_mat; r.n_weights = dm.E; }
     }
     if (dm.S > 0) {
         GemmGroup& s = g2.g[1];
@@ -388,6 +393,27 @@ int moe_expert_ffn(const moe_config* cfg, const void* x, const void* x_disp, con
     const WsLayout L = ws_layout(dm);
     return run_expert_ffn(dm, L, x, x_disp, x_disp_scales, offsets, W1, W1_scales, b1, W2, W2_scales, b2,
                           Ws1, Ws1_scales, bs1, Ws2, Ws2_scales, bs2, y, ws, static_cast<cudaStream_t>(stream));
+}
+
+int moe_expert_ffn_segments(const moe_config* cfg, const void* x_rows, const float* x_rows_scales,
+                            const int32_t* seg_offsets, const int32_t* seg_expert, int32_t n_seg,
+                            const void* W1, const float* W1_scales, const float* b1, const void* W2,
+                            const float* W2_scales, const float* b2, void* y, void* ws, void* stream) {
+    NvtxRange nvtx("moe_expert_ffn_segments");
+    Dims dm;
+    const int v = validate(cfg, &dm);
+    if (v != MOE_OK) return v;
+    if (dm.S != 0 || dm.K != 1 || dm.capacity >= 0) return MOE_ERR_INVALID_ARG;
+    if (n_seg < 1 || n_seg > 256) return MOE_ERR_INVALID_ARG;
+    if (!seg_expert || !aligned16(seg_expert)) return MOE_ERR_INVALID_ARG;
+    if (!y || !ws || !aligned16(y) || (reinterpret_cast<uintptr_t>(ws) & 255u)) return MOE_ERR_INVALID_ARG;
+    if (!ffn_args_ok(dm, nullptr, x_rows, x_rows_scales, seg_offsets, W1, W1_scales, b1, W2, W2_scales, b2,
+                     nullptr, nullptr, nullptr, nullptr, nullptr, nullptr))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(dm);
+    return run_expert_ffn(dm, L, nullptr, x_rows, x_rows_scales, seg_offsets, W1, W1_scales, b1, W2, W2_scales,
+                          b2, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, y, ws,
+                          static_cast<cudaStream_t>(stream), seg_expert, n_seg);
 }
 
 int moe_combine(const moe_config* cfg, const void* y, const float* gates, const int32_t* slot_row,

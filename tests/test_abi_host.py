@@ -226,3 +226,28 @@ def test_backward_io_binding_names_every_field():
     assert tuple(declared) == M.BACKWARD_IO_FIELDS
     with pytest.raises(KeyError):
         M.backward_io({"not_a_field": None})
+
+
+def test_expert_ffn_segments_rejects_bad_arguments_without_launch():
+    """moe_expert_ffn_segments: a layer with shared experts, top_k != 1, a
+    capacity, no segments or more than 256, a missing segment map or missing
+    FP8 scales are argument errors caught on the host (the fake addresses are
+    never dereferenced)."""
+    L = M.lib()
+    before = M.moe_kernel_launches()
+    p, ws = 0x10000, 0x100000
+
+    def call(cfg, n_seg=4, seg_expert=p, scales=None):
+        return L.moe_expert_ffn_segments(ctypes.byref(cfg), p, scales, p, seg_expert, n_seg, p, scales, p, p,
+                                         scales, p, p, ws, None)
+
+    base = dict(T=64, d_model=128, n_routed=4, top_k=1, d_ff=128)
+    ok = M.make_config(**base)
+    for bad in (dict(n_seg=0), dict(n_seg=257), dict(seg_expert=None), dict(seg_expert=p + 4)):
+        assert call(ok, **bad) == M.MOE_ERR_INVALID_ARG, bad
+    assert call(M.make_config(**dict(base, n_shared=1, d_ff_shared=64))) == M.MOE_ERR_INVALID_ARG
+    assert call(M.make_config(**dict(base, top_k=2))) == M.MOE_ERR_INVALID_ARG
+    assert call(M.make_config(**dict(base, capacity_factor=1.0))) == M.MOE_ERR_INVALID_ARG
+    fp8 = M.make_config(**dict(base, d_model=128, d_ff=256, dtype=M.MOE_FP8_E4M3_BLOCK))
+    assert call(fp8) == M.MOE_ERR_INVALID_ARG                 # FP8 rows without their scales
+    assert M.moe_kernel_launches() == before
