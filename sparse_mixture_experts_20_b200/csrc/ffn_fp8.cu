@@ -522,7 +522,13 @@ cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
 // Weight tiles are 256 wide.  128-wide tiles (FCfg<128>) double the tile
 // count on decode-sized batches, which evens out the last wave, but measured
 // slower on the V3 decode batch (0.293 against 0.269 ms): the per-stage cost
-// of the block-scaled MMA is nearly the same at N = 128 as at N = 256.
+// of the block-scaled MMA is nearly the same at N = 128 as at N = 256.  A
+// 224-wide second layer (d_model = 7168 = 32 x 224; two disjoint accumulators
+// and the scale slots fill the 512 columns, so no tile waits for the
+// previous one's overlapping columns; weight scales picked per row, since a
+// tile then starts inside a 128-row block) passed parity but measured slower
+// on the V3 prefill layer (2.26 against 2.07 ms, same box): the extra tiles
+// cost more than the overlap wait they remove.
 cudaError_t launch_grouped_ffn_fp8(const Dims&, const GemmArgs& a, cudaStream_t st) {
     return a.out_fp8 ? launch_bn<256, true>(a, st) : launch_bn<256, false>(a, st);
 }
