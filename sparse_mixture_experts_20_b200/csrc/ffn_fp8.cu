@@ -528,7 +528,9 @@ cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
 // previous one's overlapping columns; weight scales picked per row, since a
 // tile then starts inside a 128-row block) passed parity but measured slower
 // on the V3 prefill layer (2.26 against 2.07 ms, same box): the extra tiles
-// cost more than the overlap wait they remove.
+// cost more than the overlap wait they remove.  Eight epilogue warps for the
+// second layer (two per lane quadrant, 448 threads, which caps registers at
+// 128 with spills) also measured slower (2.36 against 2.23 ms, same box).
 cudaError_t launch_grouped_ffn_fp8(const Dims&, const GemmArgs& a, cudaStream_t st) {
     return a.out_fp8 ? launch_bn<256, true>(a, st) : launch_bn<256, false>(a, st);
 }
