@@ -37,17 +37,17 @@
 // waits; tcgen05.commit with a CTA mask frees the stage in both CTAs and
 // hands a finished accumulator to both epilogues.
 //
-// Per CTA (320 threads, one CTA per SM): warp 0 TMA producer (ring of 5
-// stages of 16 KB A + 16 KB B: a fifth stage measured 2-3 % faster than four
-// with double-buffered output staging), warp 1 MMA issuer (first CTA of the pair),
+// Per CTA (320 threads, one CTA per SM): warp 0 TMA producer (ring of 6
+// stages of 16 KB A + 16 KB B, paid for by one 2 KB output staging buffer per
+// epilogue warp), warp 1 MMA issuer (first CTA of the pair),
 // warps 2..9 epilogue (two warps per tensor-memory lane quadrant).
 // Epilogues:
 //   SILU_PAIR  v = acc + bias: SiLU(v) and SiLU'(v) as bf16 (recompute);
 //   DSILU      acc * SiLU'(z) read from the recompute's output, as bf16 (dz);
 //   F32        acc as fp32 (dx rows, weight gradients), or bf16 for dx rows
 //              when the group asks for it.
-// Output chunks of 32 rows x 32 columns leave through shared memory and TMA
-// bulk stores (per-thread stores of a thread's 128-byte fp32 row pieces kept
+// Output chunks of 32 rows x 32 columns (two boxes of 16 columns for fp32)
+// leave through shared memory and TMA bulk stores (per-thread stores of a thread's 128-byte fp32 row pieces kept
 // the weight-gradient kernel waiting on its store queue); rows past a
 // segment's end are stored one by one.
 // K is consumed in 16-row steps: a K-ragged segment issues only the steps
@@ -65,7 +65,7 @@ namespace {
 
 constexpr int BM = 128;                 // rows of A per CTA (M = 256 per pair)
 constexpr int BN = 256, BN_HALF = 128;  // output columns per pair tile, B rows/columns per CTA
-constexpr int BK = 64, STAGES = 5, ACC_BUFS = 2;
+constexpr int BK = 64, STAGES = 6, ACC_BUFS = 2;
 constexpr int NUM_THREADS = 320, EPI_WARPS = 8;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int MAX_SEGS = 256 + 8;
@@ -112,10 +112,9 @@ struct Smem {
     static constexpr int B_BYTES = BN_HALF * BK * 2;
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-    // per epilogue warp STG_BUFS staging buffers of one 32 x 32 output chunk
-    // (fp32: a 4 KB box in the 128-byte swizzle; bf16: 2 KB boxes in the
-    // 64-byte swizzle, two of them for the recompute's two outputs)
-    static constexpr int STG_BYTES = 4096;
+    // per epilogue warp one 2 KB staging buffer: one TMA store box of 32 rows
+    // x 64 bytes in the 64-byte swizzle (32 bf16 or 16 fp32 columns)
+    static constexpr int STG_BYTES = 2048;
     static constexpr int STG_BUFS = 1;
     static constexpr int OFF_STAGE = OFF_B + STAGES * B_BYTES;
     static constexpr int OFF_BAR = OFF_STAGE + EPI_WARPS * STG_BUFS * STG_BYTES;
@@ -430,13 +429,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
         const int half = (warp - 2) >> 2;
         const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
         // A chunk of 32 rows x 32 columns whose rows all lie in the tile's
-        // valid rows leaves through shared memory and a TMA store: the warp
-        // writes it into one of its two staging buffers (fp32 rows of 128
-        // bytes, 16-byte chunk q at q ^ (row & 7); bf16 rows of 64 bytes,
-        // chunk q at q ^ ((row >> 1) & 3): the swizzles of the boxes, which
-        // also spread the writes over the banks) and one lane stores it.  A
-        // buffer is rewritten only after the store issued from it has read
-        // it.  Other rows are stored by their threads.
+        // valid rows leaves through shared memory and TMA stores: the warp
+        // writes 32 rows of 64 bytes into its staging buffer (16-byte chunk q
+        // of a row at q ^ ((row >> 1) & 3): the box's 64-byte swizzle, which
+        // also spreads the writes over the banks) and one lane stores the
+        // box; fp32 chunks take two boxes.  The buffer is rewritten only after
+        // the store issued from it has read it.  Other rows are stored by
+        // their threads.
         uint8_t* stg = smem + L::OFF_STAGE + (warp - 2) * L::STG_BUFS * L::STG_BYTES;
         int sbuf = 0;
         auto stage_begin = [&]() -> uint8_t* {
@@ -447,15 +446,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
             __syncwarp();
             return stg + sbuf * L::STG_BYTES;
         };
-        auto stage_end = [&](const void* map0, const void* map1, int x, int y) {
+        auto stage_end = [&](const void* map, int x, int y) {
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-                tma_store_2d(map0, stg + sbuf * L::STG_BYTES, x, y);
-                if (map1) tma_store_2d(map1, stg + sbuf * L::STG_BYTES + 2048, x, y);
+                tma_store_2d(map, stg + sbuf * L::STG_BYTES, x, y);
                 bulk_commit();
             }
             if (L::STG_BUFS == 2) sbuf ^= 1;
+        };
+        // one 64-byte row of a box: 16-byte chunk q at q ^ ((row >> 1) & 3)
+        auto put_row64 = [&](uint8_t* buf, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                             uint32_t b1, uint32_t b2, uint32_t b3, uint32_t c0, uint32_t c1, uint32_t c2,
+                             uint32_t c3, uint32_t d0, uint32_t d1, uint32_t d2, uint32_t d3) {
+            uint8_t* row = buf + lane * 64;
+            const int sw = (lane >> 1) & 3;
+            *reinterpret_cast<uint4*>(row + ((0 ^ sw) << 4)) = make_uint4(a0, a1, a2, a3);
+            *reinterpret_cast<uint4*>(row + ((1 ^ sw) << 4)) = make_uint4(b0, b1, b2, b3);
+            *reinterpret_cast<uint4*>(row + ((2 ^ sw) << 4)) = make_uint4(c0, c1, c2, c3);
+            *reinterpret_cast<uint4*>(row + ((3 ^ sw) << 4)) = make_uint4(d0, d1, d2, d3);
         };
         int abuf = 0;
         uint32_t aphase = 0;
@@ -533,28 +542,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) bwd_gemm_kernel(const __grid_c
                             o0[w] = pack_bf16x2(__uint_as_float(r[u][2 * w]), __uint_as_float(r[u][2 * w + 1]));
                     }
                     if (full_rows) {
-                        uint8_t* buf = stage_begin();
+                        const int x = ti.ccol + col, y = ti.crow + r_row0;
                         if (f32_out) {
-                            uint8_t* row = buf + lane * 128;
+                            // two boxes of 16 fp32 columns
 #pragma unroll
-                            for (int q = 0; q < 8; ++q)
-                                *reinterpret_cast<uint4*>(row + ((q ^ (lane & 7)) << 4)) =
-                                    make_uint4(r[u][4 * q], r[u][4 * q + 1], r[u][4 * q + 2], r[u][4 * q + 3]);
+                            for (int hh = 0; hh < 2; ++hh) {
+                                const uint32_t* v = r[u] + 16 * hh;
+                                put_row64(stage_begin(), v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7], v[8], v[9],
+                                          v[10], v[11], v[12], v[13], v[14], v[15]);
+                                stage_end(&p.c_map[ti.grp][0], x + 16 * hh, y);
+                            }
                         } else {
-                            uint8_t* row = buf + lane * 64;
-#pragma unroll
-                            for (int q = 0; q < 4; ++q)
-                                *reinterpret_cast<uint4*>(row + ((q ^ ((lane >> 1) & 3)) << 4)) =
-                                    make_uint4(o0[4 * q], o0[4 * q + 1], o0[4 * q + 2], o0[4 * q + 3]);
+                            put_row64(stage_begin(), o0[0], o0[1], o0[2], o0[3], o0[4], o0[5], o0[6], o0[7], o0[8],
+                                      o0[9], o0[10], o0[11], o0[12], o0[13], o0[14], o0[15]);
+                            stage_end(&p.c_map[ti.grp][0], x, y);
                             if constexpr (MODE == MODE_RECOMP) {
-#pragma unroll
-                                for (int q = 0; q < 4; ++q)
-                                    *reinterpret_cast<uint4*>(row + 2048 + ((q ^ ((lane >> 1) & 3)) << 4)) =
-                                        make_uint4(o1[4 * q], o1[4 * q + 1], o1[4 * q + 2], o1[4 * q + 3]);
+                                put_row64(stage_begin(), o1[0], o1[1], o1[2], o1[3], o1[4], o1[5], o1[6], o1[7],
+                                          o1[8], o1[9], o1[10], o1[11], o1[12], o1[13], o1[14], o1[15]);
+                                stage_end(&p.c_map[ti.grp][1], x, y);
                             }
                         }
-                        stage_end(&p.c_map[ti.grp][0], MODE == MODE_RECOMP ? &p.c_map[ti.grp][1] : nullptr,
-                                  ti.ccol + col, ti.crow + r_row0);
                     } else if (f32_out) {
                         float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out0) + off);
 #pragma unroll
@@ -629,8 +636,7 @@ bool fill_group(Params& p, int gi, const BwdGemmGroup& h, bool a_mn, bool b_mn, 
     for (int o = 0; o < 2; ++o) {
         void* out = o == 0 ? h.out0 : h.out1;
         if (!out) continue;
-        const bool ok = out_f32 ? encode_tma_2d_store128(&p.c_map[gi][o], out, rows, h.ldc, 4, 32)
-                                : encode_tma_2d_store64(&p.c_map[gi][o], out, rows, h.ldc, 2, 32);
+        const bool ok = encode_tma_2d_store64(&p.c_map[gi][o], out, rows, h.ldc, out_f32 ? 4 : 2, 32);
         if (!ok) return false;
     }
     return true;

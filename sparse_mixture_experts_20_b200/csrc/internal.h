@@ -166,7 +166,6 @@ cudaError_t launch_wait_selftest(int64_t timeout_ns, int32_t* status, cudaStream
 bool encode_tma_2d(void* map, const void* base, int rows, int K, int elem, int box_rows);
 bool encode_tma_3d(void* map, const void* base, int n_mats, int N, int K, int elem, int box_rows);
 bool encode_tma_2d_store64(void* map, const void* base, int rows, int cols, int elem, int box_rows);
-bool encode_tma_2d_store128(void* map, const void* base, int rows, int cols, int elem, int box_rows);
 int device_sm_count();
 
 // Records a failed CUDA call for moe_last_cuda_error() on this thread.
