@@ -82,6 +82,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// The same test, but a thread whose phase has not completed may be suspended
+// for up to suspend_ns before the answer (it wakes when the phase completes):
+// a waiting role then spends fewer issue slots polling.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t suspend_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns) : "memory");
+    return ok != 0;
+}
+
 // Bounded wait on phase `parity` of `bar`.  Returns true when the phase
 // completed.  Returns false when *abort_flag became non-zero (another role of
 // the block gave up) or when timeout_ns elapsed; in the latter case it sets
@@ -93,7 +106,7 @@ static __device__ __noinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parit
                                                    int32_t* status, uint64_t timeout_ns) {
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, 1000u)) return true;
         if ((it & 63u) == 0) {
             if (*abort_flag) return false;
             if (global_timer_ns() - t0 > timeout_ns) {
