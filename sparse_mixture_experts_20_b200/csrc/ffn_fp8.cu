@@ -530,7 +530,9 @@ cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
 // on the V3 prefill layer (2.26 against 2.07 ms, same box): the extra tiles
 // cost more than the overlap wait they remove.  Eight epilogue warps for the
 // second layer (two per lane quadrant, 448 threads, which caps registers at
-// 128 with spills) also measured slower (2.36 against 2.23 ms, same box).
+// 128 with spills) also measured slower (2.36 against 2.23 ms, same box), and
+// 128-wide first-layer tiles for the decode batch alone (twice the tiles of
+// its 2.5 waves) gained nothing (0.325 against 0.324 ms).
 cudaError_t launch_grouped_ffn_fp8(const Dims&, const GemmArgs& a, cudaStream_t st) {
     return a.out_fp8 ? launch_bn<256, true>(a, st) : launch_bn<256, false>(a, st);
 }
