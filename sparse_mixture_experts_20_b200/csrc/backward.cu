@@ -20,7 +20,8 @@
 //   (T, n_shared * d_ff_shared) matrix, so dx and dW1 of all shared experts
 //   are one GEMM each);
 //   7. bias gradients: column sums in two fixed-order passes (16-row chunk
-//      partials, then the chunks of each segment in order);
+//      partials -- for dy made by the padding kernel as it writes dy -- then
+//      the chunks of each segment in order);
 //   8. dx = router part + shared part + the kept slots' rows (+ g * dout for
 //      slots passed through).
 // Every reduction has a fixed order: the result is bit-reproducible.
@@ -208,50 +209,73 @@ __global__ void pad_offsets_kernel(const int32_t* offsets, int E, int32_t* poff,
     if (lane == 0) poff[0] = 0;
 }
 
-// Padded rows (one warp each): x_p[pr] = x_disp[r], dy_p[pr] = g * dout[t]
-// for the rows of an expert's segment, zeros in its padding.
-__global__ void __launch_bounds__(256) pad_rows_kernel(int E, int K, int d, int rows_cap, const int32_t* offsets,
+// Padded rows in chunks of 16 (the padding unit, so a chunk lies in one
+// expert's segment): x_p[pr] = x_disp[r], dy_p[pr] = g * dout[t] (bf16) for
+// the rows of a segment, zeros in its padding, and the chunk's column sums
+// of dy_p as stored (part[ch][c], the first pass of db2).  Block = (a slab
+// of 2048 columns, a chunk); thread = 8 columns; the 16 rows' sources are
+// looked up once per chunk.
+__global__ void __launch_bounds__(256) pad_rows_kernel(int E, int K, int d, const int32_t* offsets,
                                                        const int32_t* poff, const int32_t* row_slot,
                                                        const float* gates, const __nv_bfloat16* dout,
                                                        const __nv_bfloat16* x_disp, __nv_bfloat16* x_p,
-                                                       __nv_bfloat16* dy_p) {
-    __shared__ int s_off[257], s_poff[257];
-    for (int i = threadIdx.x; i <= E; i += blockDim.x) { s_off[i] = offsets[i]; s_poff[i] = poff[i]; }
-    __syncthreads();
-    const int total = s_poff[E];
-    const int lane = threadIdx.x & 31;
-    const int warps = gridDim.x * (blockDim.x >> 5);
-    for (int pr = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); pr < total && pr < rows_cap; pr += warps) {
-        int lo = 0, hi = E - 1;                         // last e with poff[e] <= pr
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (s_poff[mid] <= pr) lo = mid; else hi = mid - 1;
-        }
-        const int e = lo, i = pr - s_poff[e];
-        uint4* xo = reinterpret_cast<uint4*>(x_p + static_cast<size_t>(pr) * d);
-        uint4* yo = reinterpret_cast<uint4*>(dy_p + static_cast<size_t>(pr) * d);
-        if (i < s_off[e + 1] - s_off[e]) {
-            const int r = s_off[e] + i;
-            const int slot = row_slot[r];
-            const float g = gates[slot];
-            const uint4* xi = reinterpret_cast<const uint4*>(x_disp + static_cast<size_t>(r) * d);
-            const uint4* di = reinterpret_cast<const uint4*>(dout + static_cast<size_t>(slot / K) * d);
-            for (int c = lane; c < d / 8; c += 32) {
-                xo[c] = xi[c];
-                uint4 v = di[c];
-                uint32_t* w = reinterpret_cast<uint32_t*>(&v);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
-                    __nv_bfloat162 o = __floats2bfloat162_rn(g * f.x, g * f.y);
-                    w[j] = *reinterpret_cast<uint32_t*>(&o);
-                }
-                yo[c] = v;
+                                                       __nv_bfloat16* dy_p, float* part) {
+    __shared__ int s_r[16], s_t[16];
+    __shared__ float s_g[16];
+    const int total = poff[E];
+    const int c = 8 * (blockIdx.x * blockDim.x + threadIdx.x);
+    for (int ch = blockIdx.y; ch * 16 < total; ch += gridDim.y) {
+        if (threadIdx.x < 16) {
+            const int pr = ch * 16 + threadIdx.x;
+            int lo = 0, hi = E - 1;                     // last e with poff[e] <= pr
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (poff[mid] <= pr) lo = mid; else hi = mid - 1;
             }
-        } else {
-            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-            for (int c = lane; c < d / 8; c += 32) { xo[c] = z; yo[c] = z; }
+            const int i = pr - poff[lo];
+            int r = -1, t = 0;
+            float g = 0.f;
+            if (i < offsets[lo + 1] - offsets[lo]) {
+                r = offsets[lo] + i;
+                const int slot = row_slot[r];
+                t = slot / K;
+                g = gates[slot];
+            }
+            s_r[threadIdx.x] = r;
+            s_t[threadIdx.x] = t;
+            s_g[threadIdx.x] = g;
         }
+        __syncthreads();
+        if (c < d) {
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+            for (int i = 0; i < 16; ++i) {
+                const size_t pr = static_cast<size_t>(ch) * 16 + i;
+                const int r = s_r[i];
+                uint4 xv = make_uint4(0u, 0u, 0u, 0u), yv = make_uint4(0u, 0u, 0u, 0u);
+                if (r >= 0) {
+                    xv = *reinterpret_cast<const uint4*>(x_disp + static_cast<size_t>(r) * d + c);
+                    yv = *reinterpret_cast<const uint4*>(dout + static_cast<size_t>(s_t[i]) * d + c);
+                    const float g = s_g[i];
+                    uint32_t* w = reinterpret_cast<uint32_t*>(&yv);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[j]));
+                        const __nv_bfloat162 o = __floats2bfloat162_rn(g * f.x, g * f.y);
+                        const float2 q = __bfloat1622float2(o);
+                        acc[2 * j] += q.x;
+                        acc[2 * j + 1] += q.y;
+                        w[j] = *reinterpret_cast<const uint32_t*>(&o);
+                    }
+                }
+                *reinterpret_cast<uint4*>(x_p + pr * d + c) = xv;
+                *reinterpret_cast<uint4*>(dy_p + pr * d + c) = yv;
+            }
+            float4* po = reinterpret_cast<float4*>(part + static_cast<size_t>(ch) * d + c);
+            po[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            po[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        }
+        __syncthreads();
     }
 }
 
@@ -278,19 +302,32 @@ __global__ void __launch_bounds__(256) colsum_chunks_kernel(const __nv_bfloat16*
 
 // out[copy * copy_stride + s * ncols + c] = sum over the chunks of segment s
 // of part[ch][c], in chunk order.  Segment s spans rows seg[s] .. seg[s+1]-1
-// (multiples of CH) or, with seg == nullptr, rows 0 .. fixed_rows-1.
+// (multiples of CH) or, with seg == nullptr, rows 0 .. fixed_rows-1.  Block =
+// (32 columns, a segment): warp w sums the w-th of 8 contiguous runs of the
+// segment's chunks (lane = column), then the 8 run sums are added in run order.
 template <int CH>
 __global__ void __launch_bounds__(256) colsum_segments_kernel(const float* part, int ncols, const int32_t* seg,
                                                               int nseg, int fixed_rows, float* out, int copies,
                                                               int copy_stride) {
-    const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (i >= static_cast<size_t>(nseg) * ncols) return;
-    const int s = static_cast<int>(i / ncols), c = static_cast<int>(i % ncols);
+    __shared__ float sm[8][32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int s = blockIdx.y, c = blockIdx.x * 32 + lane;
     const int ch0 = seg ? seg[s] / CH : 0;
     const int ch1 = seg ? seg[s + 1] / CH : (fixed_rows + CH - 1) / CH;
+    const int per = (ch1 - ch0 + 7) / 8;
+    const int a = ch0 + warp * per, b = min(ch1, a + per);
     float acc = 0.f;
-    for (int ch = ch0; ch < ch1; ++ch) acc += part[static_cast<size_t>(ch) * ncols + c];
-    for (int k = 0; k < copies; ++k) out[static_cast<size_t>(k) * copy_stride + i] = acc;
+    if (c < ncols)
+        for (int ch = a; ch < b; ++ch) acc += part[static_cast<size_t>(ch) * ncols + c];
+    sm[warp][lane] = acc;
+    __syncthreads();
+    if (warp == 0 && c < ncols) {
+        float t = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) t += sm[w][lane];
+        for (int k = 0; k < copies; ++k) out[static_cast<size_t>(k) * copy_stride + static_cast<size_t>(s) * ncols + c] = t;
+    }
+    (void)nseg;
 }
 
 // dx[t][c] = dx_router[t][c] + dx_shared[t][c] + sum_k (kept: the bf16 dx
@@ -367,7 +404,7 @@ struct TcLayout {
 constexpr int kRouterSplitTiles = 296;
 
 constexpr int kChunkRouted = 16;    // row chunk of the routed column sums (the padding unit)
-constexpr int kChunkShared = 128;
+constexpr int kChunkShared = 16;     // row chunk of the token-wide column sums
 
 TcLayout tc_layout(const Dims& dm) {
     TcLayout L{};
@@ -499,8 +536,8 @@ cudaError_t run_backward_bf16(const Dims& dm, float lam, const moe_backward_io& 
             colsum_chunks_f32_kernel<kChunkShared><<<dim3((E + 255) / 256, std::min(nch, 65535)), 256, 0, st>>>(
                 dl, E, T, part);
             check(cudaGetLastError());
-            colsum_segments_kernel<kChunkShared><<<(E + 255) / 256, 256, 0, st>>>(part, E, nullptr, 1, T,
-                                                                                 io.d_logit_bias, 1, 0);
+            colsum_segments_kernel<kChunkShared><<<dim3((E + 31) / 32, 1), 256, 0, st>>>(part, E, nullptr, 1, T,
+                                                                                     io.d_logit_bias, 1, 0);
             check(cudaGetLastError());
             ex.launches += 2;
         } else {
@@ -522,13 +559,16 @@ cudaError_t run_backward_bf16(const Dims& dm, float lam, const moe_backward_io& 
     }
     if (ex.err != cudaSuccess) { launches = ex.launches; return ex.err; }
 
-    // padded routed rows
+    // padded routed rows, with the 16-row column partials of dy_p; db2
     {
-        const int blocks = std::min((Rp + 7) / 8, sms * 8);
-        pad_rows_kernel<<<blocks, 256, 0, st>>>(E, K, d, Rp, io.offsets, poff, io.row_slot, io.gates, dout,
-                                                static_cast<const bf*>(io.x_disp), x_p, dy_p);
+        const dim3 grid((d + 2047) / 2048, std::min(Rp / kChunkRouted, 65535));
+        pad_rows_kernel<<<grid, 256, 0, st>>>(E, K, d, io.offsets, poff, io.row_slot, io.gates, dout,
+                                              static_cast<const bf*>(io.x_disp), x_p, dy_p, part);
         check(cudaGetLastError());
-        ++ex.launches;
+        colsum_segments_kernel<kChunkRouted><<<dim3((d + 31) / 32, E), 256, 0, st>>>(part, d, poff, E, 0, io.db2,
+                                                                                    1, 0);
+        check(cudaGetLastError());
+        ex.launches += 2;
     }
     // 3. recompute: SiLU(z), SiLU'(z)
     {
@@ -637,9 +677,8 @@ cudaError_t run_backward_bf16(const Dims& dm, float lam, const moe_backward_io& 
         const dim3 g1((ncols / 2 + 255) / 256, std::min(Rp / kChunkRouted, 65535));
         colsum_chunks_kernel<kChunkRouted><<<g1, 256, 0, st>>>(M, ncols, ncols, poff + E, 0, part);
         check(cudaGetLastError());
-        const size_t n = static_cast<size_t>(E) * ncols;
-        colsum_segments_kernel<kChunkRouted><<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
-            part, ncols, poff, E, 0, out, 1, 0);
+        colsum_segments_kernel<kChunkRouted><<<dim3((ncols + 31) / 32, E), 256, 0, st>>>(part, ncols, poff, E,
+                                                                                        0, out, 1, 0);
         check(cudaGetLastError());
         ex.launches += 2;
     };
@@ -647,12 +686,11 @@ cudaError_t run_backward_bf16(const Dims& dm, float lam, const moe_backward_io& 
         const dim3 g1((ncols / 2 + 255) / 256, std::min((T + kChunkShared - 1) / kChunkShared, 65535));
         colsum_chunks_kernel<kChunkShared><<<g1, 256, 0, st>>>(M, ncols, ncols, nullptr, T, part);
         check(cudaGetLastError());
-        colsum_segments_kernel<kChunkShared><<<static_cast<unsigned>((ncols + 255) / 256), 256, 0, st>>>(
-            part, ncols, nullptr, 1, T, out, copies, copy_stride);
+        colsum_segments_kernel<kChunkShared><<<dim3((ncols + 31) / 32, 1), 256, 0, st>>>(part, ncols, nullptr, 1,
+                                                                                        T, out, copies, copy_stride);
         check(cudaGetLastError());
         ex.launches += 2;
     };
-    colsum_routed(dy_p, d, io.db2);
     colsum_routed(dz_p, dff, io.db1);
     if (S > 0) {
         colsum_shared(dout, d, io.dbs2, S, d);

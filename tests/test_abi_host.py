@@ -165,7 +165,7 @@ def _bwd_tc_layout_bytes(T, d, E, K, dff, S, dffs, r_cap):
     expert (r_cap + 15 N_r, rounded to 16): bf16 x, dy, SiLU(z), SiLU'(z), dz
     and dx rows; shared bf16 SiLU(z), SiLU'(z), dz of width n_shared *
     d_ff_shared and fp32 dx; fp32 column-sum partials (16-row chunks of the
-    routed rows, 128-row chunks of the tokens)."""
+    routed rows and of the tokens)."""
     rp = (r_cap + 15 * E + 15) // 16 * 16
     sw = S * dffs
     epad = (E + 7) // 8 * 8
@@ -174,7 +174,7 @@ def _bwd_tc_layout_bytes(T, d, E, K, dff, S, dffs, r_cap):
     splits = max(splits, 1)
     chunk = (-(-T // splits) + 15) // 16 * 16
     splits = -(-T // chunk)
-    nch = (T + 127) // 128
+    nch = (T + 15) // 16
     part = max((rp // 16) * max(d, dff), nch * max(d, sw), nch * E)
     regions = [256, T * K * 4, T * E * 4, T * epad * 2, E * d * 2, splits * E * d * 4 if splits > 1 else 0,
                T * d * 4, (E + 1) * 4,
