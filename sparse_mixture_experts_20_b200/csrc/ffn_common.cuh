@@ -45,6 +45,7 @@ struct __align__(64) TcParams {
     GroupDev g[2];
     int silu;
     int out_fp8;
+    int sf_vec;               // FP8: scales read as float4 over four k-blocks
     int32_t* status;
     uint64_t timeout_ns;
 };
