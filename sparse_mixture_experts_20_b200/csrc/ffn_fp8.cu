@@ -620,7 +620,10 @@ cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
 // second layer (two per lane quadrant, 448 threads, which caps registers at
 // 128 with spills) also measured slower (2.36 against 2.23 ms, same box), and
 // 128-wide first-layer tiles for the decode batch alone (twice the tiles of
-// its 2.5 waves) gained nothing (0.325 against 0.324 ms).
+// its 2.5 waves) gained nothing (0.325 against 0.324 ms).  An L2 prefetch
+// (cp.async.bulk.prefetch.tensor) of the A and B boxes 4, 8 or 16 items ahead
+// of the ring's loads made the V3 prefill layer slower, the more so the
+// further ahead (2.05 against 2.71, 2.85 and 3.17 ms, same box).
 cudaError_t launch_grouped_ffn_fp8(const Dims&, const GemmArgs& a, cudaStream_t st) {
     return a.out_fp8 ? launch_bn<256, true>(a, st) : launch_bn<256, false>(a, st);
 }
