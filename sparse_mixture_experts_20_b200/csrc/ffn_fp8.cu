@@ -623,7 +623,11 @@ cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
 // its 2.5 waves) gained nothing (0.325 against 0.324 ms).  An L2 prefetch
 // (cp.async.bulk.prefetch.tensor) of the A and B boxes 4, 8 or 16 items ahead
 // of the ring's loads made the V3 prefill layer slower, the more so the
-// further ahead (2.05 against 2.71, 2.85 and 3.17 ms, same box).
+// further ahead (2.05 against 2.71, 2.85 and 3.17 ms, same box).  Separate
+// rings for A (2 stages, loaded by a scale-factor warp after the same wait
+// as its scale slot) and B (5 stages: 128 KB of weights in flight instead of
+// 96) passed parity but measured slower (2.39 against 2.02 ms; with 4 + 4
+// stages 2.10): the A tile then reaches the MMA too late.
 cudaError_t launch_grouped_ffn_fp8(const Dims&, const GemmArgs& a, cudaStream_t st) {
     return a.out_fp8 ? launch_bn<256, true>(a, st) : launch_bn<256, false>(a, st);
 }
