@@ -107,6 +107,33 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def probe_fp8_peak(dev, n=8192, iters=10):
+    """Dense FP8 tensor throughput of this GPU, measured once with a library
+    GEMM (torch._scaled_mm, e4m3 x e4m3 -> bf16, n^3): a denominator probe for
+    the FP8 expert GEMMs' tensor fraction, never on the measured path.
+    Returns TFLOP/s, or None where the library call is unavailable."""
+    import torch
+    try:
+        g = torch.Generator(device=dev).manual_seed(1)
+        a = torch.randn((n, n), device=dev, generator=g).to(torch.float8_e4m3fn)
+        b = torch.randn((n, n), device=dev, generator=g).to(torch.float8_e4m3fn).t()
+        one = torch.ones((), device=dev, dtype=torch.float32)
+        for _ in range(3):
+            torch._scaled_mm(a, b, one, one, out_dtype=torch.bfloat16)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record()
+        for _ in range(iters):
+            torch._scaled_mm(a, b, one, one, out_dtype=torch.bfloat16)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / iters
+        del a, b
+        return round(2.0 * n ** 3 / (ms * 1e-3) / 1e12, 1)
+    except Exception:   # a probe: its absence leaves the field null
+        return None
+
+
 def max_over_ranks(ms, world, device=None):
     """The largest of the ranks' times (every rank returns it); the job is as
     slow as its slowest replica.  Works on the nccl (CUDA tensor) and gloo
@@ -658,6 +685,13 @@ def ffn_roofline(sh, flops, fbytes, touched, ffn_ms, peaks, peak_src):
         if sus:
             sus = sus * (2.0 if fp8 else 1.0)
             roof["frac_of_sustained_peak"] = round(roof["achieved"] / sus, 4)
+    if fp8:
+        # the tensor side of the HBM-bound FP8 GEMMs, against a library FP8
+        # GEMM's dense throughput measured on this GPU in the same run
+        tfl = flops / (ffn_ms * 1e-3) / 1e12
+        roof["tensor_tflops"] = round(tfl, 1)
+        probe = peaks.get("fp8_tflops_probe")
+        roof["tensor_frac_of_fp8_probe"] = round(tfl / probe, 4) if probe else None
     roof["algorithmic"] = {"flops": flops, "bytes": fbytes, "experts_touched": touched}
     return roof
 
@@ -681,6 +715,7 @@ def run_ours(args):
     torch.cuda.set_device(dev)
     M.lib()
     peaks, peak_src = load_peaks()
+    peaks["fp8_tflops_probe"] = probe_fp8_peak(dev)
     head = measure_workload(args, args.config, workload(args), dev, world, rank, local, peaks, peak_src,
                             cpu_baseline=not args.no_cpu_baseline)
     nested = {}
@@ -699,7 +734,9 @@ def run_ours(args):
                   "routing", "device_status", "clocks", "cpu_baseline", "backward"):
             if k in head:
                 line[k] = head[k]
-        line["peaks"] = {"source": peak_src, "hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"]}
+        line["peaks"] = {"source": peak_src, "hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"],
+                         "fp8_tflops_probe": peaks["fp8_tflops_probe"],
+                         "fp8_probe": "torch._scaled_mm e4m3 8192^3 -> bf16, 10 calls after 3, CUDA events"}
         if nested:
             line["workloads"] = nested
         print(json.dumps(line), flush=True)
