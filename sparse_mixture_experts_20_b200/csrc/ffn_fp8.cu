@@ -627,11 +627,7 @@ cudaError_t launch_bn(const GemmArgs& a, cudaStream_t st) {
 // rings for A (2 stages, loaded by a scale-factor warp after the same wait
 // as its scale slot) and B (5 stages: 128 KB of weights in flight instead of
 // 96) passed parity but measured slower (2.39 against 2.02 ms; with 4 + 4
-// stages 2.10): the A tile then reaches the MMA too late.  Stages of 64
-// bytes of K (eight of 24 KB, 112 KB of weights in flight, 64-byte swizzle,
-// a separate ring of scale slots) passed parity but measured slower too
-// (2.53 against 2.10 ms): the per-stage wait, fence and commit of the MMA
-// thread then come twice per 128 columns of K.
+// stages 2.10): the A tile then reaches the MMA too late.
 cudaError_t launch_grouped_ffn_fp8(const Dims&, const GemmArgs& a, cudaStream_t st) {
     return a.out_fp8 ? launch_bn<256, true>(a, st) : launch_bn<256, false>(a, st);
 }
