@@ -107,6 +107,32 @@ struct ItemIt {
     TileInfo ti;
 };
 
+// The MMA thread's wait for a full stage, bounded like mbar_wait_bounded but
+// polling without the suspend hint: this thread is on the critical path, and
+// the hinted poll (which the waiting roles keep) measured 0.5-0.8 % slower
+// for the whole layer on the V3 prefill and decode batches.
+static __device__ __noinline__ bool mma_wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                  int32_t* status, uint64_t timeout_ns) {
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > timeout_ns) {
+                *abort_flag = 1;
+                set_device_status(status, MOE_DEV_TIMEOUT);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ bool mma_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int32_t* status,
+                                         uint64_t timeout_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return mma_wait_spin(bar, parity, abort_flag, status, timeout_ns);
+}
+
 // OUT_FP8: the first layer (bias, SiLU, e4m3 re-quantisation of h) or the
 // second (bias, bf16 y); one instance each, so that neither carries the
 // other's registers and code.
@@ -203,7 +229,7 @@ grouped_ffn_fp8_kernel(const __grid_constant__ TcParams p) {
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (abuf ? L::ACC1_COL : 0u);
                 for (int kb = 0; kb < ti.kblocks; ++kb) {
-                    if (!mbar_wait_bounded(&full[stage], phase, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
+                    if (!mma_wait(&full[stage], phase, abort_flag, p.status, p.timeout_ns)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t adesc = smem_desc_k_sw128(smem + L::OFF_A + stage * L::A_BYTES);
                     const uint64_t bdesc = smem_desc_k_sw128(smem + L::OFF_B + stage * L::B_BYTES);
