@@ -49,6 +49,9 @@ CASES = {
     # d_ff two tiles and a half, pass-through on
     "bf16-long-segments": MoEShape("k8", 1100, 256, 4, 2, 576, capacity_factor=0.9, dtype=DTYPE_BF16,
                                    overflow_mode=1),
+    # d_model = 320 (K and N tails of 64 in every GEMM that spans d), a
+    # shared expert
+    "bf16-d320-shared": MoEShape("k9", 200, 320, 8, 2, 192, n_shared=1, d_ff_shared=128, dtype=DTYPE_BF16),
 }
 
 

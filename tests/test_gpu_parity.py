@@ -51,6 +51,14 @@ CASES = {
     "bf16-k16-e256": MoEShape("m1", 200, 256, 256, 16, 128, dtype=DTYPE_BF16),
     "bf16-8-shared": MoEShape("m2", 96, 128, 8, 2, 128, n_shared=8, d_ff_shared=64, dtype=DTYPE_BF16),
     "fp8-one-token": MoEShape("m3", 1, 256, 16, 4, 256, n_shared=1, d_ff_shared=128, dtype=DTYPE_FP8),
+    # d_model not a multiple of 128 (bf16 and fp32 take multiples of 64): a
+    # K tail in the first layer and the router, an N tail of 64 columns in
+    # the second, rows of 640 / 384 bytes in the dispatch copy and combine;
+    # on the small, tensor-core and generic routers
+    "bf16-d320-shared-cap": MoEShape("t1", 333, 320, 8, 2, 192, n_shared=1, d_ff_shared=128,
+                                     capacity_factor=1.1, dtype=DTYPE_BF16),
+    "bf16-d192-tc-router": MoEShape("t2", 300, 192, 64, 4, 256, dtype=DTYPE_BF16),
+    "f32-d192-generic-router": MoEShape("t3", 150, 192, 40, 2, 192, dtype=DTYPE_F32),
     # capacity variants: slot-major priority, overflow pass-through, both
     "bf16-slotmajor-cap": MoEShape("c1", 300, 256, 8, 2, 256, capacity_factor=0.8, dtype=DTYPE_BF16,
                                    capacity_priority=1),
