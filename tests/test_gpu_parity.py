@@ -59,6 +59,10 @@ CASES = {
                                      capacity_factor=1.1, dtype=DTYPE_BF16),
     "bf16-d192-tc-router": MoEShape("t2", 300, 192, 64, 4, 256, dtype=DTYPE_BF16),
     "f32-d192-generic-router": MoEShape("t3", 150, 192, 40, 2, 192, dtype=DTYPE_F32),
+    # top-1 routing over many experts (one slot per token), with a capacity
+    # that drops and with FP8
+    "bf16-top1-cap": MoEShape("u1", 500, 256, 16, 1, 256, capacity_factor=1.0, dtype=DTYPE_BF16),
+    "fp8-top1-shared": MoEShape("u2", 300, 512, 32, 1, 256, n_shared=1, d_ff_shared=256, dtype=DTYPE_FP8),
     # capacity variants: slot-major priority, overflow pass-through, both
     "bf16-slotmajor-cap": MoEShape("c1", 300, 256, 8, 2, 256, capacity_factor=0.8, dtype=DTYPE_BF16,
                                    capacity_priority=1),
